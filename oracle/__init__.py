@@ -1,0 +1,163 @@
+"""CPU oracle for the fused int8 GroupedMatmul + MoeFinalizeRouting op.
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+benchmark's ``cpu_baseline`` / reference leg may import this package.  It shares
+no code with the CUDA library and never imports it.
+
+The arithmetic lives in ``qgmm_oracle.c`` (plain C, IEEE float, no FMA
+contraction); this module only marshals numpy arrays.  Function-by-function
+citations are in the C file's header.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional
+
+import numpy as np
+
+from .build import build as _build
+
+QO_OK = 0
+QO_ERR_NEGATIVE_COUNT = 1
+QO_ERR_NOT_MONOTONE = 2
+QO_ERR_TOTAL_GT_M = 3
+QO_ERR_BAD_ROW_INDEX = 4
+QO_ERR_ACC_OVERFLOW = 5
+QO_ERR_ARG = 6
+
+
+class OracleError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"oracle {what}: code {code}")
+        self.code = code
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build()
+        L = C.CDLL(path)
+        P, I64, I32 = C.c_void_p, C.c_int64, C.c_int
+        L.qo_group_offsets.argtypes = [P, I64, I32, I64, P]
+        L.qo_accum.argtypes = [P, P, I32, I64, I64, I64, I64, P, I32, P, I64, P, I32]
+        L.qo_finalize.argtypes = [P, P, I32, I64, I64, I64, I64, P, I32, P, P, P, P, P, I32,
+                                  P, I64, I64, I64, P, I64, P, P, P, I32]
+        L.qo_per_token_quant.argtypes = [P, I64, I64, P, P]
+        for f in (L.qo_group_offsets, L.qo_accum, L.qo_finalize, L.qo_per_token_quant):
+            f.restype = C.c_int
+        _lib = L
+    return _lib
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else C.c_void_p(a.ctypes.data)
+
+
+def _c(a: Optional[np.ndarray], dtype) -> Optional[np.ndarray]:
+    return None if a is None else np.ascontiguousarray(a, dtype=dtype)
+
+
+def group_offsets(group_list: np.ndarray, group_list_type: int, m: int) -> np.ndarray:
+    gl = _c(group_list, np.int64)
+    off = np.zeros(gl.shape[0] + 1, np.int64)
+    rc = lib().qo_group_offsets(_ptr(gl), gl.shape[0], group_list_type, m, _ptr(off))
+    if rc:
+        raise OracleError(rc, "group_offsets")
+    return off
+
+
+def _weights(x2: np.ndarray, weight: str):
+    if weight == "int8":
+        return _c(x2, np.int8), 0
+    return _c(x2, np.int32), 1
+
+
+def accum(x1, x2, group_list, group_list_type: int, weight: str = "int8",
+          rows: Optional[np.ndarray] = None, threads: Optional[int] = None) -> np.ndarray:
+    """Exact int32 accumulators ``x1[i] @ W[g(i)]`` for source rows ``rows`` (default all)."""
+    x1 = _c(x1, np.int8)
+    w, wt = _weights(x2, weight)
+    m, k = x1.shape
+    e = w.shape[0]
+    n = w.shape[2] * (8 if wt else 1)
+    r = _c(rows, np.int64)
+    nrows = m if r is None else r.shape[0]
+    out = np.zeros((nrows, n), np.int32)
+    rc = lib().qo_accum(_ptr(x1), _ptr(w), wt, m, k, n, e, _ptr(_c(group_list, np.int64)),
+                        group_list_type, _ptr(r), nrows, _ptr(out), threads or default_threads())
+    if rc:
+        raise OracleError(rc, "accum")
+    return out
+
+
+def finalize(x1, x2, group_list, group_list_type: int, *, weight: str = "int8",
+             scale=None, pertoken_scale=None, logit=None, bias=None, row_index=None,
+             shared=None, shared_offset: int = 0, output_bs: Optional[int] = None,
+             dest_rows: Optional[np.ndarray] = None, want64: bool = True, want32: bool = True,
+             threads: Optional[int] = None):
+    """The op's output rows ``dest_rows`` (default all ``output_bs`` rows).
+
+    Returns ``(out64, sabs64, out32)``: double value, double sum of |terms| per
+    element, and the f32 value in the fixed summation order (None if not asked).
+    """
+    x1 = _c(x1, np.int8)
+    w, wt = _weights(x2, weight)
+    m, k = x1.shape
+    e = w.shape[0]
+    n = w.shape[2] * (8 if wt else 1)
+    if output_bs is None:
+        output_bs = m
+    ri = None
+    rit = 0
+    if row_index is not None:
+        if row_index.dtype == np.int32:
+            ri, rit = _c(row_index, np.int32), 1
+        else:
+            ri, rit = _c(row_index, np.int64), 0
+    sh = _c(shared, np.uint16)
+    shared_bs = 0 if sh is None else sh.shape[0]
+    d = _c(dest_rows, np.int64)
+    nd = output_bs if d is None else d.shape[0]
+    out64 = np.zeros((nd, n), np.float64) if want64 else None
+    sabs = np.zeros((nd, n), np.float64) if want64 else None
+    out32 = np.zeros((nd, n), np.float32) if want32 else None
+    rc = lib().qo_finalize(_ptr(x1), _ptr(w), wt, m, k, n, e, _ptr(_c(group_list, np.int64)),
+                           group_list_type, _ptr(_c(scale, np.float32)),
+                           _ptr(_c(pertoken_scale, np.float32)), _ptr(_c(logit, np.float32)),
+                           _ptr(_c(bias, np.float32)), _ptr(ri), rit, _ptr(sh), shared_bs,
+                           shared_offset, output_bs, _ptr(d), nd, _ptr(out64), _ptr(sabs),
+                           _ptr(out32), threads or default_threads())
+    if rc:
+        raise OracleError(rc, "finalize")
+    return out64, sabs, out32
+
+
+def per_token_quant(x_bf16: np.ndarray):
+    """bf16 bits [rows, k] -> (int8 [rows, k], f32 pts [rows])."""
+    x = _c(x_bf16, np.uint16)
+    rows, k = x.shape
+    q = np.zeros((rows, k), np.int8)
+    pts = np.zeros(rows, np.float32)
+    rc = lib().qo_per_token_quant(_ptr(x), rows, k, _ptr(q), _ptr(pts))
+    if rc:
+        raise OracleError(rc, "per_token_quant")
+    return q, pts
+
+
+def problem_finalize(p, *, x1=None, pertoken_scale=None, dest_rows=None, want64=True,
+                     want32=True, threads=None):
+    """Run ``finalize`` on a ``synth.Problem`` (x1/pts override for prologue workloads)."""
+    return finalize(p.x1 if x1 is None else x1, p.x2, p.group_list, p.group_list_type,
+                    weight=p.weight, scale=p.scale,
+                    pertoken_scale=p.pertoken_scale if pertoken_scale is None else pertoken_scale,
+                    logit=p.logit, bias=p.bias, row_index=p.row_index, shared=p.shared,
+                    shared_offset=p.shared_offset, output_bs=p.output_bs, dest_rows=dest_rows,
+                    want64=want64, want32=want32, threads=threads)

@@ -1,0 +1,327 @@
+/*
+ * qgmm_oracle.c -- plain CPU oracle for the fused int8 GroupedMatmul +
+ * MoeFinalizeRouting op.  TEST INFRASTRUCTURE ONLY: the tests, the package's
+ * smoke check and the benchmark's CPU-baseline leg call it; the product path
+ * never does.  It shares no code with the CUDA library.
+ *
+ * What it follows (pages as printed, by title and section):
+ *  - "aclnnGroupedMatmulFinalizeRoutingWeightNzV2", function description: a
+ *    grouped matmul whose output rows are combined into the output by index;
+ *    parameter constraints: groupList type 0 is non-negative and monotone
+ *    non-decreasing (cumulative ends), type 1 is non-negative (per-group
+ *    counts); x2 is (e, k, n), or int32 (e, k, n/8) holding int4 values;
+ *    scale is (e, 1, n); pertokenScale is (m); sharedInput rows land at
+ *    sharedInputOffset with offset + bsdp <= outputBS; optional inputs may be
+ *    absent.
+ *  - "matmul支持pertoken量化模式", 计算示例: out[i][j] = (sum_k x[i][k] w[k][j])
+ *    * deqScale[j] * perTokenScale[i], int8 inputs, exact integer products.
+ *  - PTOAS issue 1568 (per_token_cast), 背景: the quantised value is the input
+ *    multiplied by a precomputed inverse scale.
+ *
+ * Readings where the pages are silent (each listed in the design notes):
+ *  - bias is added after the two dequant scales and before the routing weight:
+ *    y = ((acc * scale[g][j]) * pts[i] + bias[g][j]) * logit[i];
+ *  - sharedInput is added unweighted; rows outside its range start at 0;
+ *  - rows at or past the groups' total are ignored;
+ *  - the combine sums, per output element, the shared value first and then the
+ *    contributions in ascending source row order;
+ *  - int4: the lowest nibble of each int32 word is the lowest n index, two's
+ *    complement (values -8..7);
+ *  - per-token quant: a = max |x|, pts = a/127, inv = 127/a (0 for a zero row),
+ *    q = round-half-even(x * inv) clamped to [-127, 127].
+ *
+ * Precision: integer accumulation is exact (int64, checked to fit int32).
+ * Two float forms of the dequant+combine are provided:
+ *  - qo_finalize_f64: every step in double -- the value the op approximates;
+ *  - qo_finalize_f32: every step in IEEE single precision in the order above
+ *    (compiled with -ffp-contract=off, no fast-math) -- what an f32 device
+ *    computes when it keeps that order.
+ * The per-token quant decides integers from floats, so it runs in f32.
+ *
+ * Parallelism: independent destination rows are split across POSIX threads;
+ * each element's arithmetic is the same as in the single-threaded loop.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum {
+    QO_OK = 0,
+    QO_ERR_NEGATIVE_COUNT = 1,
+    QO_ERR_NOT_MONOTONE = 2,
+    QO_ERR_TOTAL_GT_M = 3,
+    QO_ERR_BAD_ROW_INDEX = 4,
+    QO_ERR_ACC_OVERFLOW = 5,
+    QO_ERR_ARG = 6,
+};
+
+/* ---- groupList -> row offsets (parameter constraints of page 1) -------- */
+int qo_group_offsets(const int64_t *group_list, int64_t e, int group_list_type,
+                     int64_t m, int64_t *off /* [e+1] */)
+{
+    if (!group_list || !off || e < 1) return QO_ERR_ARG;
+    off[0] = 0;
+    for (int64_t g = 0; g < e; ++g) {
+        int64_t v = group_list[g];
+        if (v < 0) return QO_ERR_NEGATIVE_COUNT;
+        if (group_list_type == 0) {
+            if (v < off[g]) return QO_ERR_NOT_MONOTONE;
+            off[g + 1] = v;
+        } else if (group_list_type == 1) {
+            off[g + 1] = off[g] + v;
+        } else {
+            return QO_ERR_ARG;
+        }
+    }
+    if (off[e] > m) return QO_ERR_TOTAL_GT_M;
+    return QO_OK;
+}
+
+/* weight value W(g, kk, j) of the int8 or the int32-packed int4 layout */
+static inline int32_t weight_at(const void *x2, int weight_type, int64_t k, int64_t n,
+                                int64_t g, int64_t kk, int64_t j)
+{
+    if (weight_type == 0) {
+        const int8_t *w = (const int8_t *)x2;
+        return (int32_t)w[(g * k + kk) * n + j];
+    } else {
+        const int32_t *w = (const int32_t *)x2;
+        uint32_t word = (uint32_t)w[(g * k + kk) * (n / 8) + j / 8];
+        int32_t nib = (int32_t)((word >> (4 * (j % 8))) & 0xFu);
+        return nib >= 8 ? nib - 16 : nib;
+    }
+}
+
+static int64_t group_of_row(const int64_t *off, int64_t e, int64_t i)
+{
+    for (int64_t g = 0; g < e; ++g)
+        if (i >= off[g] && i < off[g + 1]) return g;
+    return -1;
+}
+
+/* acc[j] = sum_kk x1[i][kk] * W(g, kk, j), exact; returns 0 or overflow code */
+static int accum_row(const int8_t *x1, const void *x2, int weight_type, int64_t k, int64_t n,
+                     int64_t g, int64_t i, int64_t *acc64 /* [n] scratch */, int32_t *acc)
+{
+    for (int64_t j = 0; j < n; ++j) acc64[j] = 0;
+    for (int64_t kk = 0; kk < k; ++kk) {
+        int64_t a = (int64_t)x1[i * k + kk];
+        if (a == 0) continue;
+        if (weight_type == 0) {
+            const int8_t *wrow = (const int8_t *)x2 + (g * k + kk) * n;
+            for (int64_t j = 0; j < n; ++j) acc64[j] += a * (int64_t)wrow[j];
+        } else {
+            for (int64_t j = 0; j < n; ++j) acc64[j] += a * (int64_t)weight_at(x2, 1, k, n, g, kk, j);
+        }
+    }
+    int rc = QO_OK;
+    for (int64_t j = 0; j < n; ++j) {
+        if (acc64[j] > INT32_MAX || acc64[j] < INT32_MIN) rc = QO_ERR_ACC_OVERFLOW;
+        acc[j] = (int32_t)acc64[j];
+    }
+    return rc;
+}
+
+/* ---- parallel-for over a list of items ---------------------------------- */
+typedef struct {
+    void (*fn)(void *ctx, int64_t item, int64_t *s64, int32_t *s32, int *rc);
+    void *ctx;
+    int64_t nitems, n;
+    int nthreads, tid;
+    int rc;
+} job_t;
+
+static void *job_main(void *p)
+{
+    job_t *j = (job_t *)p;
+    int64_t *s64 = (int64_t *)malloc(sizeof(int64_t) * (size_t)j->n);
+    int32_t *s32 = (int32_t *)malloc(sizeof(int32_t) * (size_t)j->n);
+    if (!s64 || !s32) { j->rc = QO_ERR_ARG; free(s64); free(s32); return NULL; }
+    for (int64_t it = j->tid; it < j->nitems; it += j->nthreads) j->fn(j->ctx, it, s64, s32, &j->rc);
+    free(s64);
+    free(s32);
+    return NULL;
+}
+
+static int run_parallel(void (*fn)(void *, int64_t, int64_t *, int32_t *, int *), void *ctx,
+                        int64_t nitems, int64_t n, int nthreads)
+{
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    job_t jobs[256];
+    pthread_t th[256];
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t].fn = fn; jobs[t].ctx = ctx; jobs[t].nitems = nitems; jobs[t].n = n;
+        jobs[t].nthreads = nthreads; jobs[t].tid = t; jobs[t].rc = QO_OK;
+    }
+    for (int t = 1; t < nthreads; ++t) pthread_create(&th[t], NULL, job_main, &jobs[t]);
+    job_main(&jobs[0]);
+    for (int t = 1; t < nthreads; ++t) pthread_join(th[t], NULL);
+    int rc = QO_OK;
+    for (int t = 0; t < nthreads; ++t) if (jobs[t].rc != QO_OK) rc = jobs[t].rc;
+    return rc;
+}
+
+/* ---- exact int32 accumulators for chosen source rows ------------------- */
+typedef struct {
+    const int8_t *x1; const void *x2; int weight_type; int64_t k, n, e;
+    const int64_t *off; const int64_t *rows; int32_t *acc_out;
+} accum_ctx;
+
+static void accum_item(void *p, int64_t it, int64_t *s64, int32_t *s32, int *rc)
+{
+    accum_ctx *c = (accum_ctx *)p;
+    (void)s32;
+    int64_t i = c->rows ? c->rows[it] : it;
+    int32_t *dst = c->acc_out + it * c->n;
+    int64_t g = group_of_row(c->off, c->e, i);
+    if (g < 0) { memset(dst, 0, sizeof(int32_t) * (size_t)c->n); return; }
+    int r = accum_row(c->x1, c->x2, c->weight_type, c->k, c->n, g, i, s64, dst);
+    if (r != QO_OK) *rc = r;
+}
+
+/* acc_out[r][j] for source rows rows[0..nrows) (rows == NULL: rows 0..nrows-1).
+ * Rows that belong to no group (at or past the total) come back as zeros. */
+int qo_accum(const int8_t *x1, const void *x2, int weight_type, int64_t m, int64_t k, int64_t n,
+             int64_t e, const int64_t *group_list, int group_list_type,
+             const int64_t *rows, int64_t nrows, int32_t *acc_out, int nthreads)
+{
+    if (!x1 || !x2 || !acc_out || k < 1 || n < 1 || (weight_type == 1 && n % 8)) return QO_ERR_ARG;
+    int64_t *off = (int64_t *)malloc(sizeof(int64_t) * (size_t)(e + 1));
+    if (!off) return QO_ERR_ARG;
+    int rc = qo_group_offsets(group_list, e, group_list_type, m, off);
+    if (rc == QO_OK) {
+        accum_ctx c = {x1, x2, weight_type, k, n, e, off, rows, acc_out};
+        rc = run_parallel(accum_item, &c, nrows, n, nthreads);
+    }
+    free(off);
+    return rc;
+}
+
+/* ---- dequant + combine -------------------------------------------------- */
+typedef struct {
+    const int8_t *x1; const void *x2; int weight_type; int64_t m, k, n, e;
+    const int64_t *off; int64_t total;
+    const float *scale, *pts, *logit, *bias;
+    const void *row_index; int row_index_type;
+    const uint16_t *shared; int64_t shared_bs, shared_offset, output_bs;
+    const int64_t *dest_rows;
+    double *out64; double *sabs64; float *out32;
+} fin_ctx;
+
+static inline float bf16_to_f32(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+static inline int64_t dest_of(const fin_ctx *c, int64_t i)
+{
+    if (!c->row_index) return i;
+    if (c->row_index_type == 0) return ((const int64_t *)c->row_index)[i];
+    return (int64_t)((const int32_t *)c->row_index)[i];
+}
+
+static void fin_item(void *p, int64_t it, int64_t *s64, int32_t *acc, int *rc)
+{
+    fin_ctx *c = (fin_ctx *)p;
+    const int64_t n = c->n;
+    int64_t r = c->dest_rows ? c->dest_rows[it] : it;
+    double *o64 = c->out64 ? c->out64 + it * n : NULL;
+    double *a64 = c->sabs64 ? c->sabs64 + it * n : NULL;
+    float *o32 = c->out32 ? c->out32 + it * n : NULL;
+
+    /* initial value: the sharedInput row landing here, else zero */
+    int in_shared = c->shared && r >= c->shared_offset && r < c->shared_offset + c->shared_bs;
+    for (int64_t j = 0; j < n; ++j) {
+        float s = in_shared ? bf16_to_f32(c->shared[(r - c->shared_offset) * n + j]) : 0.0f;
+        if (o64) o64[j] = (double)s;
+        if (a64) a64[j] = fabs((double)s);
+        if (o32) o32[j] = s;
+    }
+    /* contributions in ascending source row order */
+    for (int64_t i = 0; i < c->total; ++i) {
+        int64_t d = dest_of(c, i);
+        if (d < 0 || d >= c->output_bs) { *rc = QO_ERR_BAD_ROW_INDEX; continue; }
+        if (d != r) continue;
+        int64_t g = group_of_row(c->off, c->e, i);
+        int ar = accum_row(c->x1, c->x2, c->weight_type, c->k, n, g, i, s64, acc);
+        if (ar != QO_OK) *rc = ar;
+        const float pts = c->pts ? c->pts[i] : 1.0f;
+        const float lg = c->logit ? c->logit[i] : 1.0f;
+        for (int64_t j = 0; j < n; ++j) {
+            const float sc = c->scale ? c->scale[g * n + j] : 1.0f;
+            const float bs = c->bias ? c->bias[g * n + j] : 0.0f;
+            if (o64 || a64) {
+                double y = (((double)acc[j] * (double)sc) * (double)pts + (double)bs) * (double)lg;
+                if (o64) o64[j] += y;
+                if (a64) a64[j] += fabs(y);
+            }
+            if (o32) {
+                float y = (float)acc[j];        /* round to nearest even */
+                y = y * sc;
+                y = y * pts;
+                y = y + bs;
+                y = y * lg;
+                o32[j] = o32[j] + y;
+            }
+        }
+    }
+}
+
+/*
+ * Output rows dest_rows[0..ndest) (dest_rows == NULL: rows 0..ndest-1) of the
+ * op.  out64/sabs64 (double, may be NULL): value in double and the sum of the
+ * absolute values of the terms added into each element (for error bounds).
+ * out32 (may be NULL): the same in f32 in the fixed order.  scale, pts, logit,
+ * bias, row_index, shared may be NULL (1, 1, 1, 0, identity, absent).
+ */
+int qo_finalize(const int8_t *x1, const void *x2, int weight_type, int64_t m, int64_t k, int64_t n,
+                int64_t e, const int64_t *group_list, int group_list_type,
+                const float *scale, const float *pts, const float *logit, const float *bias,
+                const void *row_index, int row_index_type,
+                const uint16_t *shared, int64_t shared_bs, int64_t shared_offset, int64_t output_bs,
+                const int64_t *dest_rows, int64_t ndest,
+                double *out64, double *sabs64, float *out32, int nthreads)
+{
+    if (!x1 || !x2 || k < 1 || n < 1 || output_bs < 1 || (weight_type == 1 && n % 8)) return QO_ERR_ARG;
+    if (shared && (shared_offset < 0 || shared_offset + shared_bs > output_bs)) return QO_ERR_ARG;
+    int64_t *off = (int64_t *)malloc(sizeof(int64_t) * (size_t)(e + 1));
+    if (!off) return QO_ERR_ARG;
+    int rc = qo_group_offsets(group_list, e, group_list_type, m, off);
+    if (rc == QO_OK) {
+        fin_ctx c = {x1, x2, weight_type, m, k, n, e, off, off[e], scale, pts, logit, bias,
+                     row_index, row_index_type, shared, shared_bs, shared_offset, output_bs,
+                     dest_rows, out64, sabs64, out32};
+        rc = run_parallel(fin_item, &c, ndest, n, nthreads);
+    }
+    free(off);
+    return rc;
+}
+
+/* ---- per-token quantisation (f32; the decision is an integer) ----------- */
+int qo_per_token_quant(const uint16_t *x_bf16, int64_t rows, int64_t k, int8_t *q, float *pts)
+{
+    if (!x_bf16 || !q || !pts || rows < 0 || k < 1) return QO_ERR_ARG;
+    for (int64_t i = 0; i < rows; ++i) {
+        float a = 0.0f;
+        for (int64_t j = 0; j < k; ++j) {
+            float v = fabsf(bf16_to_f32(x_bf16[i * k + j]));
+            if (v > a) a = v;
+        }
+        pts[i] = a / 127.0f;
+        float inv = a > 0.0f ? 127.0f / a : 0.0f;
+        for (int64_t j = 0; j < k; ++j) {
+            float t = bf16_to_f32(x_bf16[i * k + j]) * inv;
+            float r = rintf(t);                 /* default mode: half to even */
+            if (r > 127.0f) r = 127.0f;
+            if (r < -127.0f) r = -127.0f;
+            q[i * k + j] = (int8_t)r;
+        }
+    }
+    return QO_OK;
+}

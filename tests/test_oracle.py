@@ -1,0 +1,307 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Each test names what fixes the expected value: the worked example printed on
+the PER_TOKEN matmul page, numpy's integer matmul (a library routine), closed
+forms of special cases, exact algebraic invariants, or a hand-worked case.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from synth import make_problem
+from synth.inputs import make_routing, _layout  # routing only, no weights
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _rand_problem(rng, e, counts, k, n, total_extra=0, weight="int8"):
+    m = int(np.sum(counts)) + total_extra
+    x1 = rng.integers(-127, 128, size=(m, k), dtype=np.int8)
+    if weight == "int8":
+        x2 = rng.integers(-127, 128, size=(e, k, n), dtype=np.int8)
+    else:
+        x2 = rng.integers(0, 2 ** 32, size=(e, k, n // 8), dtype=np.uint32).view(np.int32)
+    return x1, x2
+
+
+def _einsum_acc(x1, x2_int8, counts):
+    """Library reference: per-group int64 matmul by numpy."""
+    off = np.concatenate([[0], np.cumsum(counts)])
+    out = np.zeros((x1.shape[0], x2_int8.shape[2]), np.int64)
+    for g in range(len(counts)):
+        a, b = off[g], off[g + 1]
+        out[a:b] = x1[a:b].astype(np.int64) @ x2_int8[g].astype(np.int64)
+    return out
+
+
+# --- worked example (PER_TOKEN matmul page, 计算示例) --------------------------
+@pytest.mark.parametrize("gtype", [0, 1])
+def test_worked_example_exact(oracle, gtype):
+    g = _golden("per_token_worked_example.json")
+    x = np.array(g["x"], np.int8)
+    w = np.array(g["weight"], np.int8)[None]              # e = 1
+    scale = np.array(g["deqScale"], np.float32)[None]
+    pts = np.array(g["perTokenScale"], np.float32)
+    expect = np.array(g["output"], np.float64)
+    gl = np.array([2], np.int64)                           # both forms: end = count = 2
+    o64, sabs, o32 = oracle.finalize(x, w, gl, gtype, scale=scale, pertoken_scale=pts,
+                                     row_index=np.array([0, 1], np.int64), output_bs=2)
+    np.testing.assert_array_equal(o64, expect)
+    np.testing.assert_array_equal(o32.astype(np.float64), expect)
+    np.testing.assert_array_equal(oracle.accum(x, w, gl, gtype), [[9, 12, 15], [19, 26, 33]])
+
+
+# --- library routine: numpy integer matmul per group ------------------------
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_accum_matches_numpy_matmul(oracle, seed):
+    rng = np.random.default_rng(100 + seed)
+    e, k, n = 5, 96, 40
+    counts = rng.integers(0, 7, size=e)
+    counts[1] = 0                                           # an empty expert
+    x1, x2 = _rand_problem(rng, e, counts, k, n)
+    ref = _einsum_acc(x1, x2, counts)
+    for gtype, gl in ((1, counts), (0, np.cumsum(counts))):
+        got = oracle.accum(x1, x2, gl.astype(np.int64), gtype)
+        np.testing.assert_array_equal(got.astype(np.int64), ref)
+    rows = np.array([0, int(counts.sum()) - 1], np.int64)
+    np.testing.assert_array_equal(oracle.accum(x1, x2, counts, 1, rows=rows), ref[rows])
+
+
+def test_accum_extreme_values_exact(oracle):
+    """All-(-127) activations against all-127 weights: -k*127*127 exactly."""
+    k, n = 2048, 16
+    x1 = np.full((3, k), -127, np.int8)
+    x2 = np.full((1, k, n), 127, np.int8)
+    got = oracle.accum(x1, x2, np.array([3], np.int64), 1)
+    assert (got == -k * 127 * 127).all()
+
+
+def _pack_int4(vals):
+    """Independent packing for the test: value j of a word sits in bits 4*(j%8).."""
+    e, k, n = vals.shape
+    u = (vals.astype(np.int64) & 0xF).reshape(e, k, n // 8, 8)
+    words = np.zeros((e, k, n // 8), np.uint64)
+    for s in range(8):
+        words |= (u[..., s].astype(np.uint64) << np.uint64(4 * s))
+    return words.astype(np.uint32).view(np.int32)
+
+
+def test_int4_path_equals_int8_path(oracle):
+    rng = np.random.default_rng(7)
+    e, k, n = 3, 64, 48
+    counts = np.array([4, 0, 5])
+    vals = rng.integers(-8, 8, size=(e, k, n)).astype(np.int8)
+    x1 = rng.integers(-127, 128, size=(int(counts.sum()), k), dtype=np.int8)
+    a8 = oracle.accum(x1, vals, counts, 1)
+    a4 = oracle.accum(x1, _pack_int4(vals), counts, 1, weight="int4")
+    np.testing.assert_array_equal(a4, a8)
+    np.testing.assert_array_equal(a8.astype(np.int64), _einsum_acc(x1, vals, counts))
+    # sign-bit nibble: -8 and 7 are both representable
+    assert vals.min() == -8 and vals.max() == 7
+
+
+# --- closed forms of special cases -------------------------------------------
+def test_unit_scales_reduce_to_matmul_plus_index_add(oracle):
+    """scale = pts = logit = 1, no bias: out = index_add(rows -> tokens) of the matmul."""
+    rng = np.random.default_rng(11)
+    tokens, topk, e, k, n = 9, 3, 4, 32, 24
+    experts, w = make_routing(rng, tokens, topk, e, "uniform", 0.0)
+    ri, logit, counts = _layout(experts, w, e)
+    m = tokens * topk
+    x1 = rng.integers(-3, 4, size=(m, k), dtype=np.int8)   # keeps every sum exact in f32
+    x2 = rng.integers(-3, 4, size=(e, k, n), dtype=np.int8)
+    acc = _einsum_acc(x1, x2, counts)
+    ref = np.zeros((tokens, n), np.float64)
+    np.add.at(ref, ri, acc.astype(np.float64))
+    o64, sabs, o32 = oracle.finalize(x1, x2, counts, 1, row_index=ri, output_bs=tokens)
+    np.testing.assert_array_equal(o64, ref)
+    np.testing.assert_array_equal(o32.astype(np.float64), ref)
+    np.testing.assert_array_equal(sabs, _abs_index_add(ri, acc, tokens))
+
+
+def _abs_index_add(ri, acc, tokens):
+    out = np.zeros((tokens, acc.shape[1]), np.float64)
+    np.add.at(out, ri, np.abs(acc).astype(np.float64))
+    return out
+
+
+def test_shared_input_alone_lands_at_offset(oracle):
+    """x1 = 0 and no bias: the output is the bf16 sharedInput rows at the offset, zeros elsewhere."""
+    rng = np.random.default_rng(5)
+    e, k, n, m, out_bs, bs, off = 2, 16, 32, 6, 10, 4, 3
+    x1 = np.zeros((m, k), np.int8)
+    x2 = rng.integers(-127, 128, size=(e, k, n), dtype=np.int8)
+    sh_f = rng.standard_normal((bs, n)).astype(np.float32)
+    sh = (sh_f.view(np.uint32) >> 16).astype(np.uint16)   # truncate to bf16 bits
+    sh_exact = (sh.astype(np.uint32) << 16).view(np.float32)
+    ri = rng.integers(0, out_bs, size=m).astype(np.int64)
+    o64, _, o32 = oracle.finalize(x1, x2, np.array([2, 4], np.int64), 1,
+                                  scale=np.ones((e, n), np.float32), logit=np.full(m, 0.5, np.float32),
+                                  row_index=ri, shared=sh, shared_offset=off, output_bs=out_bs)
+    ref = np.zeros((out_bs, n), np.float32)
+    ref[off:off + bs] = sh_exact
+    np.testing.assert_array_equal(o32, ref)
+    np.testing.assert_array_equal(o64, ref.astype(np.float64))
+
+
+def test_bias_sits_inside_the_routing_weight(oracle):
+    """One row, scale = pts = 1, logit = 2: out = 2 * (acc + bias) (reading: bias before logit)."""
+    rng = np.random.default_rng(9)
+    k, n = 8, 16
+    x1 = rng.integers(-5, 6, size=(1, k), dtype=np.int8)
+    x2 = rng.integers(-5, 6, size=(1, k, n), dtype=np.int8)
+    bias = np.array(rng.integers(-64, 64, size=(1, n)), np.float32) / 8   # exact in f32
+    acc = x1.astype(np.int64) @ x2[0].astype(np.int64)
+    o64, _, o32 = oracle.finalize(x1, x2, np.array([1], np.int64), 1, bias=bias,
+                                  logit=np.array([2.0], np.float32), output_bs=1)
+    np.testing.assert_array_equal(o64, 2.0 * (acc + bias.astype(np.float64)))
+    np.testing.assert_array_equal(o32.astype(np.float64), 2.0 * (acc + bias.astype(np.float64)))
+
+
+# --- invariants --------------------------------------------------------------
+def test_logit_doubling_doubles_output_exactly(oracle):
+    p = make_problem("tiny", n=64)
+    a64, _, a32 = oracle.problem_finalize(p)
+    p.logit = (p.logit * np.float32(2)).astype(np.float32)
+    b64, _, b32 = oracle.problem_finalize(p)
+    np.testing.assert_array_equal(b64, 2 * a64)
+    np.testing.assert_array_equal(b32, 2 * a32)
+
+
+def test_group_list_forms_agree_and_empty_experts_change_nothing(oracle):
+    p = make_problem("tiny", n=64, e=6)
+    base = oracle.problem_finalize(p)
+    counts = p.counts
+    alt = oracle.finalize(p.x1, p.x2, np.cumsum(counts), 0, scale=p.scale,
+                          pertoken_scale=p.pertoken_scale, logit=p.logit, row_index=p.row_index,
+                          output_bs=p.output_bs)
+    for a, b in zip(base, alt):
+        np.testing.assert_array_equal(a, b)
+    # insert two empty experts (with arbitrary weights) in front and in the middle
+    rng = np.random.default_rng(3)
+    junk = rng.integers(-127, 128, size=(1, p.k, p.n), dtype=np.int8)
+    x2b = np.concatenate([junk, p.x2[:3], junk, p.x2[3:]])
+    scb = np.concatenate([p.scale[:1], p.scale[:3], p.scale[:1], p.scale[3:]])
+    cb = np.concatenate([[0], counts[:3], [0], counts[3:]]).astype(np.int64)
+    ins = oracle.finalize(p.x1, x2b, cb, 1, scale=scb, pertoken_scale=p.pertoken_scale,
+                          logit=p.logit, row_index=p.row_index, output_bs=p.output_bs)
+    for a, b in zip(base, ins):
+        np.testing.assert_array_equal(a, b)
+
+
+def test_rows_past_the_total_are_ignored(oracle):
+    rng = np.random.default_rng(21)
+    e, k, n = 3, 32, 16
+    counts = np.array([2, 3, 1])
+    x1, x2 = _rand_problem(rng, e, counts, k, n, total_extra=4)
+    ri = np.arange(x1.shape[0], dtype=np.int64) % 5
+    a = oracle.finalize(x1, x2, counts, 1, row_index=ri, output_bs=5)
+    x1b = x1.copy()
+    x1b[6:] = rng.integers(-127, 128, size=(4, k), dtype=np.int8)
+    ri_b = ri.copy()
+    ri_b[6:] = 4
+    b = oracle.finalize(x1b, x2, counts, 1, row_index=ri_b, output_bs=5)
+    for u, v in zip(a, b):
+        np.testing.assert_array_equal(u, v)
+
+
+def test_int32_row_index_same_as_int64(oracle):
+    p = make_problem("tiny", n=64)
+    a = oracle.problem_finalize(p)
+    p.row_index = p.row_index.astype(np.int32)
+    b = oracle.problem_finalize(p)
+    for u, v in zip(a, b):
+        np.testing.assert_array_equal(u, v)
+
+
+def test_f32_order_within_rounding_of_f64(oracle):
+    p = make_problem("tiny")
+    o64, sabs, o32 = oracle.problem_finalize(p)
+    err = np.abs(o32.astype(np.float64) - o64) / np.maximum(sabs, 1e-30)
+    assert err.max() < 8 * 2.0 ** -24 * 4
+
+
+def test_dest_row_subset_matches_full(oracle):
+    p = make_problem("tiny", n=128)
+    full = oracle.problem_finalize(p)
+    rows = np.array([0, 5, 17, 31], np.int64)
+    sub = oracle.problem_finalize(p, dest_rows=rows)
+    for f, s in zip(full, sub):
+        np.testing.assert_array_equal(f[rows], s)
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid_prefill", "decode", "large_prefill", "w4a8_prologue"])
+def test_routing_invariants(name):
+    """Sum of counts = m and every output row receives exactly topK contributions."""
+    from synth.inputs import CONFIGS, SEED_BASE
+    s = CONFIGS[name]
+    rng = np.random.default_rng(SEED_BASE + s.index)
+    experts, w = make_routing(rng, s.tokens, s.topk, s.e, s.routing, s.routing_param)
+    ri, logit, counts = _layout(experts, w, s.e)
+    assert counts.sum() == s.tokens * s.topk
+    assert (np.bincount(ri, minlength=s.tokens) == s.topk).all()
+    # each token's slots go to distinct experts
+    assert all(len(set(r)) == s.topk for r in experts[:256])
+    # logit rows per token sum to one (softmax weights)
+    sums = np.zeros(s.tokens)
+    np.add.at(sums, ri, logit.astype(np.float64))
+    np.testing.assert_allclose(sums, 1.0, rtol=1e-6)
+
+
+# --- groupList validation (parameter constraints, page 1) --------------------
+def test_group_list_errors(oracle):
+    m = 10
+    with pytest.raises(oracle.OracleError) as ei:
+        oracle.group_offsets(np.array([2, -1, 3]), 1, m)
+    assert ei.value.code == oracle.QO_ERR_NEGATIVE_COUNT
+    with pytest.raises(oracle.OracleError) as ei:
+        oracle.group_offsets(np.array([2, 5, 4]), 0, m)
+    assert ei.value.code == oracle.QO_ERR_NOT_MONOTONE
+    with pytest.raises(oracle.OracleError) as ei:
+        oracle.group_offsets(np.array([6, 5]), 1, m)
+    assert ei.value.code == oracle.QO_ERR_TOTAL_GT_M
+    np.testing.assert_array_equal(oracle.group_offsets(np.array([2, 2, 7]), 0, m), [0, 2, 2, 7])
+    np.testing.assert_array_equal(oracle.group_offsets(np.array([2, 0, 5]), 1, m), [0, 2, 2, 7])
+
+
+# --- per-token quant ---------------------------------------------------------
+def _bf16_bits(vals):
+    v = np.asarray(vals, np.float32)
+    bits = v.view(np.uint32)
+    assert ((bits & 0xFFFF) == 0).all(), "test values must be exact in bf16"
+    return (bits >> 16).astype(np.uint16)
+
+
+def test_per_token_quant_hand_cases(oracle):
+    # absmax 127 gives inverse exactly 1, so q = round-half-even(x): 2.5->2, 3.5->4, -2.5->-2, 0.5->0
+    row0 = [127.0, 2.5, 3.5, -2.5, 0.5, 1.5, -127.0, 0.0]
+    # absmax 2: inverse 63.5; 2 -> 127, -1 -> -63.5 -> -64, 0.5 -> 31.75 -> 32, 0.25 -> 15.875 -> 16
+    row1 = [2.0, -1.0, 0.5, 0.25, 0.0, -2.0, 1.0, 0.125]
+    row2 = [0.0] * 8
+    q, pts = oracle.per_token_quant(_bf16_bits([row0, row1, row2]))
+    np.testing.assert_array_equal(q[0], [127, 2, 4, -2, 0, 2, -127, 0])
+    np.testing.assert_array_equal(q[1], [127, -64, 32, 16, 0, -127, 64, 8])
+    np.testing.assert_array_equal(q[2], 0)
+    assert pts[0] == np.float32(1.0)
+    assert pts[1] == np.float32(2.0) / np.float32(127.0)
+    assert pts[2] == 0.0
+
+
+def test_per_token_quant_bounds(oracle):
+    from synth.inputs import bf16_bits_normal
+    rng = np.random.default_rng(17)
+    x = bf16_bits_normal(rng, (64, 512))
+    q, pts = oracle.per_token_quant(x)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert np.abs(q).max() <= 127
+    assert (np.abs(q).max(axis=1) == 127).all()
+    np.testing.assert_array_equal(pts, (np.abs(xf).max(axis=1).astype(np.float32) / np.float32(127)))
+    recon = q.astype(np.float64) * pts.astype(np.float64)[:, None]
+    assert (np.abs(xf - recon) <= pts.astype(np.float64)[:, None] * 0.50002).all()
