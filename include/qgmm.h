@@ -1,0 +1,177 @@
+/*
+ * qgmm.h -- C ABI of the B200 (sm_100a) fused int8 GroupedMatmul +
+ * MoeFinalizeRouting library (libqgmm.so).
+ *
+ * The operation (pages: "aclnnGroupedMatmulFinalizeRoutingWeightNzV2",
+ * function description and parameter constraints; "matmul支持pertoken量化模式",
+ * 计算示例):
+ *
+ *   off[0] = 0; off[g+1] = group_list[g]            (group_list_type 0: cumulative ends)
+ *               off[g+1] = off[g] + group_list[g]   (group_list_type 1: per-group counts)
+ *   for every expert g and row i in [off[g], off[g+1]):
+ *     acc[i][j] = sum_kk x1[i][kk] * W(g, kk, j)                      exact int32
+ *     y[i][j]   = ((f32(acc) * scale[g][j]) * pertoken_scale[i] + bias[g][j]) * logit[i]
+ *   out[r][j]  = (shared_offset <= r < shared_offset + shared_bs) ? f32(shared[r - shared_offset][j]) : 0
+ *   out[row_index[i]][j] += y[i][j]    for every row i below the groups' total
+ *
+ * W(g, kk, j) is x2[g][kk][j] (int8, layout (e, k, n), n contiguous), or for
+ * int4 weights the signed nibble j%8 (lowest nibble = lowest j) of the int32
+ * word x2[g][kk][j/8] (layout (e, k, n/8)).  Every f32 step rounds to nearest
+ * even; nothing is fused into an FMA.  Where the pages leave the formula open
+ * (bias position, unweighted sharedInput, nibble order, summation order) the
+ * library takes the readings written above.
+ *
+ * Conventions shared by every entry point:
+ *  - Every pointer except those of qgmm_finalize_workspace, qgmm_device_status
+ *    (flags) and qgmm_status_string is a DEVICE pointer on the current CUDA
+ *    device.  The caller owns all memory, including the workspace; the library
+ *    allocates nothing and keeps no state between calls (a per-device cache of
+ *    the SM count and the driver's tensor-map entry point aside).
+ *  - Every call is asynchronous on `cuda_stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) except qgmm_device_status, which synchronises it.
+ *  - Host-side checks run before any launch; a failing check returns its code
+ *    and launches nothing.
+ *  - Problems the host cannot see (group_list values, row_index values) are
+ *    checked on the device: offending rows are skipped, the remaining rows are
+ *    still computed, and QGMM_DEV_* bits are set in the workspace status word,
+ *    which qgmm_device_status returns.  No kernel traps or asserts.
+ *  - Every wait inside a kernel is bounded (about one second); if one runs out
+ *    the kernel sets QGMM_DEV_TIMEOUT and returns.
+ */
+#ifndef QGMM_H
+#define QGMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QGMM_OK = 0,
+    QGMM_ERR_NULL_PTR = 1,            /* a required pointer is NULL                          */
+    QGMM_ERR_SHAPE = 2,               /* a size is out of range (limits below)                */
+    QGMM_ERR_DTYPE = 3,               /* an unknown weight / index / group-list type code     */
+    QGMM_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes below qgmm_finalize_workspace's answer      */
+    QGMM_ERR_UNSUPPORTED = 5,         /* the device is not sm_100 or a feature is not built   */
+    QGMM_ERR_CUDA = 6,                /* a CUDA runtime / driver call failed                  */
+    QGMM_ERR_DEVICE_INPUT = 7,        /* qgmm_device_status found QGMM_DEV_* bits set         */
+    QGMM_ERR_ALIGNMENT = 8            /* a pointer is not 16-byte aligned                     */
+} qgmm_status;
+
+enum { QGMM_W_INT8 = 0, QGMM_W_INT4_PACKED_INT32 = 1 };   /* x2: (e,k,n) int8 | (e,k,n/8) int32 */
+enum { QGMM_IDX_INT64 = 0, QGMM_IDX_INT32 = 1 };          /* row_index element type             */
+enum { QGMM_GROUP_CUMSUM = 0, QGMM_GROUP_COUNTS = 1 };    /* group_list meaning                 */
+
+/* Device-side status bits (qgmm_device_status). */
+#define QGMM_DEV_GROUP_NEGATIVE     (1u << 0)  /* a type-1 count (or type-0 end) below zero    */
+#define QGMM_DEV_GROUP_NOT_MONOTONE (1u << 1)  /* type 0: an end smaller than the previous one */
+#define QGMM_DEV_GROUP_TOTAL_GT_M   (1u << 2)  /* the groups cover more than m rows           */
+#define QGMM_DEV_ROW_INDEX_RANGE    (1u << 3)  /* a row_index value outside [0, output_bs)    */
+#define QGMM_DEV_TIMEOUT            (1u << 4)  /* a bounded in-kernel wait ran out            */
+
+/*
+ * Problem description.
+ *   m       rows of x1 (tokens x topK), 1 <= m <= 2^24 (page 1 allows [1, 16*1024*8])
+ *   k       reduction size, 128 <= k <= 65536, k % 128 == 0 (page 1 fixes k = 2048)
+ *   n       output columns, 256 <= n <= 65536, n % 256 == 0 (page 1 fixes n = 7168)
+ *   e       experts, 1 <= e <= 1024 (page 1: [1, 256] on A2/A3, [1, 1024] on Atlas 350)
+ *   output_bs   rows of out, >= 1
+ *   weight_type     QGMM_W_INT8 | QGMM_W_INT4_PACKED_INT32
+ *   group_list_type QGMM_GROUP_CUMSUM (0) | QGMM_GROUP_COUNTS (1)
+ *   row_index_type  QGMM_IDX_INT64 | QGMM_IDX_INT32
+ *   shared_bs, shared_offset   sharedInput rows and where they land;
+ *                   shared_bs == 0 means no sharedInput;
+ *                   0 <= shared_offset and shared_offset + shared_bs <= output_bs (page 1)
+ *   deterministic   0: combine with float atomics (order unspecified);
+ *                   1: fixed per-element order -- shared value first, then the
+ *                      source rows in ascending order -- through a
+ *                      destination-sorted segmented reduce.  Bitwise
+ *                      reproducible from run to run.  (Page 1, 确定性计算.)
+ *   expected_m_per_expert   tiling hint, rows one expert is expected to get;
+ *                   0 = use m / e.  Changes only the tile shape, never the
+ *                   result.  (Page 1: tuningConfigOptional[0].)
+ */
+typedef struct {
+    int64_t m, k, n, e, output_bs;
+    int32_t weight_type, group_list_type, row_index_type;
+    int64_t shared_bs, shared_offset;
+    int32_t deterministic;
+    int64_t expected_m_per_expert;
+} qgmm_problem;
+
+/*
+ * Stage 1 (page 1: the GetWorkspaceSize call, which validates the inputs).
+ * Checks `p` and writes the workspace bytes qgmm_finalize needs with it to
+ * *ws_bytes (host pointers).  Atomic mode: 256 bytes (the status word).
+ * Deterministic mode: 256 + m*n*4 (f32 rows y) + (2*output_bs + 1 + m)*4
+ * rounded up to 256.  Errors: NULL_PTR, SHAPE, DTYPE.
+ */
+qgmm_status qgmm_finalize_workspace(const qgmm_problem *p, size_t *ws_bytes);
+
+/*
+ * Stage 2: run the operation on `cuda_stream`.
+ *   x1              int8 [m, k] row-major, required
+ *   x2              int8 [e, k, n] or int32 [e, k, n/8], row-major, required
+ *   scale           f32 [e, n] (page 1's (e, 1, n)); NULL = all ones
+ *   pertoken_scale  f32 [m]; NULL = all ones
+ *   group_list      int64 [e], required
+ *   logit           f32 [m]; NULL = all ones
+ *   row_index       int64 or int32 [m]; NULL = identity (needs output_bs >= total)
+ *   bias            f32 [e, n]; NULL = zeros
+ *   shared_input    bf16 bits [shared_bs, n]; required iff shared_bs > 0
+ *   out             f32 [output_bs, n], fully overwritten (no need to clear it)
+ *   workspace       device memory of ws_bytes bytes, 256-byte aligned
+ * x1, x2, out and shared_input must be 16-byte aligned.  Rows at or past the
+ * groups' total are ignored.
+ * Errors: NULL_PTR, SHAPE, DTYPE, ALIGNMENT, WORKSPACE_TOO_SMALL, UNSUPPORTED, CUDA.
+ */
+qgmm_status qgmm_finalize(const qgmm_problem *p, const int8_t *x1, const void *x2,
+                          const float *scale, const float *pertoken_scale,
+                          const int64_t *group_list, const float *logit, const void *row_index,
+                          const float *bias, const uint16_t *shared_input, float *out,
+                          void *workspace, size_t ws_bytes, void *cuda_stream);
+
+/*
+ * Per-token quantisation prologue (page 4, per_token_cast: the value times a
+ * precomputed inverse scale; page 2, quant mode 7 "dynamic pertoken"):
+ *   a = max_j |x[i][j]|;  scale_out[i] = a / 127;  inv = a > 0 ? 127 / a : 0
+ *   x1_out[i][j] = clamp(round_half_even(x[i][j] * inv), -127, 127)
+ * in f32 with IEEE division.  x_bf16: bf16 bits [rows, k]; x1_out int8
+ * [rows, k]; scale_out f32 [rows].  1 <= rows <= 2^31-1, k % 8 == 0,
+ * 8 <= k <= 65536; x_bf16 and x1_out 16-byte aligned.
+ * Errors: NULL_PTR, SHAPE, ALIGNMENT, UNSUPPORTED, CUDA.
+ */
+qgmm_status qgmm_per_token_quant(const uint16_t *x_bf16, int64_t rows, int64_t k, int8_t *x1_out,
+                                 float *scale_out, void *cuda_stream);
+
+/*
+ * The raw int32 accumulators acc_out[i][j] = sum_kk x1[i][kk] * W(g, kk, j)
+ * for every row i below the groups' total, written by the same grouped GEMM
+ * that qgmm_finalize runs (no epilogue arithmetic, no combine).  Rows at or
+ * past the total are not written.  acc_out: int32 [m, n], 16-byte aligned.
+ * `p` supplies m, k, n, e, weight_type, group_list_type and the tiling hint;
+ * the workspace is the atomic-mode one (>= 256 bytes).
+ * Errors: as qgmm_finalize.
+ */
+qgmm_status qgmm_debug_accum(const qgmm_problem *p, const int8_t *x1, const void *x2,
+                             const int64_t *group_list, int32_t *acc_out, void *workspace,
+                             size_t ws_bytes, void *cuda_stream);
+
+/*
+ * Synchronise `cuda_stream`, then copy the workspace status word written by
+ * the last qgmm_finalize / qgmm_debug_accum on that workspace to *flags (host).
+ * Returns QGMM_ERR_DEVICE_INPUT when any QGMM_DEV_* bit is set, QGMM_OK when
+ * none is, QGMM_ERR_CUDA when the copy fails.
+ */
+qgmm_status qgmm_device_status(const void *workspace, uint32_t *flags, void *cuda_stream);
+
+/* A static English description of a status code. */
+const char *qgmm_status_string(qgmm_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QGMM_H */

@@ -1,0 +1,167 @@
+"""B200 (sm_100a) fused int8 GroupedMatmul + MoeFinalizeRouting.
+
+A thin ctypes binding over ``libqgmm.so`` (C ABI in ``include/qgmm.h``).  It
+only marshals arguments: torch tensors are passed as device pointers together
+with the current CUDA stream; every step of the operation runs in the
+library's kernels.  There is no fallback: if the library is missing or the
+device is not a B200, the calls raise.
+
+Entry points mirror the C ABI:
+    finalize_workspace(problem) -> bytes
+    finalize(problem, x1, x2, ..., out, workspace)
+    per_token_quant(x_bf16, x1_out, scale_out)
+    debug_accum(problem, x1, x2, group_list, acc_out, workspace)
+    device_status(workspace) -> QGMM_DEV_* flags
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libqgmm.so")
+
+QGMM_OK = 0
+QGMM_ERR_NULL_PTR = 1
+QGMM_ERR_SHAPE = 2
+QGMM_ERR_DTYPE = 3
+QGMM_ERR_WORKSPACE_TOO_SMALL = 4
+QGMM_ERR_UNSUPPORTED = 5
+QGMM_ERR_CUDA = 6
+QGMM_ERR_DEVICE_INPUT = 7
+QGMM_ERR_ALIGNMENT = 8
+
+QGMM_W_INT8 = 0
+QGMM_W_INT4_PACKED_INT32 = 1
+QGMM_IDX_INT64 = 0
+QGMM_IDX_INT32 = 1
+QGMM_GROUP_CUMSUM = 0
+QGMM_GROUP_COUNTS = 1
+
+QGMM_DEV_GROUP_NEGATIVE = 1 << 0
+QGMM_DEV_GROUP_NOT_MONOTONE = 1 << 1
+QGMM_DEV_GROUP_TOTAL_GT_M = 1 << 2
+QGMM_DEV_ROW_INDEX_RANGE = 1 << 3
+QGMM_DEV_TIMEOUT = 1 << 4
+
+EXPORTS = ("qgmm_finalize_workspace", "qgmm_finalize", "qgmm_per_token_quant", "qgmm_debug_accum",
+           "qgmm_device_status", "qgmm_status_string")
+
+
+class QgmmProblem(C.Structure):
+    """Mirror of ``qgmm_problem`` (same field order, natural C alignment)."""
+    _fields_ = [
+        ("m", C.c_int64), ("k", C.c_int64), ("n", C.c_int64), ("e", C.c_int64), ("output_bs", C.c_int64),
+        ("weight_type", C.c_int32), ("group_list_type", C.c_int32), ("row_index_type", C.c_int32),
+        ("shared_bs", C.c_int64), ("shared_offset", C.c_int64),
+        ("deterministic", C.c_int32),
+        ("expected_m_per_expert", C.c_int64),
+    ]
+
+
+class QgmmError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        msg = status_string(code) if _lib is not None else str(code)
+        super().__init__(f"{what}: {msg} (status {code})")
+        self.code = code
+
+
+_lib = None
+
+
+def lib():
+    """Load libqgmm.so (built in-tree by ``build.py``); raise if it is absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libqgmm.so not built at {LIB_PATH}; run quantized_moe_grouped_persistent_b200/build.py")
+        L = C.CDLL(LIB_PATH)
+        P, I64, U = C.c_void_p, C.c_int64, C.c_size_t
+        L.qgmm_finalize_workspace.argtypes = [C.POINTER(QgmmProblem), C.POINTER(C.c_size_t)]
+        L.qgmm_finalize.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, P, P, P, P, P, P, U, P]
+        L.qgmm_per_token_quant.argtypes = [P, I64, I64, P, P, P]
+        L.qgmm_debug_accum.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, U, P]
+        L.qgmm_device_status.argtypes = [P, C.POINTER(C.c_uint32), P]
+        L.qgmm_status_string.argtypes = [C.c_int]
+        L.qgmm_status_string.restype = C.c_char_p
+        for name in EXPORTS[:-1]:
+            getattr(L, name).restype = C.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().qgmm_status_string(code).decode()
+
+
+def make_problem(m: int, k: int, n: int, e: int, output_bs: int, *, weight_type: int = QGMM_W_INT8,
+                 group_list_type: int = QGMM_GROUP_CUMSUM, row_index_type: int = QGMM_IDX_INT64,
+                 shared_bs: int = 0, shared_offset: int = 0, deterministic: bool = False,
+                 expected_m_per_expert: int = 0) -> QgmmProblem:
+    return QgmmProblem(m, k, n, e, output_bs, weight_type, group_list_type, row_index_type, shared_bs,
+                       shared_offset, int(bool(deterministic)), expected_m_per_expert)
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int, what: str):
+    if rc != QGMM_OK:
+        raise QgmmError(rc, what)
+
+
+def finalize_workspace(problem: QgmmProblem) -> int:
+    out = C.c_size_t(0)
+    _check(lib().qgmm_finalize_workspace(C.byref(problem), C.byref(out)), "qgmm_finalize_workspace")
+    return out.value
+
+
+def finalize(problem: QgmmProblem, x1, x2, scale, pertoken_scale, group_list, logit, row_index, bias,
+             shared_input, out, workspace, ws_bytes: Optional[int] = None, stream=None) -> None:
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().qgmm_finalize(C.byref(problem), _ptr(x1), _ptr(x2), _ptr(scale), _ptr(pertoken_scale),
+                             _ptr(group_list), _ptr(logit), _ptr(row_index), _ptr(bias), _ptr(shared_input),
+                             _ptr(out), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "qgmm_finalize")
+
+
+def per_token_quant(x_bf16, x1_out, scale_out, rows: Optional[int] = None, k: Optional[int] = None,
+                    stream=None) -> None:
+    if rows is None:
+        rows, k = x_bf16.shape
+    rc = lib().qgmm_per_token_quant(_ptr(x_bf16), rows, k, _ptr(x1_out), _ptr(scale_out), _stream(stream))
+    _check(rc, "qgmm_per_token_quant")
+
+
+def debug_accum(problem: QgmmProblem, x1, x2, group_list, acc_out, workspace, ws_bytes: Optional[int] = None,
+                stream=None) -> None:
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().qgmm_debug_accum(C.byref(problem), _ptr(x1), _ptr(x2), _ptr(group_list), _ptr(acc_out),
+                                _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "qgmm_debug_accum")
+
+
+def device_status(workspace, stream=None) -> int:
+    """Synchronise the stream and return the QGMM_DEV_* bits of the last call on ``workspace``."""
+    flags = C.c_uint32(0)
+    rc = lib().qgmm_device_status(_ptr(workspace), C.byref(flags), _stream(stream))
+    if rc not in (QGMM_OK, QGMM_ERR_DEVICE_INPUT):
+        raise QgmmError(rc, "qgmm_device_status")
+    return flags.value

@@ -1,0 +1,707 @@
+// kernels.cuh -- sm_100a kernels of the fused int8 GroupedMatmul +
+// MoeFinalizeRouting op ("aclnnGroupedMatmulFinalizeRoutingWeightNzV2":
+// grouped matmul whose output rows are combined into the output by index;
+// dequant rule of "matmul支持pertoken量化模式", 计算示例).
+//
+//   K1 output_init_kernel       out = sharedInput rows at the offset, else 0
+//   K2 grouped_gemm_kernel      persistent grouped GEMM, tcgen05 kind::i8 into
+//                               TMEM, TMA-fed smem ring, epilogue fused in
+//                               registers (atomic combine | f32 rows | raw int32)
+//   K3 det_* kernels            destination-sorted segmented reduce (fixed order)
+//   K0 per_token_quant_kernel   bf16 -> int8 + absmax/127 per row
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "ptx_sm100.cuh"
+#include "../../include/qgmm.h"
+
+namespace qgmm {
+
+// ---------------------------------------------------------------- tiling
+constexpr int BM = 128;          // MMA M: TMEM lanes per accumulator
+constexpr int BN = 256;          // MMA N: TMEM columns per accumulator
+constexpr int BK = 128;          // K bytes per pipeline stage (one 128-byte swizzle row)
+constexpr int UMMA_K = 32;       // K of one tcgen05.mma kind::i8
+constexpr int A_STAGE_BYTES = BM * BK;       // 16 KB (box height may be smaller)
+constexpr int B_STAGE_BYTES = BK * BN;       // 32 KB: two 128-column MN-major atoms
+constexpr int P_STAGE_BYTES = BK * BN / 2;   // 16 KB: packed int4 staging
+constexpr int B_ATOM_BYTES = BK * 128;       // one 128-column atom (LBO)
+constexpr int TMEM_COLS = 2 * BN;            // double-buffered accumulator
+constexpr int MAX_E = 1024;
+
+enum Epilogue : int { EPI_ATOMIC = 0, EPI_STORE_Y = 1, EPI_RAW_ACC = 2 };
+
+template <bool W4>
+struct GemmCfg {
+    static constexpr int STAGES = W4 ? 3 : 4;
+    static constexpr int NUM_WARPS = W4 ? 10 : 6;   // producer, MMA, 4 epilogue (+4 unpack)
+    static constexpr int THREADS = NUM_WARPS * 32;
+    static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES + (W4 ? P_STAGE_BYTES : 0);
+    static constexpr int NUM_BARS = 3 * STAGES + 2 + 2 + 1;
+    static constexpr int CTRL_BYTES = NUM_BARS * 8 + 16;
+    static constexpr int TABLE_BYTES = 2 * (MAX_E + 1) * 4;
+    static constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + CTRL_BYTES + TABLE_BYTES;
+};
+
+struct GemmArgs {
+    const int64_t *group_list;
+    int64_t m;
+    int32_t e, group_list_type;
+    int32_t k, n;
+    int32_t tile_rows;     // rows per m-tile = TMA box height of x1 (16, 32, 64 or 128)
+    int32_t slab_ntiles;   // n-tiles per slab; divides n / BN
+    const float *scale, *pts, *logit, *bias;
+    const void *row_index;
+    int32_t row_index_type;
+    int64_t output_bs;
+    float *out;            // EPI_ATOMIC: out [output_bs, n]; EPI_STORE_Y: y [m, n]
+    int32_t *acc_out;      // EPI_RAW_ACC: [m, n]
+    uint32_t *status;
+};
+
+// ---------------------------------------------------------------- groups
+// Warp-cooperative decode of groupList (page 1, parameter constraints):
+// off[g+1] = end row of group g, cum[g+1] = m-tiles of groups 0..g.
+// Invalid lists are sanitised so every offset stays in [0, m] and monotone
+// (type 0: running max of clamp(end, 0, m); type 1: clamp of the running sum
+// of max(count, 0)); the returned QGMM_DEV_* bits say what was wrong.
+__device__ __forceinline__ uint32_t decode_groups_warp(const int64_t *gl, int e, int type, int64_t m,
+                                                       int tile_rows, int32_t *off, int32_t *cum)
+{
+    const int lane = threadIdx.x & 31;
+    uint32_t flags = 0;
+    int64_t carry_end = 0;     // end of the previous chunk's last group
+    int64_t carry_sum = 0;     // type 1: unclamped running sum
+    int32_t carry_cum = 0;
+    if (lane == 0) {
+        off[0] = 0;
+        cum[0] = 0;
+    }
+    for (int base = 0; base < e; base += 32) {
+        const int g = base + lane;
+        const bool in = g < e;
+        const int64_t v = in ? gl[g] : 0;
+        if (in && v < 0) flags |= QGMM_DEV_GROUP_NEGATIVE;
+        int64_t end;
+        if (type == 0) {
+            if (in && g > 0 && v < gl[g - 1]) flags |= QGMM_DEV_GROUP_NOT_MONOTONE;
+            if (in && v > m) flags |= QGMM_DEV_GROUP_TOTAL_GT_M;
+            int64_t s = v < 0 ? 0 : (v > m ? m : v);
+            if (!in) s = 0;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int64_t o = __shfl_up_sync(0xffffffffu, s, d);
+                if (lane >= d && o > s) s = o;
+            }
+            end = s > carry_end ? s : carry_end;
+        } else {
+            int64_t s = (in && v > 0) ? v : 0;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int64_t o = __shfl_up_sync(0xffffffffu, s, d);
+                if (lane >= d) s += o;
+            }
+            s += carry_sum;
+            carry_sum = __shfl_sync(0xffffffffu, s, 31);
+            if (in && s > m) flags |= QGMM_DEV_GROUP_TOTAL_GT_M;
+            end = s > m ? m : s;
+        }
+        int64_t start = __shfl_up_sync(0xffffffffu, end, 1);
+        if (lane == 0) start = carry_end;
+        const int64_t rows = end - start;
+        int32_t mt = in ? static_cast<int32_t>((rows + tile_rows - 1) / tile_rows) : 0;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int32_t o = __shfl_up_sync(0xffffffffu, mt, d);
+            if (lane >= d) mt += o;
+        }
+        mt += carry_cum;
+        if (in) {
+            off[g + 1] = static_cast<int32_t>(end);
+            cum[g + 1] = mt;
+        }
+        carry_end = __shfl_sync(0xffffffffu, end, 31);
+        carry_cum = __shfl_sync(0xffffffffu, mt, 31);
+    }
+    // OR-reduce the flags across the warp
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) flags |= __shfl_xor_sync(0xffffffffu, flags, d);
+    __syncwarp();
+    return flags;
+}
+
+struct TileCoord {
+    int g, row0, row_end, nt;
+};
+
+// Tile t of the persistent walk.  Order: slab of slab_ntiles n-tiles, then
+// expert, then m-tile, then the n-tiles of the slab -- so consecutive tiles
+// (taken by neighbouring CTAs at the same time) share one x1 row tile and one
+// expert's weight columns, and one slab of the output stays hot in L2.
+__device__ __forceinline__ TileCoord tile_coord(int t, int MT, int SW, const int32_t *off, const int32_t *cum,
+                                                int e, int tile_rows)
+{
+    const int per_slab = MT * SW;
+    const int s = t / per_slab;
+    const int r = t - s * per_slab;
+    const int mt = r / SW;
+    TileCoord c;
+    c.nt = s * SW + (r - mt * SW);
+    int lo = 0, hi = e;  // cum[lo] <= mt < cum[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (cum[mid] <= mt) lo = mid;
+        else hi = mid;
+    }
+    c.g = lo;
+    c.row0 = off[lo] + (mt - cum[lo]) * tile_rows;
+    c.row_end = off[lo + 1];
+    return c;
+}
+
+__device__ __forceinline__ int64_t load_row_index(const void *ri, int type, int64_t i)
+{
+    if (ri == nullptr) return i;
+    if (type == QGMM_IDX_INT64) return __ldg(static_cast<const long long *>(ri) + i);
+    return static_cast<int64_t>(__ldg(static_cast<const int *>(ri) + i));
+}
+
+// int4 (two's complement, lowest nibble = lowest column) -> int8, 8 values per word.
+__device__ __forceinline__ void unpack_int4x8(uint32_t w, uint32_t &lo_out, uint32_t &hi_out)
+{
+    uint32_t lo = w & 0x0F0F0F0Fu;          // nibbles 0, 2, 4, 6
+    uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;   // nibbles 1, 3, 5, 7
+    lo |= (lo & 0x08080808u) * 30u;         // sign bit 8 -> 0xF0 fill; no carry between bytes
+    hi |= (hi & 0x08080808u) * 30u;
+    lo_out = __byte_perm(lo, hi, 0x5140);   // columns 0..3
+    hi_out = __byte_perm(lo, hi, 0x7362);   // columns 4..7
+}
+
+// ---------------------------------------------------------------- K2
+template <int EPI, bool W4>
+__global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                        const GemmArgs args)
+{
+    using Cfg = GemmCfg<W4>;
+    constexpr int S = Cfg::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *smem_a = smem;
+    uint8_t *smem_b = smem_a + S * A_STAGE_BYTES;
+    uint8_t *smem_p = smem_b + S * B_STAGE_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + size_t(S) * Cfg::STAGE_BYTES);
+    uint64_t *full = bars;            // operands ready for the MMA
+    uint64_t *empty = bars + S;       // MMA finished reading the stage
+    uint64_t *pfull = bars + 2 * S;   // W4: packed tile + x1 tile landed
+    uint64_t *tfull = bars + 3 * S;   // accumulator buffer ready for the epilogue
+    uint64_t *tempty = tfull + 2;     // epilogue drained the accumulator buffer
+    uint64_t *drain = tempty + 2;     // all issued MMAs completed
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + Cfg::NUM_BARS);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    int32_t *off = reinterpret_cast<int32_t *>(smem + size_t(S) * Cfg::STAGE_BYTES + Cfg::CTRL_BYTES);
+    int32_t *cum = off + (MAX_E + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            ptx::mbar_init(&full[s], W4 ? 4 : 1);
+            ptx::mbar_init(&empty[s], 1);
+            ptx::mbar_init(&pfull[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&tfull[b], 1);
+            ptx::mbar_init(&tempty[b], 4);
+        }
+        ptx::mbar_init(drain, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0) {
+        const uint32_t flags = decode_groups_warp(args.group_list, args.e, args.group_list_type, args.m,
+                                                  args.tile_rows, off, cum);
+        if (lane == 0) {
+            if (flags && blockIdx.x == 0) atomicOr(args.status, flags);
+            ptx::prefetch_tmap(&map_a);
+            ptx::prefetch_tmap(&map_b);
+        }
+    } else if (warp == 1) {
+        ptx::tmem_alloc(tmem_holder, TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    const int e = args.e;
+    const int MT = cum[e];
+    const int NT = args.n / BN;
+    const int SW = args.slab_ntiles;
+    const int T = MT * NT;
+    const int KB = args.k / BK;
+    const int tile_rows = args.tile_rows;
+
+    auto fail = [&]() {
+        atomicOr(args.status, QGMM_DEV_TIMEOUT);
+        *abort_flag = 1;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            const uint32_t a_bytes = static_cast<uint32_t>(tile_rows) * BK;
+            uint32_t issued[S];
+#pragma unroll
+            for (int s = 0; s < S; ++s) issued[s] = 0;
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < T && ok; t += gridDim.x) {
+                const TileCoord c = tile_coord(t, MT, SW, off, cum, e, tile_rows);
+                const int n0 = c.nt * BN;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+                        fail();
+                        ok = false;
+                        break;
+                    }
+                    if constexpr (W4) {
+                        ptx::mbar_arrive_expect_tx(&pfull[stage], a_bytes + P_STAGE_BYTES);
+                        ptx::tma_load_2d(smem_a + stage * A_STAGE_BYTES, &map_a, &pfull[stage], kb * BK, c.row0);
+                        ptx::tma_load_3d(smem_p + stage * P_STAGE_BYTES, &map_b, &pfull[stage], n0 / 8, kb * BK,
+                                         c.g);
+                    } else {
+                        ptx::mbar_arrive_expect_tx(&full[stage], a_bytes + B_STAGE_BYTES);
+                        ptx::tma_load_2d(smem_a + stage * A_STAGE_BYTES, &map_a, &full[stage], kb * BK, c.row0);
+                        uint8_t *b = smem_b + stage * B_STAGE_BYTES;
+                        ptx::tma_load_3d(b, &map_b, &full[stage], n0, kb * BK, c.g);
+                        ptx::tma_load_3d(b + B_ATOM_BYTES, &map_b, &full[stage], n0 + 128, kb * BK, c.g);
+                    }
+                    ++issued[stage];
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // let the copies already in flight land before the CTA leaves
+                for (int s = 0; s < S; ++s) {
+                    if (issued[s] == 0) continue;
+                    uint64_t *bar = W4 ? &pfull[s] : &full[s];
+                    const uint32_t par = (issued[s] - 1u) & 1u;
+                    volatile int never = 0;
+                    ptx::mbar_wait(bar, par, &never);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC = ptx::idesc_i8(BM, BN, true);
+            int stage = 0;
+            uint32_t phase = 0;
+            int lt = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < T && ok; t += gridDim.x, ++lt) {
+                const int buf = lt & 1;
+                const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
+                if (!ptx::mbar_wait(&tempty[buf], use ^ 1u, abort_flag)) {
+                    fail();
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!ptx::mbar_wait(&full[stage], phase, abort_flag)) {
+                        fail();
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t a0 = ptx::smem_addr(smem_a + stage * A_STAGE_BYTES);
+                    const uint32_t b0 = ptx::smem_addr(smem_b + stage * B_STAGE_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+                        // A: K-major, 128-byte rows, 8-row groups 1024 B apart; step K by 32 bytes
+                        const uint64_t adesc = ptx::smem_desc_sw128(a0 + kk * UMMA_K, 16, 1024);
+                        // B: MN-major, 128-column atoms B_ATOM_BYTES apart, 8-row K groups 1024 B apart
+                        const uint64_t bdesc = ptx::smem_desc_sw128(b0 + kk * UMMA_K * 128, B_ATOM_BYTES, 1024);
+                        ptx::mma_i8(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    ptx::mma_commit(&empty[stage]);
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (ok) ptx::mma_commit(&tfull[buf]);
+            }
+            ptx::mma_commit(drain);
+            volatile int never = 0;
+            ptx::mbar_wait(drain, 0, &never);
+        }
+        __syncwarp();
+    } else if (warp < 6) {
+        // ------------------------------------------------ epilogue (TMEM -> registers -> global)
+        const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        const int r_in = q * 32 + lane;         // accumulator row of this thread
+        const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+        const int n = args.n;
+        int lt = 0;
+        for (int t = blockIdx.x; t < T; t += gridDim.x, ++lt) {
+            const TileCoord c = tile_coord(t, MT, SW, off, cum, e, tile_rows);
+            const int buf = lt & 1;
+            const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
+            if (!ptx::mbar_wait(&tfull[buf], use, abort_flag)) {
+                fail();
+                break;
+            }
+            ptx::tc_fence_after();
+            const int64_t i = static_cast<int64_t>(c.row0) + r_in;
+            bool valid = r_in < tile_rows && i < c.row_end;
+            const int n0 = c.nt * BN;
+            float pts = 1.0f, lg = 1.0f;
+            int64_t dst = i;
+            if (valid) {
+                if (args.pts) pts = __ldg(args.pts + i);
+                if (args.logit) lg = __ldg(args.logit + i);
+                if (EPI == EPI_ATOMIC) {
+                    dst = load_row_index(args.row_index, args.row_index_type, i);
+                    if (dst < 0 || dst >= args.output_bs) {
+                        atomicOr(args.status, QGMM_DEV_ROW_INDEX_RANGE);
+                        valid = false;
+                    }
+                }
+            }
+            if (__any_sync(0xffffffffu, valid)) {
+                const float *sc_row = args.scale ? args.scale + static_cast<int64_t>(c.g) * n + n0 : nullptr;
+                const float *bs_row = args.bias ? args.bias + static_cast<int64_t>(c.g) * n + n0 : nullptr;
+#pragma unroll 1
+                for (int cc = 0; cc < BN; cc += 16) {
+                    uint32_t r[16];
+                    __syncwarp();
+                    ptx::tmem_ld_32x32b_x16(tmem_base + lane_addr + static_cast<uint32_t>(buf * BN + cc), r);
+                    ptx::tmem_ld_wait(r);
+                    if (!valid) {
+                        // this row is masked; the warp still reads TMEM in lockstep
+                    } else if constexpr (EPI == EPI_RAW_ACC) {
+                        int4 *o = reinterpret_cast<int4 *>(args.acc_out + i * n + n0 + cc);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            o[v] = make_int4(static_cast<int>(r[4 * v]), static_cast<int>(r[4 * v + 1]),
+                                             static_cast<int>(r[4 * v + 2]), static_cast<int>(r[4 * v + 3]));
+                    } else {
+                        float y[16];
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            float4 s4 = make_float4(1.f, 1.f, 1.f, 1.f);
+                            float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                            if (sc_row) s4 = __ldg(reinterpret_cast<const float4 *>(sc_row + cc) + v);
+                            if (bs_row) b4 = __ldg(reinterpret_cast<const float4 *>(bs_row + cc) + v);
+                            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+                            const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                float x = __int2float_rn(static_cast<int>(r[4 * v + u]));
+                                x = __fmul_rn(x, sv[u]);
+                                x = __fmul_rn(x, pts);
+                                x = __fadd_rn(x, bv[u]);
+                                y[4 * v + u] = __fmul_rn(x, lg);
+                            }
+                        }
+                        if constexpr (EPI == EPI_ATOMIC) {
+                            float *o = args.out + dst * n + n0 + cc;
+#pragma unroll
+                            for (int v = 0; v < 4; ++v)
+                                ptx::red_add_v4(o + 4 * v, y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]);
+                        } else {
+                            float4 *o = reinterpret_cast<float4 *>(args.out + i * n + n0 + cc);
+#pragma unroll
+                            for (int v = 0; v < 4; ++v)
+                                o[v] = make_float4(y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]);
+                        }
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
+        }
+    } else if constexpr (W4) {
+        // ------------------------------------------------ int4 -> int8 unpack into the MN-major B tile
+        const int ut = threadIdx.x - 6 * 32;    // 0..127
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < T && ok; t += gridDim.x) {
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!ptx::mbar_wait(&pfull[stage], phase, abort_flag)) {
+                    fail();
+                    ok = false;
+                    break;
+                }
+                const uint8_t *p = smem_p + stage * P_STAGE_BYTES;
+                uint8_t *b = smem_b + stage * B_STAGE_BYTES;
+                const int qc = ut & 7;          // 16-byte packed chunk of the row: columns 32*qc .. 32*qc+31
+#pragma unroll
+                for (int it = 0; it < 8; ++it) {
+                    const int kr = (ut >> 3) + 16 * it;   // k row within the stage
+                    const uint4 w = *reinterpret_cast<const uint4 *>(p + kr * 128 + qc * 16);
+                    uint4 o0, o1;
+                    unpack_int4x8(w.x, o0.x, o0.y);
+                    unpack_int4x8(w.y, o0.z, o0.w);
+                    unpack_int4x8(w.z, o1.x, o1.y);
+                    unpack_int4x8(w.w, o1.z, o1.w);
+                    const int atom = qc >> 2;                 // 128-column atom
+                    const int c0 = (2 * qc) & 7;              // 16-column chunk inside the atom
+                    uint8_t *rowp = b + atom * B_ATOM_BYTES + kr * 128;
+                    *reinterpret_cast<uint4 *>(rowp + ((c0 ^ (kr & 7)) << 4)) = o0;
+                    *reinterpret_cast<uint4 *>(rowp + (((c0 + 1) ^ (kr & 7)) << 4)) = o1;
+                }
+                ptx::fence_async_shared();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&full[stage]);
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- K1
+// out[r][:] = f32(shared[r - off][:]) for r in [off, off + bs), else 0.  Also
+// clears the call's status word.  One float4 (four columns) per thread step.
+__global__ void output_init_kernel(float *__restrict__ out, int64_t output_bs, int32_t n,
+                                   const uint16_t *__restrict__ shared, int64_t shared_bs, int64_t shared_off,
+                                   uint32_t *status)
+{
+    if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
+    const int64_t q_per_row = n / 4;
+    const int64_t total = output_bs * q_per_row;
+    for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total;
+         idx += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t r = idx / q_per_row;
+        const int64_t c4 = idx - r * q_per_row;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (shared && r >= shared_off && r < shared_off + shared_bs) {
+            const uint2 h = __ldg(reinterpret_cast<const uint2 *>(shared + (r - shared_off) * n) + c4);
+            v.x = __uint_as_float(h.x << 16);
+            v.y = __uint_as_float(h.x & 0xFFFF0000u);
+            v.z = __uint_as_float(h.y << 16);
+            v.w = __uint_as_float(h.y & 0xFFFF0000u);
+        }
+        reinterpret_cast<float4 *>(out)[idx] = v;
+    }
+}
+
+__global__ void clear_status_kernel(uint32_t *status)
+{
+    *status = 0u;
+}
+
+// ---------------------------------------------------------------- K3 (deterministic combine)
+// Workspace: counts[output_bs] (histogram, then fill cursor), starts[output_bs+1], list[m].
+__global__ void det_clear_kernel(int32_t *counts, int64_t output_bs, uint32_t *status)
+{
+    if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
+    for (int64_t r = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; r < output_bs;
+         r += int64_t(gridDim.x) * blockDim.x)
+        counts[r] = 0;
+}
+
+// Shared by the histogram and fill kernels: rows below the total (from groupList).
+__device__ __forceinline__ int64_t groups_total_block(const int64_t *gl, int e, int type, int64_t m, int32_t *off,
+                                                      int32_t *cum, uint32_t *status, bool report)
+{
+    if (threadIdx.x < 32) {
+        const uint32_t f = decode_groups_warp(gl, e, type, m, BM, off, cum);
+        if (threadIdx.x == 0 && report && f) atomicOr(status, f);
+    }
+    __syncthreads();
+    return off[e];
+}
+
+__global__ void det_hist_kernel(const int64_t *gl, int e, int type, int64_t m, const void *row_index, int ri_type,
+                                int64_t output_bs, int32_t *counts, uint32_t *status)
+{
+    __shared__ int32_t off[MAX_E + 1], cum[MAX_E + 1];
+    const int64_t total = groups_total_block(gl, e, type, m, off, cum, status, blockIdx.x == 0);
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t d = load_row_index(row_index, ri_type, i);
+        if (d < 0 || d >= output_bs) {
+            atomicOr(status, QGMM_DEV_ROW_INDEX_RANGE);
+            continue;
+        }
+        atomicAdd(counts + d, 1);
+    }
+}
+
+// Single block: exclusive scan of counts into starts; counts becomes the fill cursor.
+__global__ void det_scan_kernel(int32_t *counts, int32_t *starts, int64_t output_bs)
+{
+    __shared__ int32_t warp_sums[32];
+    __shared__ int32_t carry;
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int64_t base = 0; base < output_bs; base += blockDim.x) {
+        const int64_t r = base + threadIdx.x;
+        const int32_t v = r < output_bs ? counts[r] : 0;
+        int32_t s = v;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int32_t o = __shfl_up_sync(0xffffffffu, s, d);
+            if (lane >= d) s += o;
+        }
+        if (lane == 31) warp_sums[w] = s;
+        __syncthreads();
+        if (w == 0) {
+            int32_t ws = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int32_t o = __shfl_up_sync(0xffffffffu, ws, d);
+                if (lane >= d) ws += o;
+            }
+            if (lane < nw) warp_sums[lane] = ws;
+        }
+        __syncthreads();
+        const int32_t excl = carry + (w ? warp_sums[w - 1] : 0) + s - v;
+        if (r < output_bs) {
+            starts[r] = excl;
+            counts[r] = excl;
+        }
+        __syncthreads();
+        if (threadIdx.x == blockDim.x - 1) carry = excl + v;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) starts[output_bs] = carry;
+}
+
+__global__ void det_fill_kernel(const int64_t *gl, int e, int type, int64_t m, const void *row_index, int ri_type,
+                                int64_t output_bs, int32_t *cursor, int32_t *list)
+{
+    __shared__ int32_t off[MAX_E + 1], cum[MAX_E + 1];
+    const int64_t total = groups_total_block(gl, e, type, m, off, cum, nullptr, false);
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t d = load_row_index(row_index, ri_type, i);
+        if (d < 0 || d >= output_bs) continue;
+        const int32_t pos = atomicAdd(cursor + d, 1);
+        list[pos] = static_cast<int32_t>(i);
+    }
+}
+
+// Sort each destination's source rows ascending (buckets hold about topK rows).
+__global__ void det_sort_kernel(const int32_t *starts, int32_t *list, int64_t output_bs)
+{
+    for (int64_t r = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; r < output_bs;
+         r += int64_t(gridDim.x) * blockDim.x) {
+        const int32_t a = starts[r], b = starts[r + 1];
+        for (int32_t x = a + 1; x < b; ++x) {
+            const int32_t v = list[x];
+            int32_t y = x - 1;
+            while (y >= a && list[y] > v) {
+                list[y + 1] = list[y];
+                --y;
+            }
+            list[y + 1] = v;
+        }
+    }
+}
+
+// out[r][:] = shared-or-0, then += y[j][:] for the bucket's rows j in ascending order.
+__global__ void det_reduce_kernel(float *__restrict__ out, const float *__restrict__ y, int32_t n,
+                                  const int32_t *__restrict__ starts, const int32_t *__restrict__ list,
+                                  int64_t output_bs, const uint16_t *__restrict__ shared, int64_t shared_bs,
+                                  int64_t shared_off)
+{
+    const int32_t q_per_row = n / 4;
+    for (int64_t r = blockIdx.x; r < output_bs; r += gridDim.x) {
+        const int32_t a = starts[r], b = starts[r + 1];
+        const bool sh = shared && r >= shared_off && r < shared_off + shared_bs;
+        for (int32_t c4 = threadIdx.x; c4 < q_per_row; c4 += blockDim.x) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (sh) {
+                const uint2 h = __ldg(reinterpret_cast<const uint2 *>(shared + (r - shared_off) * n) + c4);
+                acc.x = __uint_as_float(h.x << 16);
+                acc.y = __uint_as_float(h.x & 0xFFFF0000u);
+                acc.z = __uint_as_float(h.y << 16);
+                acc.w = __uint_as_float(h.y & 0xFFFF0000u);
+            }
+            for (int32_t x = a; x < b; ++x) {
+                const float4 v = __ldg(reinterpret_cast<const float4 *>(y + int64_t(list[x]) * n) + c4);
+                acc.x = __fadd_rn(acc.x, v.x);
+                acc.y = __fadd_rn(acc.y, v.y);
+                acc.z = __fadd_rn(acc.z, v.z);
+                acc.w = __fadd_rn(acc.w, v.w);
+            }
+            reinterpret_cast<float4 *>(out + r * n)[c4] = acc;
+        }
+    }
+}
+
+// ---------------------------------------------------------------- K0
+// One warp per row: absmax over the row, then q = clamp(rn(x * (127/a)), +-127)
+// and scale = a / 127, all in IEEE f32 (page 4, per_token_cast: value times a
+// precomputed inverse).  k % 8 == 0; 16-byte vector loads, 8-byte stores.
+__global__ void per_token_quant_kernel(const uint16_t *__restrict__ x, int64_t rows, int32_t k, int8_t *__restrict__ q,
+                                       float *__restrict__ scale_out)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warps_total = int64_t(gridDim.x) * (blockDim.x >> 5);
+    const int32_t v_per_row = k / 8;
+    for (int64_t row = blockIdx.x * int64_t(blockDim.x >> 5) + (threadIdx.x >> 5); row < rows; row += warps_total) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + row * k);
+        float a = 0.f;
+        for (int32_t v = lane; v < v_per_row; v += 32) {
+            const uint4 h = __ldg(src + v);
+            const uint32_t w[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                a = fmaxf(a, fabsf(__uint_as_float(w[u] << 16)));
+                a = fmaxf(a, fabsf(__uint_as_float(w[u] & 0xFFFF0000u)));
+            }
+        }
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, d));
+        const float inv = a > 0.f ? __fdiv_rn(127.0f, a) : 0.0f;
+        if (lane == 0) scale_out[row] = __fdiv_rn(a, 127.0f);
+        uint2 *dst = reinterpret_cast<uint2 *>(q + row * k);
+        for (int32_t v = lane; v < v_per_row; v += 32) {
+            const uint4 h = __ldg(src + v);
+            const uint32_t w[4] = {h.x, h.y, h.z, h.w};
+            uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float f0 = __uint_as_float(w[u] << 16);
+                const float f1 = __uint_as_float(w[u] & 0xFFFF0000u);
+                float r0 = rintf(__fmul_rn(f0, inv));
+                float r1 = rintf(__fmul_rn(f1, inv));
+                r0 = fminf(fmaxf(r0, -127.0f), 127.0f);
+                r1 = fminf(fmaxf(r1, -127.0f), 127.0f);
+                const uint32_t b0 = static_cast<uint32_t>(static_cast<int32_t>(r0)) & 0xFFu;
+                const uint32_t b1 = static_cast<uint32_t>(static_cast<int32_t>(r1)) & 0xFFu;
+                packed[u >> 1] |= (b0 | (b1 << 8)) << (16 * (u & 1));
+            }
+            dst[v] = make_uint2(packed[0], packed[1]);
+        }
+    }
+}
+
+}  // namespace qgmm

@@ -1,0 +1,399 @@
+// qgmm.cu -- host side of libqgmm.so: argument checks, workspace sizing, tile
+// planning, TMA tensor maps and kernel launches for the C ABI in qgmm.h.
+//
+// Two-stage call as on the "aclnnGroupedMatmulFinalizeRoutingWeightNzV2" page
+// (first call validates and sizes the workspace, second call runs on a
+// stream).  The library allocates no memory and keeps no per-call state.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.cuh"
+
+#define QGMM_API extern "C" __attribute__((visibility("default")))
+
+namespace qgmm {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int64_t kMaxM = int64_t(1) << 24;
+constexpr int kMaxDevices = 64;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct DeviceInfo {
+    int sms = 0;
+    int major = 0;
+    bool attr_set[3][2] = {};
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+qgmm_status device_info(DeviceInfo **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QGMM_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (d.sms == 0) {
+        int sms = 0, major = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return QGMM_ERR_CUDA;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+            return QGMM_ERR_CUDA;
+        d.sms = sms;
+        d.major = major;
+    }
+    if (d.major != 10) return QGMM_ERR_UNSUPPORTED;
+    *out = &d;
+    return QGMM_OK;
+}
+
+qgmm_status check_problem(const qgmm_problem *p)
+{
+    if (!p) return QGMM_ERR_NULL_PTR;
+    if (p->weight_type != QGMM_W_INT8 && p->weight_type != QGMM_W_INT4_PACKED_INT32) return QGMM_ERR_DTYPE;
+    if (p->group_list_type != QGMM_GROUP_CUMSUM && p->group_list_type != QGMM_GROUP_COUNTS) return QGMM_ERR_DTYPE;
+    if (p->row_index_type != QGMM_IDX_INT64 && p->row_index_type != QGMM_IDX_INT32) return QGMM_ERR_DTYPE;
+    if (p->m < 1 || p->m > kMaxM) return QGMM_ERR_SHAPE;
+    if (p->k < BK || p->k > 65536 || p->k % BK) return QGMM_ERR_SHAPE;
+    if (p->n < BN || p->n > 65536 || p->n % BN) return QGMM_ERR_SHAPE;
+    if (p->e < 1 || p->e > MAX_E) return QGMM_ERR_SHAPE;
+    if (p->output_bs < 1 || p->output_bs > (int64_t(1) << 31) - 2) return QGMM_ERR_SHAPE;
+    if (p->shared_bs < 0 || p->shared_offset < 0 || p->shared_offset + p->shared_bs > p->output_bs)
+        return QGMM_ERR_SHAPE;
+    if (p->deterministic != 0 && p->deterministic != 1) return QGMM_ERR_SHAPE;
+    if (p->expected_m_per_expert < 0) return QGMM_ERR_SHAPE;
+    return QGMM_OK;
+}
+
+struct DetLayout {
+    size_t y, counts, starts, list, total;
+};
+
+DetLayout det_layout(const qgmm_problem *p)
+{
+    DetLayout L;
+    L.y = kAlign;
+    L.counts = L.y + align_up(size_t(p->m) * size_t(p->n) * 4);
+    L.starts = L.counts + align_up(size_t(p->output_bs) * 4);
+    L.list = L.starts + align_up(size_t(p->output_bs + 1) * 4);
+    L.total = L.list + align_up(size_t(p->m) * 4);
+    return L;
+}
+
+size_t workspace_bytes(const qgmm_problem *p)
+{
+    return p->deterministic ? det_layout(p).total : kAlign;
+}
+
+int env_int(const char *name, int dflt)
+{
+    const char *v = std::getenv(name);
+    if (!v || !*v) return dflt;
+    return std::atoi(v);
+}
+
+struct Plan {
+    int tile_rows;
+    int slab_ntiles;
+    int grid;
+};
+
+Plan make_plan(const qgmm_problem *p, int sms, int epi)
+{
+    Plan pl;
+    const int64_t hint = p->expected_m_per_expert > 0 ? p->expected_m_per_expert : (p->m + p->e - 1) / p->e;
+    pl.tile_rows = hint <= 16 ? 16 : hint <= 32 ? 32 : hint <= 64 ? 64 : 128;
+    const int forced_rows = env_int("QGMM_TILE_ROWS", 0);
+    if (forced_rows == 16 || forced_rows == 32 || forced_rows == 64 || forced_rows == 128) pl.tile_rows = forced_rows;
+
+    const int NT = static_cast<int>(p->n / BN);
+    int sw = NT;
+    if (epi == EPI_ATOMIC) {
+        // keep one slab of the output (output_bs x slab columns, f32) within ~48 MB of L2
+        const double per_ntile = double(p->output_bs) * BN * 4.0;
+        const double budget = 48.0 * 1024 * 1024;
+        sw = 1;
+        for (int d = 1; d <= NT; ++d)
+            if (NT % d == 0 && d * per_ntile <= budget) sw = d;
+    }
+    const int forced_sw = env_int("QGMM_SLAB_NTILES", 0);
+    if (forced_sw > 0 && forced_sw <= NT && NT % forced_sw == 0) sw = forced_sw;
+    pl.slab_ntiles = sw;
+
+    const int64_t max_mt = (p->m + pl.tile_rows - 1) / pl.tile_rows + p->e;
+    const int64_t max_tiles = max_mt * NT;
+    pl.grid = static_cast<int>(max_tiles < sms ? max_tiles : sms);
+    if (pl.grid < 1) pl.grid = 1;
+    return pl;
+}
+
+qgmm_status make_maps(const qgmm_problem *p, const int8_t *x1, const void *x2, int tile_rows, CUtensorMap *ma,
+                      CUtensorMap *mb)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return QGMM_ERR_CUDA;
+    {
+        const cuuint64_t gdim[2] = {cuuint64_t(p->k), cuuint64_t(p->m)};
+        const cuuint64_t gstride[1] = {cuuint64_t(p->k)};
+        const cuuint32_t box[2] = {cuuint32_t(BK), cuuint32_t(tile_rows)};
+        const cuuint32_t es[2] = {1, 1};
+        if (enc(ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(x1), gdim, gstride, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return QGMM_ERR_CUDA;
+    }
+    if (p->weight_type == QGMM_W_INT8) {
+        const cuuint64_t gdim[3] = {cuuint64_t(p->n), cuuint64_t(p->k), cuuint64_t(p->e)};
+        const cuuint64_t gstride[2] = {cuuint64_t(p->n), cuuint64_t(p->n) * cuuint64_t(p->k)};
+        const cuuint32_t box[3] = {128, cuuint32_t(BK), 1};
+        const cuuint32_t es[3] = {1, 1, 1};
+        if (enc(mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(x2), gdim, gstride, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return QGMM_ERR_CUDA;
+    } else {
+        const cuuint64_t words = cuuint64_t(p->n / 8);
+        const cuuint64_t gdim[3] = {words, cuuint64_t(p->k), cuuint64_t(p->e)};
+        const cuuint64_t gstride[2] = {words * 4, words * 4 * cuuint64_t(p->k)};
+        const cuuint32_t box[3] = {32, cuuint32_t(BK), 1};
+        const cuuint32_t es[3] = {1, 1, 1};
+        if (enc(mb, CU_TENSOR_MAP_DATA_TYPE_INT32, 3, const_cast<void *>(x2), gdim, gstride, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return QGMM_ERR_CUDA;
+    }
+    return QGMM_OK;
+}
+
+template <int EPI, bool W4>
+qgmm_status launch_gemm_t(DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma, const CUtensorMap &mb,
+                          const GemmArgs &a, cudaStream_t st)
+{
+    auto kern = grouped_gemm_kernel<EPI, W4>;
+    const size_t smem = GemmCfg<W4>::SMEM_BYTES;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!dev->attr_set[EPI][W4 ? 1 : 0]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+                return QGMM_ERR_CUDA;
+            dev->attr_set[EPI][W4 ? 1 : 0] = true;
+        }
+    }
+    kern<<<pl.grid, GemmCfg<W4>::THREADS, smem, st>>>(ma, mb, a);
+    return cudaGetLastError() == cudaSuccess ? QGMM_OK : QGMM_ERR_CUDA;
+}
+
+qgmm_status launch_gemm(int epi, DeviceInfo *dev, const qgmm_problem *p, const Plan &pl, const CUtensorMap &ma,
+                        const CUtensorMap &mb, const GemmArgs &a, cudaStream_t st)
+{
+    const bool w4 = p->weight_type == QGMM_W_INT4_PACKED_INT32;
+    if (std::getenv("QGMM_LOG"))
+        std::fprintf(stderr, "qgmm: gemm epi=%d w4=%d m=%lld k=%lld n=%lld e=%lld tile_rows=%d slab=%d grid=%d\n", epi,
+                     int(w4), (long long)p->m, (long long)p->k, (long long)p->n, (long long)p->e, pl.tile_rows,
+                     pl.slab_ntiles, pl.grid);
+    switch (epi) {
+    case EPI_ATOMIC: return w4 ? launch_gemm_t<EPI_ATOMIC, true>(dev, pl, ma, mb, a, st)
+                               : launch_gemm_t<EPI_ATOMIC, false>(dev, pl, ma, mb, a, st);
+    case EPI_STORE_Y: return w4 ? launch_gemm_t<EPI_STORE_Y, true>(dev, pl, ma, mb, a, st)
+                                : launch_gemm_t<EPI_STORE_Y, false>(dev, pl, ma, mb, a, st);
+    default: return w4 ? launch_gemm_t<EPI_RAW_ACC, true>(dev, pl, ma, mb, a, st)
+                       : launch_gemm_t<EPI_RAW_ACC, false>(dev, pl, ma, mb, a, st);
+    }
+}
+
+GemmArgs base_args(const qgmm_problem *p, const int64_t *group_list, const Plan &pl, uint32_t *status)
+{
+    GemmArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.group_list = group_list;
+    a.m = p->m;
+    a.e = static_cast<int32_t>(p->e);
+    a.group_list_type = p->group_list_type;
+    a.k = static_cast<int32_t>(p->k);
+    a.n = static_cast<int32_t>(p->n);
+    a.tile_rows = pl.tile_rows;
+    a.slab_ntiles = pl.slab_ntiles;
+    a.row_index_type = p->row_index_type;
+    a.output_bs = p->output_bs;
+    a.status = status;
+    return a;
+}
+
+int grid_for(int64_t work, int per_block, int sms, int blocks_per_sm)
+{
+    int64_t g = (work + per_block - 1) / per_block;
+    const int64_t cap = int64_t(sms) * blocks_per_sm;
+    if (g > cap) g = cap;
+    if (g < 1) g = 1;
+    return static_cast<int>(g);
+}
+
+}  // namespace
+}  // namespace qgmm
+
+using namespace qgmm;
+
+QGMM_API qgmm_status qgmm_finalize_workspace(const qgmm_problem *p, size_t *ws_bytes)
+{
+    if (!ws_bytes) return QGMM_ERR_NULL_PTR;
+    const qgmm_status s = check_problem(p);
+    if (s != QGMM_OK) return s;
+    *ws_bytes = workspace_bytes(p);
+    return QGMM_OK;
+}
+
+QGMM_API qgmm_status qgmm_finalize(const qgmm_problem *p, const int8_t *x1, const void *x2, const float *scale,
+                                   const float *pertoken_scale, const int64_t *group_list, const float *logit,
+                                   const void *row_index, const float *bias, const uint16_t *shared_input,
+                                   float *out, void *workspace, size_t ws_bytes, void *cuda_stream)
+{
+    qgmm_status s = check_problem(p);
+    if (s != QGMM_OK) return s;
+    if (!x1 || !x2 || !group_list || !out || !workspace) return QGMM_ERR_NULL_PTR;
+    if (p->shared_bs > 0 && !shared_input) return QGMM_ERR_NULL_PTR;
+    if (!aligned16(x1) || !aligned16(x2) || !aligned16(out) || (p->shared_bs > 0 && !aligned16(shared_input)) ||
+        (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || !aligned16(scale) || !aligned16(bias))
+        return QGMM_ERR_ALIGNMENT;
+    if (ws_bytes < workspace_bytes(p)) return QGMM_ERR_WORKSPACE_TOO_SMALL;
+    DeviceInfo *dev = nullptr;
+    if ((s = device_info(&dev)) != QGMM_OK) return s;
+
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    uint32_t *status = static_cast<uint32_t *>(workspace);
+    const int epi = p->deterministic ? EPI_STORE_Y : EPI_ATOMIC;
+    const Plan pl = make_plan(p, dev->sms, epi);
+    CUtensorMap ma, mb;
+    if ((s = make_maps(p, x1, x2, pl.tile_rows, &ma, &mb)) != QGMM_OK) return s;
+
+    GemmArgs a = base_args(p, group_list, pl, status);
+    a.scale = scale;
+    a.pts = pertoken_scale;
+    a.logit = logit;
+    a.bias = bias;
+    a.row_index = row_index;
+    const uint16_t *shared = p->shared_bs > 0 ? shared_input : nullptr;
+
+    if (!p->deterministic) {
+        const int64_t quads = p->output_bs * (p->n / 4);
+        output_init_kernel<<<grid_for(quads, 256, dev->sms, 8), 256, 0, st>>>(
+            out, p->output_bs, static_cast<int32_t>(p->n), shared, p->shared_bs, p->shared_offset, status);
+        if (cudaGetLastError() != cudaSuccess) return QGMM_ERR_CUDA;
+        a.out = out;
+        return launch_gemm(EPI_ATOMIC, dev, p, pl, ma, mb, a, st);
+    }
+
+    const DetLayout L = det_layout(p);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *y = reinterpret_cast<float *>(ws + L.y);
+    int32_t *counts = reinterpret_cast<int32_t *>(ws + L.counts);
+    int32_t *starts = reinterpret_cast<int32_t *>(ws + L.starts);
+    int32_t *list = reinterpret_cast<int32_t *>(ws + L.list);
+    const int e = static_cast<int>(p->e);
+    det_clear_kernel<<<grid_for(p->output_bs, 256, dev->sms, 4), 256, 0, st>>>(counts, p->output_bs, status);
+    det_hist_kernel<<<grid_for(p->m, 256, dev->sms, 4), 256, 0, st>>>(
+        group_list, e, p->group_list_type, p->m, row_index, p->row_index_type, p->output_bs, counts, status);
+    det_scan_kernel<<<1, 1024, 0, st>>>(counts, starts, p->output_bs);
+    det_fill_kernel<<<grid_for(p->m, 256, dev->sms, 4), 256, 0, st>>>(
+        group_list, e, p->group_list_type, p->m, row_index, p->row_index_type, p->output_bs, counts, list);
+    det_sort_kernel<<<grid_for(p->output_bs, 256, dev->sms, 4), 256, 0, st>>>(starts, list, p->output_bs);
+    if (cudaGetLastError() != cudaSuccess) return QGMM_ERR_CUDA;
+    a.out = y;
+    if ((s = launch_gemm(EPI_STORE_Y, dev, p, pl, ma, mb, a, st)) != QGMM_OK) return s;
+    det_reduce_kernel<<<grid_for(p->output_bs, 1, dev->sms, 8), 256, 0, st>>>(
+        out, y, static_cast<int32_t>(p->n), starts, list, p->output_bs, shared, p->shared_bs, p->shared_offset);
+    return cudaGetLastError() == cudaSuccess ? QGMM_OK : QGMM_ERR_CUDA;
+}
+
+QGMM_API qgmm_status qgmm_debug_accum(const qgmm_problem *p, const int8_t *x1, const void *x2,
+                                      const int64_t *group_list, int32_t *acc_out, void *workspace,
+                                      size_t ws_bytes, void *cuda_stream)
+{
+    qgmm_status s = check_problem(p);
+    if (s != QGMM_OK) return s;
+    if (!x1 || !x2 || !group_list || !acc_out || !workspace) return QGMM_ERR_NULL_PTR;
+    if (!aligned16(x1) || !aligned16(x2) || !aligned16(acc_out) ||
+        (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+        return QGMM_ERR_ALIGNMENT;
+    if (ws_bytes < kAlign) return QGMM_ERR_WORKSPACE_TOO_SMALL;
+    DeviceInfo *dev = nullptr;
+    if ((s = device_info(&dev)) != QGMM_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    uint32_t *status = static_cast<uint32_t *>(workspace);
+    const Plan pl = make_plan(p, dev->sms, EPI_RAW_ACC);
+    CUtensorMap ma, mb;
+    if ((s = make_maps(p, x1, x2, pl.tile_rows, &ma, &mb)) != QGMM_OK) return s;
+    clear_status_kernel<<<1, 1, 0, st>>>(status);
+    if (cudaGetLastError() != cudaSuccess) return QGMM_ERR_CUDA;
+    GemmArgs a = base_args(p, group_list, pl, status);
+    a.acc_out = acc_out;
+    return launch_gemm(EPI_RAW_ACC, dev, p, pl, ma, mb, a, st);
+}
+
+QGMM_API qgmm_status qgmm_per_token_quant(const uint16_t *x_bf16, int64_t rows, int64_t k, int8_t *x1_out,
+                                          float *scale_out, void *cuda_stream)
+{
+    if (!x_bf16 || !x1_out || !scale_out) return QGMM_ERR_NULL_PTR;
+    if (rows < 1 || rows > (int64_t(1) << 31) - 1 || k < 8 || k > 65536 || k % 8) return QGMM_ERR_SHAPE;
+    if (!aligned16(x_bf16) || !aligned16(x1_out)) return QGMM_ERR_ALIGNMENT;
+    DeviceInfo *dev = nullptr;
+    qgmm_status s = device_info(&dev);
+    if (s != QGMM_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    per_token_quant_kernel<<<grid_for(rows, 8, dev->sms, 8), 256, 0, st>>>(x_bf16, rows, static_cast<int32_t>(k),
+                                                                           x1_out, scale_out);
+    return cudaGetLastError() == cudaSuccess ? QGMM_OK : QGMM_ERR_CUDA;
+}
+
+QGMM_API qgmm_status qgmm_device_status(const void *workspace, uint32_t *flags, void *cuda_stream)
+{
+    if (!workspace || !flags) return QGMM_ERR_NULL_PTR;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return QGMM_ERR_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpy(&v, workspace, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return QGMM_ERR_CUDA;
+    *flags = v;
+    return v ? QGMM_ERR_DEVICE_INPUT : QGMM_OK;
+}
+
+QGMM_API const char *qgmm_status_string(qgmm_status s)
+{
+    switch (s) {
+    case QGMM_OK: return "ok";
+    case QGMM_ERR_NULL_PTR: return "a required pointer is NULL";
+    case QGMM_ERR_SHAPE: return "a size is out of range";
+    case QGMM_ERR_DTYPE: return "unknown weight, row-index or group-list type";
+    case QGMM_ERR_WORKSPACE_TOO_SMALL: return "workspace smaller than qgmm_finalize_workspace reports";
+    case QGMM_ERR_UNSUPPORTED: return "device is not sm_100 (B200)";
+    case QGMM_ERR_CUDA: return "a CUDA call failed";
+    case QGMM_ERR_DEVICE_INPUT: return "the device found invalid group_list or row_index values";
+    case QGMM_ERR_ALIGNMENT: return "a pointer is not suitably aligned";
+    }
+    return "unknown status";
+}

@@ -34,3 +34,13 @@ def problem_cache():
             _PROBLEMS[key] = make_problem(name, **kw)
         return _PROBLEMS[key]
     return get
+
+
+@pytest.fixture(scope="session")
+def qgmm():
+    """The binding over the in-tree CUDA library (built here if missing or stale)."""
+    from quantized_moe_grouped_persistent_b200 import build
+    build.build()
+    import quantized_moe_grouped_persistent_b200 as q
+    q.lib()
+    return q

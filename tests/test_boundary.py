@@ -1,0 +1,167 @@
+"""The C ABI boundary, on the host: the library loads, exports every function
+``include/qgmm.h`` declares, its struct layout matches the binding, and every
+host-side check returns its documented code before anything is launched.
+
+No test here reaches a kernel launch: each call fails a host check first.
+"""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qgmm.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^(?:qgmm_status|const char \*)\s*(qgmm_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_abi():
+    assert _declared_functions() == sorted([
+        "qgmm_finalize_workspace", "qgmm_finalize", "qgmm_per_token_quant", "qgmm_debug_accum",
+        "qgmm_device_status", "qgmm_status_string"])
+
+
+def test_library_exports_every_declared_symbol(qgmm):
+    out = subprocess.run(["nm", "-D", "--defined-only", qgmm.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r" T (\w+)$", out, re.M))
+    for name in _declared_functions():
+        assert name in exported, name
+    # nothing but the C ABI is exported from the library's own code
+    assert {s for s in exported if s.startswith("qgmm")} == set(_declared_functions())
+
+
+def test_problem_struct_layout_matches_header(qgmm, tmp_path):
+    src = tmp_path / "layout.c"
+    src.write_text("""
+#include <stdio.h>
+#include <stddef.h>
+#include "qgmm.h"
+#define F(x) printf(#x " %zu\\n", offsetof(qgmm_problem, x));
+int main(void) {
+  printf("size %zu\\n", sizeof(qgmm_problem));
+  F(m) F(k) F(n) F(e) F(output_bs) F(weight_type) F(group_list_type) F(row_index_type)
+  F(shared_bs) F(shared_offset) F(deterministic) F(expected_m_per_expert)
+  return 0;
+}
+""")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    lines = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = dict(l.split() for l in lines if l)
+    P = qgmm.QgmmProblem
+    assert int(got["size"]) == C.sizeof(P)
+    for name, _ in P._fields_:
+        assert int(got[name]) == getattr(P, name).offset, name
+
+
+def _prob(qgmm, **kw):
+    base = dict(m=64, k=256, n=512, e=4, output_bs=32)
+    base.update(kw)
+    args = {k: base.pop(k) for k in ("m", "k", "n", "e", "output_bs")}
+    return qgmm.make_problem(args["m"], args["k"], args["n"], args["e"], args["output_bs"], **base)
+
+
+def _ws(qgmm, p):
+    out = C.c_size_t(0)
+    rc = qgmm.lib().qgmm_finalize_workspace(C.byref(p), C.byref(out))
+    return rc, out.value
+
+
+def test_workspace_sizes(qgmm):
+    rc, n = _ws(qgmm, _prob(qgmm))
+    assert rc == qgmm.QGMM_OK and n == 256
+    m, nn, obs = 64, 512, 32
+    rc, n = _ws(qgmm, _prob(qgmm, deterministic=True))
+    al = lambda v: (v + 255) // 256 * 256
+    assert rc == qgmm.QGMM_OK
+    assert n == 256 + al(m * nn * 4) + al(obs * 4) + al((obs + 1) * 4) + al(m * 4)
+    assert qgmm.finalize_workspace(_prob(qgmm, m=131072, k=2048, n=7168, e=256, output_bs=16384)) == 256
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(m=0), "SHAPE"), (dict(m=(1 << 24) + 1), "SHAPE"),
+    (dict(k=100), "SHAPE"), (dict(k=64), "SHAPE"), (dict(k=65536 + 128), "SHAPE"),
+    (dict(n=128), "SHAPE"), (dict(n=300), "SHAPE"), (dict(n=7168 + 128), "SHAPE"),
+    (dict(e=0), "SHAPE"), (dict(e=1025), "SHAPE"), (dict(output_bs=0), "SHAPE"),
+    (dict(shared_bs=33), "SHAPE"), (dict(shared_bs=8, shared_offset=25), "SHAPE"),
+    (dict(shared_offset=-1), "SHAPE"), (dict(expected_m_per_expert=-1), "SHAPE"),
+    (dict(weight_type=2), "DTYPE"), (dict(group_list_type=2), "DTYPE"), (dict(row_index_type=5), "DTYPE"),
+])
+def test_stage_one_rejects(qgmm, kw, code):
+    rc, _ = _ws(qgmm, _prob(qgmm, **kw))
+    assert rc == getattr(qgmm, "QGMM_ERR_" + code)
+
+
+def test_stage_one_accepts_page_limits(qgmm):
+    for kw in (dict(m=1), dict(m=131072, k=2048, n=7168, e=256), dict(e=1024), dict(k=65536),
+               dict(shared_bs=32, shared_offset=0), dict(shared_bs=8, shared_offset=24)):
+        assert _ws(qgmm, _prob(qgmm, **kw))[0] == qgmm.QGMM_OK, kw
+
+
+def test_null_arguments(qgmm):
+    L = qgmm.lib()
+    assert L.qgmm_finalize_workspace(None, None) == qgmm.QGMM_ERR_NULL_PTR
+    p = _prob(qgmm)
+    assert L.qgmm_finalize_workspace(C.byref(p), None) == qgmm.QGMM_ERR_NULL_PTR
+    fake = 1 << 20  # never dereferenced: every call below fails a host check
+    args = [fake, fake, None, None, fake, None, None, None, None, fake, fake, 256, None]
+    for idx in (0, 1, 4, 9, 10):   # x1, x2, group_list, out, workspace
+        a = list(args)
+        a[idx] = None
+        assert L.qgmm_finalize(C.byref(p), *a) == qgmm.QGMM_ERR_NULL_PTR, idx
+    ps = _prob(qgmm, shared_bs=4)
+    assert L.qgmm_finalize(C.byref(ps), *args) == qgmm.QGMM_ERR_NULL_PTR   # shared rows without a pointer
+    assert L.qgmm_finalize(None, *args) == qgmm.QGMM_ERR_NULL_PTR
+    assert L.qgmm_per_token_quant(None, 4, 64, fake, fake, None) == qgmm.QGMM_ERR_NULL_PTR
+    assert L.qgmm_debug_accum(C.byref(p), fake, fake, None, fake, fake, 256, None) == qgmm.QGMM_ERR_NULL_PTR
+    assert L.qgmm_device_status(None, None, None) == qgmm.QGMM_ERR_NULL_PTR
+
+
+def test_alignment_and_workspace_checks(qgmm):
+    L = qgmm.lib()
+    p = _prob(qgmm)
+    a16 = 1 << 20
+    for idx in (0, 1, 9):   # x1, x2, out misaligned
+        a = [a16, a16, None, None, a16, None, None, None, None, a16, a16, 256, None]
+        a[idx] = a16 + 8
+        assert L.qgmm_finalize(C.byref(p), *a) == qgmm.QGMM_ERR_ALIGNMENT, idx
+    a = [a16, a16, a16 + 4, None, a16, None, None, None, None, a16, a16, 256, None]   # scale misaligned
+    assert L.qgmm_finalize(C.byref(p), *a) == qgmm.QGMM_ERR_ALIGNMENT
+    a = [a16, a16, None, None, a16, None, None, None, None, a16, a16 + 16, 256, None]  # workspace not 256-aligned
+    assert L.qgmm_finalize(C.byref(p), *a) == qgmm.QGMM_ERR_ALIGNMENT
+    a = [a16, a16, None, None, a16, None, None, None, None, a16, a16, 255, None]
+    assert L.qgmm_finalize(C.byref(p), *a) == qgmm.QGMM_ERR_WORKSPACE_TOO_SMALL
+    pd = _prob(qgmm, deterministic=True)
+    a = [a16, a16, None, None, a16, None, None, None, None, a16, a16, 256, None]
+    assert L.qgmm_finalize(C.byref(pd), *a) == qgmm.QGMM_ERR_WORKSPACE_TOO_SMALL
+    assert L.qgmm_debug_accum(C.byref(p), a16, a16, a16, a16 + 4, a16, 256, None) == qgmm.QGMM_ERR_ALIGNMENT
+    assert L.qgmm_debug_accum(C.byref(p), a16, a16, a16, a16, a16, 128, None) == qgmm.QGMM_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_per_token_quant_host_checks(qgmm):
+    L = qgmm.lib()
+    a16 = 1 << 20
+    assert L.qgmm_per_token_quant(a16, 4, 12, a16, a16, None) == qgmm.QGMM_ERR_SHAPE   # k % 8
+    assert L.qgmm_per_token_quant(a16, 0, 64, a16, a16, None) == qgmm.QGMM_ERR_SHAPE
+    assert L.qgmm_per_token_quant(a16 + 2, 4, 64, a16, a16, None) == qgmm.QGMM_ERR_ALIGNMENT
+
+
+def test_status_strings(qgmm):
+    for code in range(9):
+        s = qgmm.status_string(code)
+        assert s and s != "unknown status"
+    assert qgmm.status_string(99) == "unknown status"
+
+
+def test_binding_raises_without_library(tmp_path, monkeypatch):
+    import quantized_moe_grouped_persistent_b200 as q
+    monkeypatch.setattr(q, "_lib", None)
+    monkeypatch.setattr(q, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        q.lib()
