@@ -1,0 +1,443 @@
+#!/usr/bin/env python
+"""Benchmark of the fused int8 GroupedMatmul + MoeFinalizeRouting op on B200.
+
+One step = one ``qgmm_finalize`` call (output init + persistent grouped GEMM
+with the fused dequant/combine epilogue; plus the per-token quant prologue on
+workloads that have one) over one batch of seeded synthetic inputs already
+resident in HBM.  Default workload: the large prefill (tokens=16384, topK=8,
+m=131072, e=256, k=2048, n=7168, Dirichlet(0.3) routing, bf16 sharedInput),
+atomic combine.  The metric is effective INT8 TOPS = 2 * sum_g m_g * k * n / t.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch
+(weak scaling, no collective on the data path); ``value`` is all ranks' work
+over the slowest rank's device time.
+
+``--impl reference`` times the CPU oracle instead, on a bounded sample of the
+same workload's output rows (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "effective INT8 TOPS and % of B200 dense INT8 peak; HBM GB/s at decode m"
+NOMINAL_INT8_TOPS = 4500.0
+NOMINAL_HBM_GBS = 8000.0
+KERNEL_SOURCES = ["quantized_moe_grouped_persistent_b200/csrc/kernels.cuh",
+                  "quantized_moe_grouped_persistent_b200/csrc/ptx_sm100.cuh"]
+TRAFFIC_SUMMARY = {
+    "large_prefill": "profiles/grouped_gemm_large_prefill.md",
+    "decode": "profiles/grouped_gemm_decode.md",
+}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="large_prefill")
+    ap.add_argument("--deterministic", action="store_true", help="time the fixed-order combine instead")
+    ap.add_argument("--no-extras", action="store_true", help="skip the decode / deterministic / e2e side runs")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sustained=d["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def kernel_sources_sha():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, rel), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload):
+    """DRAM bytes per launch of the grouped GEMM from the committed ncu summary, if still current."""
+    rel = TRAFFIC_SUMMARY.get(workload)
+    if not rel or not os.path.exists(os.path.join(ROOT, rel)):
+        return None
+    text = open(os.path.join(ROOT, rel)).read()
+    m_sha = re.search(r"kernel_sources_sha256:\s*([0-9a-f]+)", text)
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not m_sha or not m_b or m_sha.group(1) != kernel_sources_sha():
+        return None
+    return int(m_b.group(1))
+
+
+def total_rows(p):
+    return int(p.counts.sum())
+
+
+def int_ops(p):
+    return 2.0 * total_rows(p) * p.k * p.n
+
+
+def algorithmic_bytes(p):
+    """Bytes the step must move at least once: the used experts' weights (and their
+    scale/bias rows), x1 (or the bf16 activations), the per-row vectors, the output
+    written once, and the sharedInput read once."""
+    used = int((p.counts > 0).sum())
+    w_bytes = p.k * p.n if p.weight == "int8" else p.k * p.n // 2
+    per_expert = w_bytes + 4 * p.n + (4 * p.n if p.bias is not None else 0)
+    b = used * per_expert
+    m = total_rows(p)
+    b += m * p.k if p.x1 is not None else m * p.k * 2 + m * p.k + 4 * m   # prologue reads bf16, writes int8 + scale
+    b += m * (4 + 4 + p.row_index.dtype.itemsize)
+    b += p.output_bs * p.n * 4
+    if p.shared is not None:
+        b += p.shared.size * 2
+    return float(b)
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.ident = str(device_index)
+        try:
+            import torch
+            u = getattr(torch.cuda.get_device_properties(device_index), "uuid", None)
+            if u is not None:
+                s = str(u)
+                self.ident = s if s.startswith("GPU-") else "GPU-" + s
+        except Exception:
+            pass
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.ident, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower().startswith("active")})
+        sm = sorted(x[0] for x in rows)
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(x[1] for x in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- device timing
+def time_steps(d, steps, warmup, deterministic, dist=None):
+    """Device time of `steps` back-to-back calls (CUDA events on the launch stream),
+    and the grouped-GEMM kernel's own average duration from events recorded by the
+    library around its launch."""
+    import torch
+    from quantized_moe_grouped_persistent_b200 import finalize_profiled
+    stream = torch.cuda.current_stream()
+    prob = d.problem(deterministic)
+    ws = d.workspace(deterministic)
+
+    def step(b, e):
+        d.quantize()
+        finalize_profiled(prob, d.x1, d.x2, d.scale, d.pts, d.group_list, d.logit, d.row_index, d.bias, d.shared,
+                          d.out, ws, b, e, stream=stream)
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for b, e in ev:            # torch creates the underlying cudaEvent_t on first record
+        b.record(stream)
+        e.record(stream)
+    for _ in range(warmup):
+        step(*ev[0])
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(steps):
+        step(*ev[s])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    gemm_ms = sum(b.elapsed_time(e) for b, e in ev) / steps
+    return ms, gemm_ms
+
+
+def time_e2e(d, p, steps, warmup, deterministic):
+    """Same call through host buffers: per step, pinned host -> device copies of the
+    step's inputs (activations, routing, sharedInput), the op, and the output back
+    to pinned host memory; weights stay resident like a served layer's parameters."""
+    import numpy as np
+    import torch
+    stream = torch.cuda.current_stream()
+    pairs = []
+
+    def pin(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            a = a.view(np.int16)
+        return torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+
+    if d.prologue:
+        pairs.append((pin(p.x_bf16), d.x_bf16))
+    else:
+        pairs += [(pin(p.x1), d.x1), (pin(p.pertoken_scale), d.pts)]
+    pairs += [(pin(p.group_list.astype(np.int64)), d.group_list), (pin(p.logit), d.logit),
+              (pin(p.row_index), d.row_index)]
+    if p.shared is not None:
+        pairs.append((pin(p.shared), d.shared))
+    host_out = torch.empty(tuple(d.out.shape), dtype=torch.float32).pin_memory()
+    h2d = sum(h.numel() * h.element_size() for h, _ in pairs)
+    d2h = host_out.numel() * 4
+
+    def step():
+        for h, dv in pairs:
+            dv.copy_(h, non_blocking=True)
+        d.run(deterministic=deterministic, stream=stream)
+        host_out.copy_(d.out, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1) / steps, h2d, d2h
+
+
+# ----------------------------------------------------------------------------- CPU oracle timing
+def oracle_sample_time(p, target_s, seed):
+    """Time the oracle on a seeded sample of output rows sized to about target_s seconds."""
+    import numpy as np
+    import oracle
+    from synth import sample_rows
+    threads = oracle.default_threads()
+    counts = np.bincount(p.row_index, minlength=p.output_bs)
+    kw = {}
+    if p.x1 is None:
+        q, s = oracle.per_token_quant(p.x_bf16)
+        kw = dict(x1=q, pertoken_scale=s)
+
+    def run(nrows, sd):
+        rows = sample_rows(sd, p.output_bs, nrows)
+        t = time.perf_counter()
+        oracle.problem_finalize(p, dest_rows=rows, want32=False, threads=threads, **kw)
+        return time.perf_counter() - t, 2.0 * float(counts[rows].sum()) * p.k * p.n, rows.size
+
+    t_cal, _, n_cal = run(max(2, threads // 2), seed)
+    per_row = max(t_cal / n_cal, 1e-6)
+    nrows = int(max(threads, min(p.output_bs, target_s / per_row)))
+    t, ops, nr = run(nrows, seed + 1)
+    return t, ops, nr, threads
+
+
+def reference_arm(args, p, spec_desc):
+    """The oracle as the reference arm: each step times a bounded sample of output rows."""
+    import numpy as np
+    import oracle
+    from synth import sample_rows
+    threads = oracle.default_threads()
+    counts = np.bincount(p.row_index, minlength=p.output_bs)
+    kw = {}
+    if p.x1 is None:
+        q, s = oracle.per_token_quant(p.x_bf16)
+        kw = dict(x1=q, pertoken_scale=s)
+    # size one step to about two seconds of host work
+    rows = sample_rows(7, p.output_bs, max(2, threads // 2))
+    t0 = time.perf_counter()
+    oracle.problem_finalize(p, dest_rows=rows, want32=False, threads=threads, **kw)
+    per_row = max((time.perf_counter() - t0) / rows.size, 1e-6)
+    nrows = int(max(1, min(p.output_bs, 2.0 / per_row)))
+    for w in range(args.warmup):
+        oracle.problem_finalize(p, dest_rows=sample_rows(100 + w, p.output_bs, max(1, nrows // 8)), want32=False,
+                                threads=threads, **kw)
+    total_t, total_ops = 0.0, 0.0
+    for s in range(args.steps):
+        rows = sample_rows(1000 + s, p.output_bs, nrows)
+        t0 = time.perf_counter()
+        oracle.problem_finalize(p, dest_rows=rows, want32=False, threads=threads, **kw)
+        total_t += time.perf_counter() - t0
+        total_ops += 2.0 * float(counts[rows].sum()) * p.k * p.n
+    value = total_ops / total_t / 1e12
+    sample = f"{nrows} of {p.output_bs} output rows per step (every contributing source row in full), {args.steps} steps"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": spec_desc, "mode": "deterministic order (oracle)"},
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    args = parse_args()
+    from synth import CONFIGS, make_problem
+    from synth.inputs import SEED_BASE
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    spec = CONFIGS[args.workload]
+    mode = "deterministic" if args.deterministic else "atomic"
+    spec_desc = f"{args.workload}: {spec.description}; {mode} combine"
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        p = make_problem(args.workload)
+        reference_arm(args, p, spec_desc)
+        return
+
+    import torch
+    from quantized_moe_grouped_persistent_b200.device import DeviceProblem
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist = tdist
+    else:
+        torch.cuda.set_device(0)
+    dev_index = torch.cuda.current_device()
+
+    seed = SEED_BASE + spec.index + 1000 * rank
+    p = make_problem(args.workload, seed=seed if rank else None)
+    d = DeviceProblem(p)
+    ops = int_ops(p)
+    peaks = load_peaks()
+    int8_peak_sustained = 2.0 * peaks["bf16_sustained"]   # dense int8 = 2 x dense bf16 (nominal ratio)
+
+    sampler = ClockSampler(dev_index)
+    d.run(deterministic=args.deterministic)                # first call: module load, tensor maps
+    torch.cuda.synchronize()
+    flags = d.status(args.deterministic)
+    sampler.start()
+    ms, gemm_ms = time_steps(d, args.steps, args.warmup, args.deterministic, dist)
+    clocks = sampler.stop()
+    mx = torch.tensor([ms, gemm_ms], dtype=torch.float64, device="cuda")
+    if dist is not None:
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+    ms_max, gemm_max = float(mx[0]), float(mx[1])
+    value = world * ops / (ms_max * 1e-3) / 1e12
+    launches_per_step = (7 if args.deterministic else 2) + (1 if d.prologue else 0)
+
+    extras = {}
+    if world == 1 and not args.no_extras:
+        e2e_ms, h2d, d2h = time_e2e(d, p, max(3, args.steps // 4), 2, args.deterministic)
+        extras["e2e"] = {"value": ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS", "h2d_bytes_per_step": h2d,
+                         "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+        if not args.deterministic:
+            dms, dgemm = time_steps(d, max(3, args.steps // 2), 2, True)
+            extras["deterministic"] = {"ms_per_step": dms, "value": ops / (dms * 1e-3) / 1e12, "unit": "TOPS",
+                                       "gemm_ms": dgemm}
+    del d
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_extras and args.workload != "decode":
+        pd = make_problem("decode")
+        dd = DeviceProblem(pd)
+        dd.run()
+        torch.cuda.synchronize()
+        dms, dgemm = time_steps(dd, max(10, args.steps), 3, False)
+        dbytes = algorithmic_bytes(pd)
+        extras["decode"] = {
+            "workload": "decode: " + CONFIGS["decode"].description + "; atomic combine",
+            "value": dbytes / (dms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": dms,
+            "algorithmic_bytes": dbytes,
+            "roofline": {"bound": "hbm", "achieved": dbytes / (dgemm * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": dbytes / (dgemm * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "traffic": committed_traffic("decode"), "kernel_ms": dgemm,
+                         "peak_source": peaks["source"] + " copy bandwidth"},
+            "pct_of_nominal_8tbs": 100.0 * dbytes / (dms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
+        }
+        del dd
+        torch.cuda.empty_cache()
+
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        t, sops, nr, threads = oracle_sample_time(p, args.cpu_seconds, 4242)
+        cpu = {"value": sops / t / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
+               "sample": f"{nr} of {p.output_bs} output rows of the same workload (every contributing source "
+                         f"row in full, double-precision dequant/combine), {t:.1f} s"}
+
+    if rank == 0:
+        achieved = ops / (gemm_max * 1e-3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": spec_desc, "tokens": p.tokens, "topk": p.topk, "m": p.m, "e": p.e, "k": p.k,
+                       "n": p.n, "output_bs": p.output_bs, "mode": mode,
+                       "l2": "inputs larger than L2 (x2 %.2f GB per rank), no flush" % (p.x2.nbytes / 1e9),
+                       "parallelism": f"dp{world} (independent batch per GPU)"},
+            "pct_of_dense_int8_peak": {"nominal_4500": 100.0 * value / world / NOMINAL_INT8_TOPS,
+                                       "measured_sustained": 100.0 * value / world / int8_peak_sustained},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": int8_peak_sustained, "unit": "TOPS",
+                         "frac": achieved / int8_peak_sustained, "traffic": committed_traffic(args.workload),
+                         "kernel": "grouped_gemm_kernel", "kernel_ms": gemm_max,
+                         "peak_source": f"{peaks['source']} bf16 sustained x 2 (dense int8 : bf16 nominal ratio)"},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+            "device_status": flags,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        line.update(extras)
+        if "e2e" not in line:
+            line["e2e"] = None
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -134,6 +134,20 @@ qgmm_status qgmm_finalize(const qgmm_problem *p, const int8_t *x1, const void *x
                           void *workspace, size_t ws_bytes, void *cuda_stream);
 
 /*
+ * qgmm_finalize, plus two caller-owned cudaEvent_t handles recorded on
+ * `cuda_stream` immediately before and after the grouped-GEMM launch, so a
+ * caller can time that kernel alone inside a live call.  The result is the
+ * same as qgmm_finalize's.  Errors: as qgmm_finalize, and NULL_PTR when
+ * either event is NULL.
+ */
+qgmm_status qgmm_finalize_profiled(const qgmm_problem *p, const int8_t *x1, const void *x2,
+                                   const float *scale, const float *pertoken_scale,
+                                   const int64_t *group_list, const float *logit, const void *row_index,
+                                   const float *bias, const uint16_t *shared_input, float *out,
+                                   void *workspace, size_t ws_bytes, void *cuda_stream,
+                                   void *gemm_begin_event, void *gemm_end_event);
+
+/*
  * Per-token quantisation prologue (page 4, per_token_cast: the value times a
  * precomputed inverse scale; page 2, quant mode 7 "dynamic pertoken"):
  *   a = max_j |x[i][j]|;  scale_out[i] = a / 127;  inv = a > 0 ? 127 / a : 0

@@ -45,8 +45,8 @@ QGMM_DEV_GROUP_TOTAL_GT_M = 1 << 2
 QGMM_DEV_ROW_INDEX_RANGE = 1 << 3
 QGMM_DEV_TIMEOUT = 1 << 4
 
-EXPORTS = ("qgmm_finalize_workspace", "qgmm_finalize", "qgmm_per_token_quant", "qgmm_debug_accum",
-           "qgmm_device_status", "qgmm_status_string")
+EXPORTS = ("qgmm_finalize_workspace", "qgmm_finalize", "qgmm_finalize_profiled", "qgmm_per_token_quant",
+           "qgmm_debug_accum", "qgmm_device_status", "qgmm_status_string")
 
 
 class QgmmProblem(C.Structure):
@@ -80,6 +80,7 @@ def lib():
         P, I64, U = C.c_void_p, C.c_int64, C.c_size_t
         L.qgmm_finalize_workspace.argtypes = [C.POINTER(QgmmProblem), C.POINTER(C.c_size_t)]
         L.qgmm_finalize.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, P, P, P, P, P, P, U, P]
+        L.qgmm_finalize_profiled.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, P, P, P, P, P, P, U, P, P, P]
         L.qgmm_per_token_quant.argtypes = [P, I64, I64, P, P, P]
         L.qgmm_debug_accum.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, U, P]
         L.qgmm_device_status.argtypes = [P, C.POINTER(C.c_uint32), P]
@@ -139,6 +140,22 @@ def finalize(problem: QgmmProblem, x1, x2, scale, pertoken_scale, group_list, lo
                              _ptr(group_list), _ptr(logit), _ptr(row_index), _ptr(bias), _ptr(shared_input),
                              _ptr(out), _ptr(workspace), ws_bytes, _stream(stream))
     _check(rc, "qgmm_finalize")
+
+
+def finalize_profiled(problem: QgmmProblem, x1, x2, scale, pertoken_scale, group_list, logit, row_index, bias,
+                      shared_input, out, workspace, begin_event, end_event, ws_bytes: Optional[int] = None,
+                      stream=None) -> None:
+    """``finalize`` that also records ``begin_event``/``end_event`` (torch.cuda.Event) around the GEMM launch.
+
+    torch creates an event's handle on its first ``record()``; record each event once before passing it.
+    """
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().qgmm_finalize_profiled(C.byref(problem), _ptr(x1), _ptr(x2), _ptr(scale), _ptr(pertoken_scale),
+                                      _ptr(group_list), _ptr(logit), _ptr(row_index), _ptr(bias),
+                                      _ptr(shared_input), _ptr(out), _ptr(workspace), ws_bytes, _stream(stream),
+                                      begin_event.cuda_event, end_event.cuda_event)
+    _check(rc, "qgmm_finalize_profiled")
 
 
 def per_token_quant(x_bf16, x1_out, scale_out, rows: Optional[int] = None, k: Optional[int] = None,

@@ -269,10 +269,12 @@ QGMM_API qgmm_status qgmm_finalize_workspace(const qgmm_problem *p, size_t *ws_b
     return QGMM_OK;
 }
 
-QGMM_API qgmm_status qgmm_finalize(const qgmm_problem *p, const int8_t *x1, const void *x2, const float *scale,
-                                   const float *pertoken_scale, const int64_t *group_list, const float *logit,
-                                   const void *row_index, const float *bias, const uint16_t *shared_input,
-                                   float *out, void *workspace, size_t ws_bytes, void *cuda_stream)
+namespace {
+qgmm_status finalize_impl(const qgmm_problem *p, const int8_t *x1, const void *x2, const float *scale,
+                          const float *pertoken_scale, const int64_t *group_list, const float *logit,
+                          const void *row_index, const float *bias, const uint16_t *shared_input, float *out,
+                          void *workspace, size_t ws_bytes, void *cuda_stream, cudaEvent_t ev_begin,
+                          cudaEvent_t ev_end)
 {
     qgmm_status s = check_problem(p);
     if (s != QGMM_OK) return s;
@@ -306,7 +308,10 @@ QGMM_API qgmm_status qgmm_finalize(const qgmm_problem *p, const int8_t *x1, cons
             out, p->output_bs, static_cast<int32_t>(p->n), shared, p->shared_bs, p->shared_offset, status);
         if (cudaGetLastError() != cudaSuccess) return QGMM_ERR_CUDA;
         a.out = out;
-        return launch_gemm(EPI_ATOMIC, dev, p, pl, ma, mb, a, st);
+        if (ev_begin && cudaEventRecord(ev_begin, st) != cudaSuccess) return QGMM_ERR_CUDA;
+        if ((s = launch_gemm(EPI_ATOMIC, dev, p, pl, ma, mb, a, st)) != QGMM_OK) return s;
+        if (ev_end && cudaEventRecord(ev_end, st) != cudaSuccess) return QGMM_ERR_CUDA;
+        return QGMM_OK;
     }
 
     const DetLayout L = det_layout(p);
@@ -325,10 +330,35 @@ QGMM_API qgmm_status qgmm_finalize(const qgmm_problem *p, const int8_t *x1, cons
     det_sort_kernel<<<grid_for(p->output_bs, 256, dev->sms, 4), 256, 0, st>>>(starts, list, p->output_bs);
     if (cudaGetLastError() != cudaSuccess) return QGMM_ERR_CUDA;
     a.out = y;
+    if (ev_begin && cudaEventRecord(ev_begin, st) != cudaSuccess) return QGMM_ERR_CUDA;
     if ((s = launch_gemm(EPI_STORE_Y, dev, p, pl, ma, mb, a, st)) != QGMM_OK) return s;
+    if (ev_end && cudaEventRecord(ev_end, st) != cudaSuccess) return QGMM_ERR_CUDA;
     det_reduce_kernel<<<grid_for(p->output_bs, 1, dev->sms, 8), 256, 0, st>>>(
         out, y, static_cast<int32_t>(p->n), starts, list, p->output_bs, shared, p->shared_bs, p->shared_offset);
     return cudaGetLastError() == cudaSuccess ? QGMM_OK : QGMM_ERR_CUDA;
+}
+}  // namespace
+
+QGMM_API qgmm_status qgmm_finalize(const qgmm_problem *p, const int8_t *x1, const void *x2, const float *scale,
+                                   const float *pertoken_scale, const int64_t *group_list, const float *logit,
+                                   const void *row_index, const float *bias, const uint16_t *shared_input,
+                                   float *out, void *workspace, size_t ws_bytes, void *cuda_stream)
+{
+    return finalize_impl(p, x1, x2, scale, pertoken_scale, group_list, logit, row_index, bias, shared_input, out,
+                         workspace, ws_bytes, cuda_stream, nullptr, nullptr);
+}
+
+QGMM_API qgmm_status qgmm_finalize_profiled(const qgmm_problem *p, const int8_t *x1, const void *x2,
+                                            const float *scale, const float *pertoken_scale,
+                                            const int64_t *group_list, const float *logit, const void *row_index,
+                                            const float *bias, const uint16_t *shared_input, float *out,
+                                            void *workspace, size_t ws_bytes, void *cuda_stream,
+                                            void *gemm_begin_event, void *gemm_end_event)
+{
+    if (!gemm_begin_event || !gemm_end_event) return QGMM_ERR_NULL_PTR;
+    return finalize_impl(p, x1, x2, scale, pertoken_scale, group_list, logit, row_index, bias, shared_input, out,
+                         workspace, ws_bytes, cuda_stream, static_cast<cudaEvent_t>(gemm_begin_event),
+                         static_cast<cudaEvent_t>(gemm_end_event));
 }
 
 QGMM_API qgmm_status qgmm_debug_accum(const qgmm_problem *p, const int8_t *x1, const void *x2,

@@ -22,8 +22,8 @@ def _declared_functions():
 
 def test_header_declares_the_abi():
     assert _declared_functions() == sorted([
-        "qgmm_finalize_workspace", "qgmm_finalize", "qgmm_per_token_quant", "qgmm_debug_accum",
-        "qgmm_device_status", "qgmm_status_string"])
+        "qgmm_finalize_workspace", "qgmm_finalize", "qgmm_finalize_profiled", "qgmm_per_token_quant",
+        "qgmm_debug_accum", "qgmm_device_status", "qgmm_status_string"])
 
 
 def test_library_exports_every_declared_symbol(qgmm):
@@ -121,6 +121,7 @@ def test_null_arguments(qgmm):
     assert L.qgmm_per_token_quant(None, 4, 64, fake, fake, None) == qgmm.QGMM_ERR_NULL_PTR
     assert L.qgmm_debug_accum(C.byref(p), fake, fake, None, fake, fake, 256, None) == qgmm.QGMM_ERR_NULL_PTR
     assert L.qgmm_device_status(None, None, None) == qgmm.QGMM_ERR_NULL_PTR
+    assert L.qgmm_finalize_profiled(C.byref(p), *args, None, None) == qgmm.QGMM_ERR_NULL_PTR
 
 
 def test_alignment_and_workspace_checks(qgmm):
