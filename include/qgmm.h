@@ -57,7 +57,8 @@ typedef enum {
     QGMM_ERR_UNSUPPORTED = 5,         /* the device is not sm_100 or a feature is not built   */
     QGMM_ERR_CUDA = 6,                /* a CUDA runtime / driver call failed                  */
     QGMM_ERR_DEVICE_INPUT = 7,        /* qgmm_device_status found QGMM_DEV_* bits set         */
-    QGMM_ERR_ALIGNMENT = 8            /* a pointer is not 16-byte aligned                     */
+    QGMM_ERR_ALIGNMENT = 8,           /* a pointer is not 16-byte aligned                     */
+    QGMM_ERR_SCRATCH_LIMIT = 9        /* qgmm_finalize_static_scratch: scratch above its cap  */
 } qgmm_status;
 
 enum { QGMM_W_INT8 = 0, QGMM_W_INT4_PACKED_INT32 = 1 };   /* x2: (e,k,n) int8 | (e,k,n/8) int32 */
@@ -146,6 +147,46 @@ qgmm_status qgmm_finalize_profiled(const qgmm_problem *p, const int8_t *x1, cons
                                    const float *bias, const uint16_t *shared_input, float *out,
                                    void *workspace, size_t ws_bytes, void *cuda_stream,
                                    void *gemm_begin_event, void *gemm_end_event);
+
+/*
+ * qgmm_finalize for callers that cannot allocate device memory.  (No
+ * counterpart on the pages: this entry point exists for this library's users.)
+ *
+ * Some callers are handed only their inputs and outputs and cannot call
+ * cudaMalloc for a workspace: a plugin slot in a host inference engine that
+ * grants no workspace, or a serving loop that must not call cudaMalloc or
+ * cudaFree because those calls can synchronise the whole device.  This entry
+ * point takes the same arguments as qgmm_finalize minus the workspace, and
+ * uses instead a file-scope device array of QGMM_STATIC_SCRATCH_BYTES (16 MiB)
+ * inside the library.  Every GPU that loads the library holds that array until
+ * the process exits.  The entry point allocates nothing (no cudaMalloc, no
+ * cudaFree, no allocating library routine).
+ *
+ *  - Limit: the problem's workspace (qgmm_finalize_workspace) must fit in
+ *    16 MiB.  Atomic mode needs 256 bytes, so it always fits; deterministic
+ *    mode fits while 256 + m*n*4 + (2*output_bs + 1 + m)*4, each part rounded
+ *    up to 256 bytes, stays within 16 MiB (for example m = 128, n = 7168).
+ *    Larger problems return QGMM_ERR_SCRATCH_LIMIT before anything is launched.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call shares the one array, which keeps the last call's contents.
+ *    Each call clears what must start at zero (the status word and the
+ *    deterministic mode's bucket counts) before using it.  Calls whose work
+ *    overlaps on one GPU (for example on two streams, or from two host
+ *    threads) race on the array and give wrong results: serialise them.
+ *    Each device has its own copy of the array, so calls on different
+ *    devices do not interfere.
+ *  - Device-side input checks still run and bad rows are still skipped, but
+ *    the status word lives in the library's array and is not reported.
+ * Errors: as qgmm_finalize, and QGMM_ERR_SCRATCH_LIMIT.
+ */
+#define QGMM_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+qgmm_status qgmm_finalize_static_scratch(const qgmm_problem *p, const int8_t *x1, const void *x2,
+                                         const float *scale, const float *pertoken_scale,
+                                         const int64_t *group_list, const float *logit,
+                                         const void *row_index, const float *bias,
+                                         const uint16_t *shared_input, float *out, void *cuda_stream);
 
 /*
  * Per-token quantisation prologue (page 4, per_token_cast: the value times a

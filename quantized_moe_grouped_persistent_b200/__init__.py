@@ -31,6 +31,8 @@ QGMM_ERR_UNSUPPORTED = 5
 QGMM_ERR_CUDA = 6
 QGMM_ERR_DEVICE_INPUT = 7
 QGMM_ERR_ALIGNMENT = 8
+QGMM_ERR_SCRATCH_LIMIT = 9
+QGMM_STATIC_SCRATCH_BYTES = 16 << 20
 
 QGMM_W_INT8 = 0
 QGMM_W_INT4_PACKED_INT32 = 1
@@ -46,7 +48,7 @@ QGMM_DEV_ROW_INDEX_RANGE = 1 << 3
 QGMM_DEV_TIMEOUT = 1 << 4
 
 EXPORTS = ("qgmm_finalize_workspace", "qgmm_finalize", "qgmm_finalize_profiled", "qgmm_per_token_quant",
-           "qgmm_debug_accum", "qgmm_device_status", "qgmm_status_string")
+           "qgmm_debug_accum", "qgmm_device_status", "qgmm_finalize_static_scratch", "qgmm_status_string")
 
 
 class QgmmProblem(C.Structure):
@@ -84,6 +86,7 @@ def lib():
         L.qgmm_per_token_quant.argtypes = [P, I64, I64, P, P, P]
         L.qgmm_debug_accum.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, U, P]
         L.qgmm_device_status.argtypes = [P, C.POINTER(C.c_uint32), P]
+        L.qgmm_finalize_static_scratch.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, P, P, P, P, P, P]
         L.qgmm_status_string.argtypes = [C.c_int]
         L.qgmm_status_string.restype = C.c_char_p
         for name in EXPORTS[:-1]:
@@ -182,3 +185,17 @@ def device_status(workspace, stream=None) -> int:
     if rc not in (QGMM_OK, QGMM_ERR_DEVICE_INPUT):
         raise QgmmError(rc, "qgmm_device_status")
     return flags.value
+
+
+def finalize_static_scratch(problem: QgmmProblem, x1, x2, scale, pertoken_scale, group_list, logit, row_index,
+                            bias, shared_input, out, stream=None) -> None:
+    """``finalize`` without a workspace argument, for callers that cannot allocate device memory.
+
+    The library uses its own 16 MiB device array as scratch (see ``qgmm_finalize_static_scratch`` in
+    ``include/qgmm.h``): problems whose workspace would exceed it raise with ``QGMM_ERR_SCRATCH_LIMIT``,
+    the first call on a device looks up the array's address, and calls that overlap on one GPU race.
+    """
+    rc = lib().qgmm_finalize_static_scratch(C.byref(problem), _ptr(x1), _ptr(x2), _ptr(scale),
+                                            _ptr(pertoken_scale), _ptr(group_list), _ptr(logit), _ptr(row_index),
+                                            _ptr(bias), _ptr(shared_input), _ptr(out), _stream(stream))
+    _check(rc, "qgmm_finalize_static_scratch")

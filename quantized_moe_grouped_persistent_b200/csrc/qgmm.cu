@@ -424,6 +424,54 @@ QGMM_API const char *qgmm_status_string(qgmm_status s)
     case QGMM_ERR_CUDA: return "a CUDA call failed";
     case QGMM_ERR_DEVICE_INPUT: return "the device found invalid group_list or row_index values";
     case QGMM_ERR_ALIGNMENT: return "a pointer is not suitably aligned";
+    case QGMM_ERR_SCRATCH_LIMIT: return "the problem needs more scratch than the library's static array holds";
     }
     return "unknown status";
+}
+
+// ---------------------------------------------------------------------------
+// qgmm_finalize for callers that cannot allocate device memory.  The
+// workspace is this file-scope array instead of caller memory; every GPU that
+// loads the library holds it until the process exits.
+static __device__ __align__(256) unsigned char qgmm_static_scratch[QGMM_STATIC_SCRATCH_BYTES];
+
+namespace qgmm {
+namespace {
+void *g_static_scratch_addr[kMaxDevices] = {};
+
+// Device address of qgmm_static_scratch on the current device, looked up once
+// per device.  In host code the array's name is only a host-side stand-in, so
+// it is never handed to a kernel directly.
+qgmm_status static_scratch_address(void **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QGMM_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_static_scratch_addr[dev]) {
+        void *p = nullptr;
+        const cudaError_t rc = cudaGetSymbolAddress(&p, qgmm_static_scratch);
+        if (rc != cudaSuccess || !p) return QGMM_ERR_CUDA;
+        g_static_scratch_addr[dev] = p;
+    }
+    *out = g_static_scratch_addr[dev];
+    return QGMM_OK;
+}
+}  // namespace
+}  // namespace qgmm
+
+QGMM_API qgmm_status qgmm_finalize_static_scratch(const qgmm_problem *p, const int8_t *x1, const void *x2,
+                                                  const float *scale, const float *pertoken_scale,
+                                                  const int64_t *group_list, const float *logit,
+                                                  const void *row_index, const float *bias,
+                                                  const uint16_t *shared_input, float *out, void *cuda_stream)
+{
+    qgmm_status s = check_problem(p);
+    if (s != QGMM_OK) return s;
+    if (workspace_bytes(p) > QGMM_STATIC_SCRATCH_BYTES) return QGMM_ERR_SCRATCH_LIMIT;
+    DeviceInfo *dev = nullptr;
+    if ((s = device_info(&dev)) != QGMM_OK) return s;
+    void *scratch = nullptr;
+    if ((s = static_scratch_address(&scratch)) != QGMM_OK) return s;
+    return finalize_impl(p, x1, x2, scale, pertoken_scale, group_list, logit, row_index, bias, shared_input, out,
+                         scratch, QGMM_STATIC_SCRATCH_BYTES, cuda_stream, nullptr, nullptr);
 }

@@ -23,7 +23,7 @@ def _declared_functions():
 def test_header_declares_the_abi():
     assert _declared_functions() == sorted([
         "qgmm_finalize_workspace", "qgmm_finalize", "qgmm_finalize_profiled", "qgmm_per_token_quant",
-        "qgmm_debug_accum", "qgmm_device_status", "qgmm_status_string"])
+        "qgmm_debug_accum", "qgmm_device_status", "qgmm_finalize_static_scratch", "qgmm_status_string"])
 
 
 def test_library_exports_every_declared_symbol(qgmm):
@@ -154,7 +154,7 @@ def test_per_token_quant_host_checks(qgmm):
 
 
 def test_status_strings(qgmm):
-    for code in range(9):
+    for code in range(10):
         s = qgmm.status_string(code)
         assert s and s != "unknown status"
     assert qgmm.status_string(99) == "unknown status"
