@@ -31,6 +31,7 @@ constexpr int P_STAGE_BYTES = BK * BN / 2;   // 16 KB: packed int4 staging
 constexpr int B_ATOM_BYTES = BK * 128;       // one 128-column atom (LBO)
 constexpr int TMEM_COLS = 2 * BN;            // double-buffered accumulator
 constexpr int MAX_E = 1024;
+constexpr int EPI_LD = 36;                   // staging row stride in floats (conflict-free float4 access)
 
 enum Epilogue : int { EPI_ATOMIC = 0, EPI_STORE_Y = 1, EPI_RAW_ACC = 2 };
 
@@ -41,9 +42,16 @@ struct GemmCfg {
     static constexpr int THREADS = NUM_WARPS * 32;
     static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES + (W4 ? P_STAGE_BYTES : 0);
     static constexpr int NUM_BARS = 3 * STAGES + 2 + 2 + 1;
-    static constexpr int CTRL_BYTES = NUM_BARS * 8 + 16;
-    static constexpr int TABLE_BYTES = 2 * (MAX_E + 1) * 4;
-    static constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + CTRL_BYTES + TABLE_BYTES;
+    static constexpr int CTRL_BYTES = (NUM_BARS * 8 + 16 + 15) / 16 * 16;
+    static constexpr int TABLE_BYTES = (2 * (MAX_E + 1) * 4 + 15) / 16 * 16;
+    static constexpr int EPI_STAGE_BYTES = 4 * 32 * EPI_LD * 4;   // per epilogue warp: 32 rows x 32 cols (+pad)
+    static constexpr int ROWINFO_BYTES = 4 * 32 * 16;              // per row: pts, logit, destination
+    static constexpr size_t OFF_CTRL = size_t(STAGES) * STAGE_BYTES;
+    static constexpr size_t OFF_TABLE = OFF_CTRL + CTRL_BYTES;
+    static constexpr size_t OFF_EPI = OFF_TABLE + TABLE_BYTES;
+    static constexpr size_t OFF_ROWS = OFF_EPI + EPI_STAGE_BYTES;
+    static constexpr size_t SMEM_BYTES = 1024 + OFF_ROWS + ROWINFO_BYTES;
+    static_assert(SMEM_BYTES <= 232448, "shared memory above the sm_100 per-block limit");
 };
 
 struct GemmArgs {
@@ -180,6 +188,64 @@ __device__ __forceinline__ void unpack_int4x8(uint32_t w, uint32_t &lo_out, uint
     hi_out = __byte_perm(lo, hi, 0x7362);   // columns 4..7
 }
 
+// ---------------------------------------------------------------- K2 epilogue helpers
+constexpr int NCHUNK = BN / 32;   // 32-column chunks per accumulator
+
+// Thread = accumulator row: write its 32 values of one chunk into the warp's
+// staging rows (f32 of the int32 value, or its raw bits for the debug output).
+template <int EPI>
+__device__ __forceinline__ void epi_stage_chunk(float *stage, int lane, const uint32_t (&r)[32])
+{
+    float *srow = stage + lane * EPI_LD;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+        float4 f;
+        if constexpr (EPI == EPI_RAW_ACC) {
+            f = make_float4(__int_as_float(r[4 * v]), __int_as_float(r[4 * v + 1]), __int_as_float(r[4 * v + 2]),
+                            __int_as_float(r[4 * v + 3]));
+        } else {
+            f = make_float4(__int2float_rn(static_cast<int>(r[4 * v])), __int2float_rn(static_cast<int>(r[4 * v + 1])),
+                            __int2float_rn(static_cast<int>(r[4 * v + 2])),
+                            __int2float_rn(static_cast<int>(r[4 * v + 3])));
+        }
+        *reinterpret_cast<float4 *>(srow + 4 * v) = f;
+    }
+}
+
+// Transposed read of a staged chunk: lane (sub, col4) takes 4 columns of rows
+// sub, sub+4, ..., so each warp instruction covers 4 rows x 128 contiguous bytes.
+// The dequant runs here in the op's order: ((f32(acc) * scale) * pts + bias) * logit.
+template <int EPI>
+__device__ __forceinline__ void epi_write_chunk(const GemmArgs &args, const float *stage, const float *rp,
+                                                const float *rl, const long long *rd, int sub, int col4, int n,
+                                                int64_t chunk_col0, float4 s4, float4 b4)
+{
+    const int64_t col = chunk_col0 + col4;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+        const int row = sub + 4 * it;
+        const long long d = rd[row];
+        const float4 v = *reinterpret_cast<const float4 *>(stage + row * EPI_LD + col4);
+        if (d >= 0) {
+            if constexpr (EPI == EPI_RAW_ACC) {
+                *reinterpret_cast<int4 *>(args.acc_out + d * n + col) =
+                    make_int4(__float_as_int(v.x), __float_as_int(v.y), __float_as_int(v.z), __float_as_int(v.w));
+            } else {
+                const float p = rp[row], l = rl[row];
+                const float y0 = __fmul_rn(__fadd_rn(__fmul_rn(__fmul_rn(v.x, s4.x), p), b4.x), l);
+                const float y1 = __fmul_rn(__fadd_rn(__fmul_rn(__fmul_rn(v.y, s4.y), p), b4.y), l);
+                const float y2 = __fmul_rn(__fadd_rn(__fmul_rn(__fmul_rn(v.z, s4.z), p), b4.z), l);
+                const float y3 = __fmul_rn(__fadd_rn(__fmul_rn(__fmul_rn(v.w, s4.w), p), b4.w), l);
+                if constexpr (EPI == EPI_ATOMIC) {
+                    ptx::red_add_v4(args.out + d * n + col, y0, y1, y2, y3);
+                } else {
+                    *reinterpret_cast<float4 *>(args.out + d * n + col) = make_float4(y0, y1, y2, y3);
+                }
+            }
+        }
+    }
+}
+
 // ---------------------------------------------------------------- K2
 template <int EPI, bool W4>
 __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
@@ -193,7 +259,7 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
     uint8_t *smem_a = smem;
     uint8_t *smem_b = smem_a + S * A_STAGE_BYTES;
     uint8_t *smem_p = smem_b + S * B_STAGE_BYTES;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + size_t(S) * Cfg::STAGE_BYTES);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_CTRL);
     uint64_t *full = bars;            // operands ready for the MMA
     uint64_t *empty = bars + S;       // MMA finished reading the stage
     uint64_t *pfull = bars + 2 * S;   // W4: packed tile + x1 tile landed
@@ -202,8 +268,12 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
     uint64_t *drain = tempty + 2;     // all issued MMAs completed
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + Cfg::NUM_BARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
-    int32_t *off = reinterpret_cast<int32_t *>(smem + size_t(S) * Cfg::STAGE_BYTES + Cfg::CTRL_BYTES);
+    int32_t *off = reinterpret_cast<int32_t *>(smem + Cfg::OFF_TABLE);
     int32_t *cum = off + (MAX_E + 1);
+    float *epi_stage = reinterpret_cast<float *>(smem + Cfg::OFF_EPI);
+    float *row_pts = reinterpret_cast<float *>(smem + Cfg::OFF_ROWS);
+    float *row_lg = row_pts + 4 * 32;
+    long long *row_dst = reinterpret_cast<long long *>(row_lg + 4 * 32);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -350,85 +420,96 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
         }
         __syncwarp();
     } else if (warp < 6) {
-        // ------------------------------------------------ epilogue (TMEM -> registers -> global)
-        const int q = warp & 3;                 // TMEM lane quarter this warp may access
-        const int r_in = q * 32 + lane;         // accumulator row of this thread
+        // ------------------------------------------------ epilogue (TMEM -> registers -> smem -> global)
+        // Each warp owns one TMEM lane quarter (32 accumulator rows).  A 32x32
+        // chunk is read with tcgen05.ld (thread = row), converted to f32 and
+        // staged in shared memory; it is then read back transposed so that 8
+        // lanes cover one row's 32 columns (128 contiguous bytes) and one warp
+        // instruction writes 4 whole rows segments.  The dequant arithmetic runs
+        // in the transposed phase, in the op's order:
+        //   ((f32(acc) * scale) * pts + bias) * logit
+        const int q = warp & 3;
         const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+        float *stage = epi_stage + q * (32 * EPI_LD);
+        float *rp = row_pts + q * 32;
+        float *rl = row_lg + q * 32;
+        long long *rd = row_dst + q * 32;
         const int n = args.n;
+        const int sub = lane >> 3;            // row (mod 4) handled in the transposed phase
+        const int col4 = (lane & 7) * 4;      // first of the 4 columns handled in the transposed phase
         int lt = 0;
         for (int t = blockIdx.x; t < T; t += gridDim.x, ++lt) {
             const TileCoord c = tile_coord(t, MT, SW, off, cum, e, tile_rows);
             const int buf = lt & 1;
             const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
+            // per-row data of this warp's 32 rows, fetched while the MMA still runs
+            const int r_in = q * 32 + lane;
+            const int64_t i = static_cast<int64_t>(c.row0) + r_in;
+            float pts = 1.0f, lg = 1.0f;
+            long long dst = -1;
+            if (r_in < tile_rows && i < c.row_end) {
+                if (args.pts) pts = __ldg(args.pts + i);
+                if (args.logit) lg = __ldg(args.logit + i);
+                if (EPI == EPI_ATOMIC) {
+                    const int64_t d = load_row_index(args.row_index, args.row_index_type, i);
+                    if (d < 0 || d >= args.output_bs) atomicOr(args.status, QGMM_DEV_ROW_INDEX_RANGE);
+                    else dst = d;
+                } else {
+                    dst = i;
+                }
+            }
+            rp[lane] = pts;
+            rl[lane] = lg;
+            rd[lane] = dst;
+            const bool any = __any_sync(0xffffffffu, dst >= 0);
+            // this lane's 4 columns of every 32-column chunk of scale and bias
+            float4 sc[NCHUNK], bs[NCHUNK];
+#pragma unroll
+            for (int k = 0; k < NCHUNK; ++k) {
+                sc[k] = make_float4(1.f, 1.f, 1.f, 1.f);
+                bs[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            if (EPI != EPI_RAW_ACC && any) {
+                const int64_t base = static_cast<int64_t>(c.g) * n + static_cast<int64_t>(c.nt) * BN + col4;
+                if (args.scale) {
+#pragma unroll
+                    for (int k = 0; k < NCHUNK; ++k)
+                        sc[k] = __ldg(reinterpret_cast<const float4 *>(args.scale + base + k * 32));
+                }
+                if (args.bias) {
+#pragma unroll
+                    for (int k = 0; k < NCHUNK; ++k)
+                        bs[k] = __ldg(reinterpret_cast<const float4 *>(args.bias + base + k * 32));
+                }
+            }
+            __syncwarp();
             if (!ptx::mbar_wait(&tfull[buf], use, abort_flag)) {
                 fail();
                 break;
             }
             ptx::tc_fence_after();
-            const int64_t i = static_cast<int64_t>(c.row0) + r_in;
-            bool valid = r_in < tile_rows && i < c.row_end;
-            const int n0 = c.nt * BN;
-            float pts = 1.0f, lg = 1.0f;
-            int64_t dst = i;
-            if (valid) {
-                if (args.pts) pts = __ldg(args.pts + i);
-                if (args.logit) lg = __ldg(args.logit + i);
-                if (EPI == EPI_ATOMIC) {
-                    dst = load_row_index(args.row_index, args.row_index_type, i);
-                    if (dst < 0 || dst >= args.output_bs) {
-                        atomicOr(args.status, QGMM_DEV_ROW_INDEX_RANGE);
-                        valid = false;
-                    }
-                }
-            }
-            if (__any_sync(0xffffffffu, valid)) {
-                const float *sc_row = args.scale ? args.scale + static_cast<int64_t>(c.g) * n + n0 : nullptr;
-                const float *bs_row = args.bias ? args.bias + static_cast<int64_t>(c.g) * n + n0 : nullptr;
-#pragma unroll 1
-                for (int cc = 0; cc < BN; cc += 16) {
-                    uint32_t r[16];
+            if (any) {
+                const int64_t n0 = static_cast<int64_t>(c.nt) * BN;
+                const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(buf * BN);
+                // tcgen05.ld of chunk 0 first; chunk k+1 is issued while chunk k is written out
+                uint32_t ra[32], rb[32];
+                ptx::tmem_ld_32x32b_x32(tbase, ra);
+#pragma unroll
+                for (int pc = 0; pc < NCHUNK; pc += 2) {
+                    ptx::tmem_ld_wait(ra);
+                    epi_stage_chunk<EPI>(stage, lane, ra);
+                    ptx::tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>((pc + 1) * 32), rb);
                     __syncwarp();
-                    ptx::tmem_ld_32x32b_x16(tmem_base + lane_addr + static_cast<uint32_t>(buf * BN + cc), r);
-                    ptx::tmem_ld_wait(r);
-                    if (!valid) {
-                        // this row is masked; the warp still reads TMEM in lockstep
-                    } else if constexpr (EPI == EPI_RAW_ACC) {
-                        int4 *o = reinterpret_cast<int4 *>(args.acc_out + i * n + n0 + cc);
-#pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            o[v] = make_int4(static_cast<int>(r[4 * v]), static_cast<int>(r[4 * v + 1]),
-                                             static_cast<int>(r[4 * v + 2]), static_cast<int>(r[4 * v + 3]));
-                    } else {
-                        float y[16];
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            float4 s4 = make_float4(1.f, 1.f, 1.f, 1.f);
-                            float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                            if (sc_row) s4 = __ldg(reinterpret_cast<const float4 *>(sc_row + cc) + v);
-                            if (bs_row) b4 = __ldg(reinterpret_cast<const float4 *>(bs_row + cc) + v);
-                            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-                            const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                float x = __int2float_rn(static_cast<int>(r[4 * v + u]));
-                                x = __fmul_rn(x, sv[u]);
-                                x = __fmul_rn(x, pts);
-                                x = __fadd_rn(x, bv[u]);
-                                y[4 * v + u] = __fmul_rn(x, lg);
-                            }
-                        }
-                        if constexpr (EPI == EPI_ATOMIC) {
-                            float *o = args.out + dst * n + n0 + cc;
-#pragma unroll
-                            for (int v = 0; v < 4; ++v)
-                                ptx::red_add_v4(o + 4 * v, y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]);
-                        } else {
-                            float4 *o = reinterpret_cast<float4 *>(args.out + i * n + n0 + cc);
-#pragma unroll
-                            for (int v = 0; v < 4; ++v)
-                                o[v] = make_float4(y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]);
-                        }
-                    }
+                    epi_write_chunk<EPI>(args, stage, rp, rl, rd, sub, col4, n, n0 + pc * 32, sc[pc], bs[pc]);
+                    __syncwarp();
+                    ptx::tmem_ld_wait(rb);
+                    epi_stage_chunk<EPI>(stage, lane, rb);
+                    if (pc + 2 < NCHUNK)
+                        ptx::tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>((pc + 2) * 32), ra);
+                    __syncwarp();
+                    epi_write_chunk<EPI>(args, stage, rp, rl, rd, sub, col4, n, n0 + (pc + 1) * 32, sc[pc + 1],
+                                         bs[pc + 1]);
+                    __syncwarp();
                 }
             }
             ptx::tc_fence_before();
