@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--no-extras", action="store_true", help="skip the decode / deterministic / e2e side runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
+    ap.add_argument("--tokens", type=int, default=None, help="shrink the workload (profiling proxies)")
+    ap.add_argument("--experts", type=int, default=None, help="shrink the workload (profiling proxies)")
     return ap.parse_args()
 
 
@@ -350,7 +352,9 @@ def main():
     dev_index = torch.cuda.current_device()
 
     seed = SEED_BASE + spec.index + 1000 * rank
-    p = make_problem(args.workload, seed=seed if rank else None)
+    p = make_problem(args.workload, seed=seed if rank else None, tokens=args.tokens, e=args.experts)
+    if args.tokens or args.experts:
+        spec_desc += f" (reduced: tokens={p.tokens}, e={p.e})"
     d = DeviceProblem(p)
     ops = int_ops(p)
     peaks = load_peaks()

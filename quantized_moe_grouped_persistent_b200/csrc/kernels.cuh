@@ -38,7 +38,8 @@ enum Epilogue : int { EPI_ATOMIC = 0, EPI_STORE_Y = 1, EPI_RAW_ACC = 2 };
 template <bool W4>
 struct GemmCfg {
     static constexpr int STAGES = W4 ? 3 : 4;
-    static constexpr int NUM_WARPS = W4 ? 10 : 6;   // producer, MMA, 4 epilogue (+4 unpack)
+    static constexpr int NUM_WARPS = 10;   // producer, MMA, then 8 epilogue (int8) or 4 epilogue + 4 unpack (W4)
+    static constexpr int EPI_WARPS = W4 ? 4 : 8;
     static constexpr int THREADS = NUM_WARPS * 32;
     static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES + (W4 ? P_STAGE_BYTES : 0);
     static constexpr int NUM_BARS = 3 * STAGES + 2 + 2 + 1;
@@ -246,6 +247,232 @@ __device__ __forceinline__ void epi_write_chunk(const GemmArgs &args, const floa
     }
 }
 
+// Shared-memory scratch of one epilogue warp.
+struct EpiSmem {
+    float *stage;      // 32 rows x EPI_LD floats
+    float *rp, *rl;    // per-row pertoken scale and logit
+    long long *rd;     // per-row output row (-1: skip)
+};
+
+__device__ __forceinline__ EpiSmem epi_smem(float *epi_stage, float *row_pts, float *row_lg, long long *row_dst, int slot)
+{
+    EpiSmem sm;
+    sm.stage = epi_stage + slot * (32 * EPI_LD);
+    sm.rp = row_pts + slot * 32;
+    sm.rl = row_lg + slot * 32;
+    sm.rd = row_dst + slot * 32;
+    return sm;
+}
+
+// Epilogue of one accumulator tile for one warp, which owns TMEM lane quarter
+// q (accumulator rows 32q .. 32q+31 of this CTA).  Accumulator row r is source
+// row row_base + r; it is valid when r < rows_here and the source row lies
+// below the group's end.  A 32x32 chunk is read with tcgen05.ld (thread = row),
+// converted to f32 and staged in shared memory, then read back transposed so
+// that 8 lanes cover one row's 32 columns (128 contiguous bytes) and one warp
+// instruction writes 4 row segments.  The dequant runs in the transposed phase,
+// in the op's order ((f32(acc) * scale) * pts + bias) * logit.  Per-row data
+// and this lane's scale/bias columns are fetched before waiting for the
+// accumulator, and TMEM chunk k+1 is loaded while chunk k is written out.
+// Returns false if the wait for the accumulator ran out.
+template <int EPI, int NCH>
+__device__ __forceinline__ bool epilogue_tile(const GemmArgs &args, const TileCoord &c, int64_t row_base,
+                                              int rows_here, uint32_t tmem_acc, int q, int col_begin, int lane,
+                                              uint64_t *tfull_bar, uint32_t use, volatile int *abort_flag,
+                                              const EpiSmem &sm)
+{
+    const int n = args.n;
+    const int sub = lane >> 3;            // row (mod 4) handled in the transposed phase
+    const int col4 = (lane & 7) * 4;      // first of the 4 columns handled in the transposed phase
+    const int r_in = q * 32 + lane;
+    const int64_t i = row_base + r_in;
+    float pts = 1.0f, lg = 1.0f;
+    long long dst = -1;
+    if (r_in < rows_here && i < c.row_end) {
+        if (args.pts) pts = __ldg(args.pts + i);
+        if (args.logit) lg = __ldg(args.logit + i);
+        if (EPI == EPI_ATOMIC) {
+            const int64_t d = load_row_index(args.row_index, args.row_index_type, i);
+            if (d < 0 || d >= args.output_bs) atomicOr(args.status, QGMM_DEV_ROW_INDEX_RANGE);
+            else dst = d;
+        } else {
+            dst = i;
+        }
+    }
+    sm.rp[lane] = pts;
+    sm.rl[lane] = lg;
+    sm.rd[lane] = dst;
+    const bool any = __any_sync(0xffffffffu, dst >= 0);
+    float4 sc[NCH], bs[NCH];
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+        sc[k] = make_float4(1.f, 1.f, 1.f, 1.f);
+        bs[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (EPI != EPI_RAW_ACC && any) {
+        const int64_t base = static_cast<int64_t>(c.g) * n + static_cast<int64_t>(c.nt) * BN + col_begin + col4;
+        if (args.scale) {
+#pragma unroll
+            for (int k = 0; k < NCH; ++k) sc[k] = __ldg(reinterpret_cast<const float4 *>(args.scale + base + k * 32));
+        }
+        if (args.bias) {
+#pragma unroll
+            for (int k = 0; k < NCH; ++k) bs[k] = __ldg(reinterpret_cast<const float4 *>(args.bias + base + k * 32));
+        }
+    }
+    __syncwarp();
+    if (!ptx::mbar_wait(tfull_bar, use, abort_flag)) return false;
+    ptx::tc_fence_after();
+    if (any) {
+        const int64_t n0 = static_cast<int64_t>(c.nt) * BN + col_begin;
+        const uint32_t tbase = tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(col_begin);
+        uint32_t ra[32], rb[32];
+        ptx::tmem_ld_32x32b_x32(tbase, ra);
+#pragma unroll
+        for (int pc = 0; pc < NCH; pc += 2) {
+            ptx::tmem_ld_wait(ra);
+            epi_stage_chunk<EPI>(sm.stage, lane, ra);
+            ptx::tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>((pc + 1) * 32), rb);
+            __syncwarp();
+            epi_write_chunk<EPI>(args, sm.stage, sm.rp, sm.rl, sm.rd, sub, col4, n, n0 + pc * 32, sc[pc], bs[pc]);
+            __syncwarp();
+            ptx::tmem_ld_wait(rb);
+            epi_stage_chunk<EPI>(sm.stage, lane, rb);
+            if (pc + 2 < NCH) ptx::tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>((pc + 2) * 32), ra);
+            __syncwarp();
+            epi_write_chunk<EPI>(args, sm.stage, sm.rp, sm.rl, sm.rd, sub, col4, n, n0 + (pc + 1) * 32, sc[pc + 1],
+                                 bs[pc + 1]);
+            __syncwarp();
+        }
+    }
+    ptx::tc_fence_before();
+    __syncwarp();
+    return true;
+}
+
+// Direct epilogue (int8 kernels): one warp owns TMEM lane quarter q and the
+// EPI_COLS columns [col_begin, col_begin + EPI_COLS) of the tile.  tcgen05.ld
+// .16x256b gives thread t the rows t/4 and t/4 + 8 of a 16-lane half and two
+// adjacent columns of every 8-column block, so 4 threads cover 32 contiguous
+// bytes of a row and each warp instruction reduces 8 rows x 32 bytes (whole
+// sectors) straight from registers; no shared-memory round trip.  Per-row
+// data of the thread's 4 rows and its scale/bias columns are loaded before the
+// wait for the accumulator.  The dequant runs in the op's order
+// ((f32(acc) * scale) * pts + bias) * logit.  Returns false if the wait ran out.
+constexpr int EPI_COLS = 128;
+constexpr int EPI_CHUNKS = EPI_COLS / 64;
+
+template <int EPI>
+__device__ __forceinline__ void epi_direct_rows(const GemmArgs &args, const uint32_t (&v)[32], long long dA,
+                                                long long dB, float pA, float pB, float lA, float lB,
+                                                const float2 (&sc)[8], const float2 (&bs)[8], int n, int64_t col0)
+{
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int64_t col = col0 + 8 * j;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const long long d = h ? dB : dA;
+            if (d < 0) continue;
+            const uint32_t u0 = v[4 * j + 2 * h], u1 = v[4 * j + 2 * h + 1];
+            if constexpr (EPI == EPI_RAW_ACC) {
+                *reinterpret_cast<int2 *>(args.acc_out + d * n + col) =
+                    make_int2(static_cast<int>(u0), static_cast<int>(u1));
+            } else {
+                const float p = h ? pB : pA, l = h ? lB : lA;
+                const float y0 = __fmul_rn(
+                    __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(u0)), sc[j].x), p), bs[j].x), l);
+                const float y1 = __fmul_rn(
+                    __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(u1)), sc[j].y), p), bs[j].y), l);
+                if constexpr (EPI == EPI_ATOMIC) {
+                    ptx::red_add_v2(args.out + d * n + col, y0, y1);
+                } else {
+                    *reinterpret_cast<float2 *>(args.out + d * n + col) = make_float2(y0, y1);
+                }
+            }
+        }
+    }
+}
+
+template <int EPI>
+__device__ __forceinline__ bool epilogue_tile_direct(const GemmArgs &args, const TileCoord &c, int64_t row_base,
+                                                     int rows_here, uint32_t tmem_acc, int q, int col_begin, int lane,
+                                                     uint64_t *tfull_bar, uint32_t use, volatile int *abort_flag)
+{
+    const int n = args.n;
+    const int t0 = lane & 3, t1 = lane >> 2;
+    float pts[4], lg[4];
+    long long dst[4];
+    bool mine = false;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {   // k: (16-lane half) * 2 + (upper 8 rows of the half)
+        const int r_in = q * 32 + (k >> 1) * 16 + (k & 1) * 8 + t1;
+        const int64_t i = row_base + r_in;
+        pts[k] = 1.0f;
+        lg[k] = 1.0f;
+        dst[k] = -1;
+        if (r_in < rows_here && i < c.row_end) {
+            if (args.pts) pts[k] = __ldg(args.pts + i);
+            if (args.logit) lg[k] = __ldg(args.logit + i);
+            if (EPI == EPI_ATOMIC) {
+                const int64_t d = load_row_index(args.row_index, args.row_index_type, i);
+                if (d < 0 || d >= args.output_bs) atomicOr(args.status, QGMM_DEV_ROW_INDEX_RANGE);
+                else dst[k] = d;
+            } else {
+                dst[k] = i;
+            }
+        }
+        mine |= dst[k] >= 0;
+    }
+    const bool any = __any_sync(0xffffffffu, mine);
+    const int64_t n0 = static_cast<int64_t>(c.nt) * BN + col_begin + 2 * t0;
+    float2 sc[EPI_CHUNKS][8], bs[EPI_CHUNKS][8];
+#pragma unroll
+    for (int ch = 0; ch < EPI_CHUNKS; ++ch)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            sc[ch][j] = make_float2(1.f, 1.f);
+            bs[ch][j] = make_float2(0.f, 0.f);
+        }
+    if (EPI != EPI_RAW_ACC && any) {
+        const int64_t base = static_cast<int64_t>(c.g) * n + n0;
+        if (args.scale) {
+#pragma unroll
+            for (int ch = 0; ch < EPI_CHUNKS; ++ch)
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    sc[ch][j] = __ldg(reinterpret_cast<const float2 *>(args.scale + base + 64 * ch + 8 * j));
+        }
+        if (args.bias) {
+#pragma unroll
+            for (int ch = 0; ch < EPI_CHUNKS; ++ch)
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    bs[ch][j] = __ldg(reinterpret_cast<const float2 *>(args.bias + base + 64 * ch + 8 * j));
+        }
+    }
+    __syncwarp();
+    if (!ptx::mbar_wait(tfull_bar, use, abort_flag)) return false;
+    ptx::tc_fence_after();
+    if (any) {
+#pragma unroll
+        for (int ch = 0; ch < EPI_CHUNKS; ++ch) {
+            uint32_t va[32], vb[32];
+            const uint32_t col = tmem_acc + static_cast<uint32_t>(col_begin + 64 * ch);
+            ptx::tmem_ld_16x256b_x8(col + (static_cast<uint32_t>(q * 32) << 16), va);
+            ptx::tmem_ld_16x256b_x8(col + (static_cast<uint32_t>(q * 32 + 16) << 16), vb);
+            ptx::tmem_ld_wait2(va, vb);
+            epi_direct_rows<EPI>(args, va, dst[0], dst[1], pts[0], pts[1], lg[0], lg[1], sc[ch], bs[ch], n,
+                                 n0 + 64 * ch);
+            epi_direct_rows<EPI>(args, vb, dst[2], dst[3], pts[2], pts[3], lg[2], lg[3], sc[ch], bs[ch], n,
+                                 n0 + 64 * ch);
+        }
+    }
+    ptx::tc_fence_before();
+    __syncwarp();
+    return true;
+}
+
 // ---------------------------------------------------------------- K2
 template <int EPI, bool W4>
 __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
@@ -286,7 +513,7 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(&tfull[b], 1);
-            ptx::mbar_init(&tempty[b], 4);
+            ptx::mbar_init(&tempty[b], Cfg::EPI_WARPS);
         }
         ptx::mbar_init(drain, 1);
         *abort_flag = 0;
@@ -419,101 +646,36 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
             ptx::mbar_wait(drain, 0, &never);
         }
         __syncwarp();
-    } else if (warp < 6) {
-        // ------------------------------------------------ epilogue (TMEM -> registers -> smem -> global)
-        // Each warp owns one TMEM lane quarter (32 accumulator rows).  A 32x32
-        // chunk is read with tcgen05.ld (thread = row), converted to f32 and
-        // staged in shared memory; it is then read back transposed so that 8
-        // lanes cover one row's 32 columns (128 contiguous bytes) and one warp
-        // instruction writes 4 whole rows segments.  The dequant arithmetic runs
-        // in the transposed phase, in the op's order:
-        //   ((f32(acc) * scale) * pts + bias) * logit
+    } else if (!W4) {
+        // ------------------------------------------------ epilogue, int8: 8 warps, direct from TMEM
         const int q = warp & 3;
-        const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
-        float *stage = epi_stage + q * (32 * EPI_LD);
-        float *rp = row_pts + q * 32;
-        float *rl = row_lg + q * 32;
-        long long *rd = row_dst + q * 32;
-        const int n = args.n;
-        const int sub = lane >> 3;            // row (mod 4) handled in the transposed phase
-        const int col4 = (lane & 7) * 4;      // first of the 4 columns handled in the transposed phase
+        const int col_begin = ((warp - 2) >> 2) * EPI_COLS;
         int lt = 0;
         for (int t = blockIdx.x; t < T; t += gridDim.x, ++lt) {
             const TileCoord c = tile_coord(t, MT, SW, off, cum, e, tile_rows);
             const int buf = lt & 1;
             const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
-            // per-row data of this warp's 32 rows, fetched while the MMA still runs
-            const int r_in = q * 32 + lane;
-            const int64_t i = static_cast<int64_t>(c.row0) + r_in;
-            float pts = 1.0f, lg = 1.0f;
-            long long dst = -1;
-            if (r_in < tile_rows && i < c.row_end) {
-                if (args.pts) pts = __ldg(args.pts + i);
-                if (args.logit) lg = __ldg(args.logit + i);
-                if (EPI == EPI_ATOMIC) {
-                    const int64_t d = load_row_index(args.row_index, args.row_index_type, i);
-                    if (d < 0 || d >= args.output_bs) atomicOr(args.status, QGMM_DEV_ROW_INDEX_RANGE);
-                    else dst = d;
-                } else {
-                    dst = i;
-                }
-            }
-            rp[lane] = pts;
-            rl[lane] = lg;
-            rd[lane] = dst;
-            const bool any = __any_sync(0xffffffffu, dst >= 0);
-            // this lane's 4 columns of every 32-column chunk of scale and bias
-            float4 sc[NCHUNK], bs[NCHUNK];
-#pragma unroll
-            for (int k = 0; k < NCHUNK; ++k) {
-                sc[k] = make_float4(1.f, 1.f, 1.f, 1.f);
-                bs[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-            if (EPI != EPI_RAW_ACC && any) {
-                const int64_t base = static_cast<int64_t>(c.g) * n + static_cast<int64_t>(c.nt) * BN + col4;
-                if (args.scale) {
-#pragma unroll
-                    for (int k = 0; k < NCHUNK; ++k)
-                        sc[k] = __ldg(reinterpret_cast<const float4 *>(args.scale + base + k * 32));
-                }
-                if (args.bias) {
-#pragma unroll
-                    for (int k = 0; k < NCHUNK; ++k)
-                        bs[k] = __ldg(reinterpret_cast<const float4 *>(args.bias + base + k * 32));
-                }
-            }
-            __syncwarp();
-            if (!ptx::mbar_wait(&tfull[buf], use, abort_flag)) {
+            if (!epilogue_tile_direct<EPI>(args, c, c.row0, tile_rows, tmem_base + static_cast<uint32_t>(buf * BN), q,
+                                           col_begin, lane, &tfull[buf], use, abort_flag)) {
                 fail();
                 break;
             }
-            ptx::tc_fence_after();
-            if (any) {
-                const int64_t n0 = static_cast<int64_t>(c.nt) * BN;
-                const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(buf * BN);
-                // tcgen05.ld of chunk 0 first; chunk k+1 is issued while chunk k is written out
-                uint32_t ra[32], rb[32];
-                ptx::tmem_ld_32x32b_x32(tbase, ra);
-#pragma unroll
-                for (int pc = 0; pc < NCHUNK; pc += 2) {
-                    ptx::tmem_ld_wait(ra);
-                    epi_stage_chunk<EPI>(stage, lane, ra);
-                    ptx::tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>((pc + 1) * 32), rb);
-                    __syncwarp();
-                    epi_write_chunk<EPI>(args, stage, rp, rl, rd, sub, col4, n, n0 + pc * 32, sc[pc], bs[pc]);
-                    __syncwarp();
-                    ptx::tmem_ld_wait(rb);
-                    epi_stage_chunk<EPI>(stage, lane, rb);
-                    if (pc + 2 < NCHUNK)
-                        ptx::tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>((pc + 2) * 32), ra);
-                    __syncwarp();
-                    epi_write_chunk<EPI>(args, stage, rp, rl, rd, sub, col4, n, n0 + (pc + 1) * 32, sc[pc + 1],
-                                         bs[pc + 1]);
-                    __syncwarp();
-                }
+            if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------ epilogue, W4: 4 warps, staged through smem
+        const int q = warp & 3;
+        const EpiSmem sm = epi_smem(epi_stage, row_pts, row_lg, row_dst, q);
+        int lt = 0;
+        for (int t = blockIdx.x; t < T; t += gridDim.x, ++lt) {
+            const TileCoord c = tile_coord(t, MT, SW, off, cum, e, tile_rows);
+            const int buf = lt & 1;
+            const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
+            if (!epilogue_tile<EPI, NCHUNK>(args, c, c.row0, tile_rows, tmem_base + static_cast<uint32_t>(buf * BN), q,
+                                            0, lane, &tfull[buf], use, abort_flag, sm)) {
+                fail();
+                break;
             }
-            ptx::tc_fence_before();
-            __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
         }
     } else if constexpr (W4) {
@@ -563,6 +725,228 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
     if (warp == 1) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- K2, CTA-pair form
+// Two CTAs of a cluster share one 256 x 256 tile: each loads 128 rows of x1
+// and 128 columns of the expert's weights, the leader issues
+// tcgen05.mma.cta_group::2 (M = 256, N = 256) that reads both CTAs' halves, and
+// each CTA's TMEM receives its own 128 accumulator rows.  Per SM this moves a
+// third fewer operand bytes per MAC than the single-CTA 128 x 256 tile, and the
+// same shared memory holds six stages instead of four.
+constexpr int PAIR_ROWS = 256;                 // rows per pair tile
+constexpr int PAIR_A_BYTES = 128 * BK;         // this CTA's rows
+constexpr int PAIR_B_BYTES = BK * 128;         // this CTA's columns (one MN-major atom)
+
+struct PairCfg {
+    static constexpr int STAGES = 5;
+    static constexpr int THREADS = 320;        // producer, MMA, 8 epilogue warps
+    static constexpr int STAGE_BYTES = PAIR_A_BYTES + PAIR_B_BYTES;
+    static constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 1;
+    static constexpr int CTRL_BYTES = (NUM_BARS * 8 + 16 + 15) / 16 * 16;
+    static constexpr int TABLE_BYTES = (2 * (MAX_E + 1) * 4 + 15) / 16 * 16;
+    static constexpr int EPI_STAGE_BYTES = 8 * 32 * EPI_LD * 4;   // 8 epilogue warps x 32 rows x 32 cols (+pad)
+    static constexpr int ROWINFO_BYTES = 8 * 32 * 16;
+    static constexpr size_t OFF_CTRL = size_t(STAGES) * STAGE_BYTES;
+    static constexpr size_t OFF_TABLE = OFF_CTRL + CTRL_BYTES;
+    static constexpr size_t OFF_EPI = OFF_TABLE + TABLE_BYTES;
+    static constexpr size_t OFF_ROWS = OFF_EPI + EPI_STAGE_BYTES;
+    static constexpr size_t SMEM_BYTES = 1024 + OFF_ROWS + ROWINFO_BYTES;
+    static_assert(SMEM_BYTES <= 232448, "shared memory above the sm_100 per-block limit");
+};
+
+template <int EPI>
+__global__ void __launch_bounds__(PairCfg::THREADS, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                             const GemmArgs args)
+{
+    constexpr int S = PairCfg::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *smem_a = smem;
+    uint8_t *smem_b = smem_a + S * PAIR_A_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + PairCfg::OFF_CTRL);
+    uint64_t *full = bars;            // leader: both CTAs' operands landed
+    uint64_t *empty = bars + S;       // both: pair MMAs finished reading the stage
+    uint64_t *tfull = bars + 2 * S;   // both: accumulator buffer ready
+    uint64_t *tempty = tfull + 2;     // leader: both CTAs' epilogues drained the buffer
+    uint64_t *drain = tempty + 2;     // leader: all issued MMAs completed
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + PairCfg::NUM_BARS);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    int32_t *off = reinterpret_cast<int32_t *>(smem + PairCfg::OFF_TABLE);
+    int32_t *cum = off + (MAX_E + 1);
+    float *epi_stage = reinterpret_cast<float *>(smem + PairCfg::OFF_EPI);
+    float *row_pts = reinterpret_cast<float *>(smem + PairCfg::OFF_ROWS);
+    float *row_lg = row_pts + 8 * 32;
+    long long *row_dst = reinterpret_cast<long long *>(row_lg + 8 * 32);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = ptx::cluster_ctarank();
+    const bool leader = rank == 0;
+    const int cluster = blockIdx.x >> 1;
+    const int nclusters = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&tfull[b], 1);
+            ptx::mbar_init(&tempty[b], 16);   // 8 epilogue warps in each CTA
+        }
+        ptx::mbar_init(drain, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0) {
+        const uint32_t flags =
+            decode_groups_warp(args.group_list, args.e, args.group_list_type, args.m, PAIR_ROWS, off, cum);
+        if (lane == 0) {
+            if (flags && blockIdx.x == 0) atomicOr(args.status, flags);
+            ptx::prefetch_tmap(&map_a);
+            ptx::prefetch_tmap(&map_b);
+        }
+    } else if (warp == 1) {
+        ptx::tmem_alloc_pair(tmem_holder, TMEM_COLS);
+        ptx::tmem_relinquish_pair();
+    }
+    ptx::tc_fence_before();
+    ptx::cluster_sync();   // barriers of both CTAs initialised before any TMA or remote arrive
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    const int e = args.e;
+    const int MT = cum[e];
+    const int NT = args.n / BN;
+    const int SW = args.slab_ntiles;
+    const int T = MT * NT;
+    const int KB = args.k / BK;
+
+    auto fail = [&]() {
+        atomicOr(args.status, QGMM_DEV_TIMEOUT);
+        *abort_flag = 1;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            constexpr uint32_t TX = 2u * (PAIR_A_BYTES + PAIR_B_BYTES);   // both halves count on the leader
+            uint32_t issued[S];
+#pragma unroll
+            for (int s = 0; s < S; ++s) issued[s] = 0;
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int t = cluster; t < T && ok; t += nclusters) {
+                const TileCoord c = tile_coord(t, MT, SW, off, cum, e, PAIR_ROWS);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+                        fail();
+                        ok = false;
+                        break;
+                    }
+                    if (leader) ptx::mbar_arrive_expect_tx(&full[stage], TX);
+                    const uint32_t fb = ptx::map_to_rank(&full[stage], 0);
+                    ptx::tma_load_2d_pair(smem_a + stage * PAIR_A_BYTES, &map_a, fb, kb * BK,
+                                          c.row0 + 128 * static_cast<int>(rank));
+                    ptx::tma_load_3d_pair(smem_b + stage * PAIR_B_BYTES, &map_b, fb,
+                                          c.nt * BN + 128 * static_cast<int>(rank), kb * BK, c.g);
+                    ++issued[stage];
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok && leader) {
+                for (int s = 0; s < S; ++s) {
+                    if (issued[s] == 0) continue;
+                    volatile int never = 0;
+                    ptx::mbar_wait(&full[s], (issued[s] - 1u) & 1u, &never);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (leader CTA only)
+        if (lane == 0 && leader) {
+            constexpr uint32_t IDESC = ptx::idesc_i8(2 * BM, BN, true);
+            int stage = 0;
+            uint32_t phase = 0;
+            int lt = 0;
+            bool ok = true;
+            for (int t = cluster; t < T && ok; t += nclusters, ++lt) {
+                const int buf = lt & 1;
+                const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
+                if (!ptx::mbar_wait(&tempty[buf], use ^ 1u, abort_flag)) {
+                    fail();
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!ptx::mbar_wait(&full[stage], phase, abort_flag)) {
+                        fail();
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t a0 = ptx::smem_addr(smem_a + stage * PAIR_A_BYTES);
+                    const uint32_t b0 = ptx::smem_addr(smem_b + stage * PAIR_B_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+                        const uint64_t adesc = ptx::smem_desc_sw128(a0 + kk * UMMA_K, 16, 1024);
+                        const uint64_t bdesc = ptx::smem_desc_sw128(b0 + kk * UMMA_K * 128, B_ATOM_BYTES, 1024);
+                        ptx::mma_i8_pair(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    ptx::mma_commit_pair(ptx::map_to_rank(&empty[stage], 0));
+                    ptx::mma_commit_pair(ptx::map_to_rank(&empty[stage], 1));
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (ok) {
+                    ptx::mma_commit_pair(ptx::map_to_rank(&tfull[buf], 0));
+                    ptx::mma_commit_pair(ptx::map_to_rank(&tfull[buf], 1));
+                }
+            }
+            ptx::mma_commit_pair(ptx::map_to_rank(drain, 0));
+            volatile int never = 0;
+            ptx::mbar_wait(drain, 0, &never);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ epilogue (both CTAs, own 128 rows)
+        const int q = warp & 3;
+        const int col_begin = ((warp - 2) >> 2) * EPI_COLS;
+        const EpiSmem sm = epi_smem(epi_stage, row_pts, row_lg, row_dst, warp - 2);
+        uint32_t tempty_leader[2];
+        tempty_leader[0] = ptx::map_to_rank(&tempty[0], 0);
+        tempty_leader[1] = ptx::map_to_rank(&tempty[1], 0);
+        int lt = 0;
+        for (int t = cluster; t < T; t += nclusters, ++lt) {
+            const TileCoord c = tile_coord(t, MT, SW, off, cum, e, PAIR_ROWS);
+            const int buf = lt & 1;
+            const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
+            if (!epilogue_tile<EPI, EPI_COLS / 32>(args, c, static_cast<int64_t>(c.row0) + 128 * static_cast<int>(rank),
+                                                   128, tmem_base + static_cast<uint32_t>(buf * BN), q, col_begin, lane,
+                                                   &tfull[buf], use, abort_flag, sm)) {
+                fail();
+                break;
+            }
+            if (lane == 0) ptx::mbar_arrive_cluster(tempty_leader[buf]);
+        }
+    }
+
+    ptx::tc_fence_before();
+    ptx::cluster_sync();   // no remote arrive or pair MMA still targets either CTA
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc_pair(tmem_base, TMEM_COLS);
     }
 }
 

@@ -32,6 +32,8 @@ struct DeviceInfo {
     int sms = 0;
     int major = 0;
     bool attr_set[3][2] = {};
+    bool pair_attr_set[3] = {};
+    int pair_clusters[3] = {};   // co-resident CTA pairs of the pair kernel, per epilogue kind
 };
 
 std::mutex g_mu;
@@ -123,6 +125,7 @@ struct Plan {
     int tile_rows;
     int slab_ntiles;
     int grid;
+    bool pair;   // CTA-pair kernel (tcgen05 cta_group::2, 256-row tiles)
 };
 
 Plan make_plan(const qgmm_problem *p, int sms, int epi)
@@ -136,9 +139,11 @@ Plan make_plan(const qgmm_problem *p, int sms, int epi)
     const int NT = static_cast<int>(p->n / BN);
     int sw = NT;
     if (epi == EPI_ATOMIC) {
-        // keep one slab of the output (output_bs x slab columns, f32) within ~48 MB of L2
+        // One slab of the output (output_bs x slab columns, f32) of at most ~128 MB,
+        // the L2 size: wider slabs let the combine's reductions miss L2, narrower
+        // ones re-read x1 once per slab.
         const double per_ntile = double(p->output_bs) * BN * 4.0;
-        const double budget = 48.0 * 1024 * 1024;
+        const double budget = 128.0 * 1024 * 1024;
         sw = 1;
         for (int d = 1; d <= NT; ++d)
             if (NT % d == 0 && d * per_ntile <= budget) sw = d;
@@ -147,10 +152,15 @@ Plan make_plan(const qgmm_problem *p, int sms, int epi)
     if (forced_sw > 0 && forced_sw <= NT && NT % forced_sw == 0) sw = forced_sw;
     pl.slab_ntiles = sw;
 
-    const int64_t max_mt = (p->m + pl.tile_rows - 1) / pl.tile_rows + p->e;
+    // Full-height tiles of int8 weights run on CTA pairs; decode-sized tiles and
+    // int4 weights on single CTAs.
+    pl.pair = pl.tile_rows == 128 && p->weight_type == QGMM_W_INT8 && env_int("QGMM_PAIR", 1) != 0;
+    const int rows_per_tile = pl.pair ? 256 : pl.tile_rows;
+    const int64_t max_mt = (p->m + rows_per_tile - 1) / rows_per_tile + p->e;
     const int64_t max_tiles = max_mt * NT;
     pl.grid = static_cast<int>(max_tiles < sms ? max_tiles : sms);
     if (pl.grid < 1) pl.grid = 1;
+    if (pl.pair) pl.grid = static_cast<int>(2 * (max_tiles < sms / 2 ? max_tiles : sms / 2));
     return pl;
 }
 
@@ -210,14 +220,59 @@ qgmm_status launch_gemm_t(DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma
     return cudaGetLastError() == cudaSuccess ? QGMM_OK : QGMM_ERR_CUDA;
 }
 
+template <int EPI>
+qgmm_status launch_pair_t(DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma, const CUtensorMap &mb,
+                          const GemmArgs &a, cudaStream_t st)
+{
+    auto kern = grouped_gemm_pair_kernel<EPI>;
+    const size_t smem = PairCfg::SMEM_BYTES;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(PairCfg::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!dev->pair_attr_set[EPI]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+                return QGMM_ERR_CUDA;
+            cfg.gridDim = dim3(static_cast<unsigned>(dev->sms & ~1), 1, 1);
+            int clusters = 0;
+            if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1)
+                return QGMM_ERR_CUDA;
+            dev->pair_clusters[EPI] = clusters;
+            dev->pair_attr_set[EPI] = true;
+        }
+    }
+    int grid = pl.grid;
+    if (grid > 2 * dev->pair_clusters[EPI]) grid = 2 * dev->pair_clusters[EPI];
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    if (cudaLaunchKernelEx(&cfg, kern, ma, mb, a) != cudaSuccess) return QGMM_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? QGMM_OK : QGMM_ERR_CUDA;
+}
+
 qgmm_status launch_gemm(int epi, DeviceInfo *dev, const qgmm_problem *p, const Plan &pl, const CUtensorMap &ma,
                         const CUtensorMap &mb, const GemmArgs &a, cudaStream_t st)
 {
     const bool w4 = p->weight_type == QGMM_W_INT4_PACKED_INT32;
     if (std::getenv("QGMM_LOG"))
-        std::fprintf(stderr, "qgmm: gemm epi=%d w4=%d m=%lld k=%lld n=%lld e=%lld tile_rows=%d slab=%d grid=%d\n", epi,
-                     int(w4), (long long)p->m, (long long)p->k, (long long)p->n, (long long)p->e, pl.tile_rows,
-                     pl.slab_ntiles, pl.grid);
+        std::fprintf(stderr,
+                     "qgmm: gemm epi=%d w4=%d pair=%d m=%lld k=%lld n=%lld e=%lld tile_rows=%d slab=%d grid=%d\n",
+                     epi, int(w4), int(pl.pair), (long long)p->m, (long long)p->k, (long long)p->n, (long long)p->e,
+                     pl.tile_rows, pl.slab_ntiles, pl.grid);
+    if (pl.pair) {
+        switch (epi) {
+        case EPI_ATOMIC: return launch_pair_t<EPI_ATOMIC>(dev, pl, ma, mb, a, st);
+        case EPI_STORE_Y: return launch_pair_t<EPI_STORE_Y>(dev, pl, ma, mb, a, st);
+        default: return launch_pair_t<EPI_RAW_ACC>(dev, pl, ma, mb, a, st);
+        }
+    }
     switch (epi) {
     case EPI_ATOMIC: return w4 ? launch_gemm_t<EPI_ATOMIC, true>(dev, pl, ma, mb, a, st)
                                : launch_gemm_t<EPI_ATOMIC, false>(dev, pl, ma, mb, a, st);
