@@ -35,6 +35,26 @@ constexpr int EPI_LD = 36;                   // staging row stride in floats (co
 
 enum Epilogue : int { EPI_ATOMIC = 0, EPI_STORE_Y = 1, EPI_RAW_ACC = 2 };
 
+// Row tiling of each expert's rows.  A group of r rows has h = ceil(r / 128)
+// half tiles of 128 rows.
+//   SCHED_TILES      ceil(r / tile_rows) tiles of tile_rows rows (single CTA)
+//   SCHED_PAIRS      floor(h / 2) pair tiles of 256 rows (CTA pair); an odd
+//                    last half tile is left to a SCHED_TAILS launch
+//   SCHED_PAIRS_ALL  ceil(h / 2) pair tiles of 256 rows, tails included
+//   SCHED_TAILS      h % 2 tiles: the group's last 128 rows when h is odd
+enum Schedule : int { SCHED_TILES = 0, SCHED_PAIRS = 1, SCHED_PAIRS_ALL = 2, SCHED_TAILS = 3 };
+
+__device__ __forceinline__ int32_t tiles_of_group(int64_t rows, int sched, int tile_rows)
+{
+    const int64_t h = (rows + 127) / 128;
+    switch (sched) {
+    case SCHED_PAIRS: return static_cast<int32_t>(h / 2);
+    case SCHED_PAIRS_ALL: return static_cast<int32_t>((h + 1) / 2);
+    case SCHED_TAILS: return static_cast<int32_t>(h & 1);
+    default: return static_cast<int32_t>((rows + tile_rows - 1) / tile_rows);
+    }
+}
+
 template <bool W4>
 struct GemmCfg {
     static constexpr int STAGES = W4 ? 3 : 4;
@@ -61,6 +81,7 @@ struct GemmArgs {
     int32_t e, group_list_type;
     int32_t k, n;
     int32_t tile_rows;     // rows per m-tile = TMA box height of x1 (16, 32, 64 or 128)
+    int32_t sched;         // which m-tiles this launch covers (SCHED_*)
     int32_t slab_ntiles;   // n-tiles per slab; divides n / BN
     const float *scale, *pts, *logit, *bias;
     const void *row_index;
@@ -78,7 +99,7 @@ struct GemmArgs {
 // (type 0: running max of clamp(end, 0, m); type 1: clamp of the running sum
 // of max(count, 0)); the returned QGMM_DEV_* bits say what was wrong.
 __device__ __forceinline__ uint32_t decode_groups_warp(const int64_t *gl, int e, int type, int64_t m,
-                                                       int tile_rows, int32_t *off, int32_t *cum)
+                                                       int tile_rows, int sched, int32_t *off, int32_t *cum)
 {
     const int lane = threadIdx.x & 31;
     uint32_t flags = 0;
@@ -121,7 +142,7 @@ __device__ __forceinline__ uint32_t decode_groups_warp(const int64_t *gl, int e,
         int64_t start = __shfl_up_sync(0xffffffffu, end, 1);
         if (lane == 0) start = carry_end;
         const int64_t rows = end - start;
-        int32_t mt = in ? static_cast<int32_t>((rows + tile_rows - 1) / tile_rows) : 0;
+        int32_t mt = in ? tiles_of_group(rows, sched, tile_rows) : 0;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
             const int32_t o = __shfl_up_sync(0xffffffffu, mt, d);
@@ -151,7 +172,7 @@ struct TileCoord {
 // (taken by neighbouring CTAs at the same time) share one x1 row tile and one
 // expert's weight columns, and one slab of the output stays hot in L2.
 __device__ __forceinline__ TileCoord tile_coord(int t, int MT, int SW, const int32_t *off, const int32_t *cum,
-                                                int e, int tile_rows)
+                                                int e, int tile_rows, int sched)
 {
     const int per_slab = MT * SW;
     const int s = t / per_slab;
@@ -166,8 +187,13 @@ __device__ __forceinline__ TileCoord tile_coord(int t, int MT, int SW, const int
         else hi = mid;
     }
     c.g = lo;
-    c.row0 = off[lo] + (mt - cum[lo]) * tile_rows;
     c.row_end = off[lo + 1];
+    if (sched == SCHED_TAILS)
+        c.row0 = off[lo] + 128 * ((off[lo + 1] - off[lo] + 127) / 128 - 1);
+    else if (sched == SCHED_PAIRS || sched == SCHED_PAIRS_ALL)
+        c.row0 = off[lo] + (mt - cum[lo]) * 256;
+    else
+        c.row0 = off[lo] + (mt - cum[lo]) * tile_rows;
     return c;
 }
 
@@ -519,11 +545,12 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
+    volatile uint32_t *group_flags = reinterpret_cast<volatile uint32_t *>(tmem_holder + 2);
     if (warp == 0) {
         const uint32_t flags = decode_groups_warp(args.group_list, args.e, args.group_list_type, args.m,
-                                                  args.tile_rows, off, cum);
+                                                  args.tile_rows, args.sched, off, cum);
         if (lane == 0) {
-            if (flags && blockIdx.x == 0) atomicOr(args.status, flags);
+            *group_flags = flags;
             ptx::prefetch_tmap(&map_a);
             ptx::prefetch_tmap(&map_b);
         }
@@ -560,7 +587,7 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
             uint32_t phase = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < T && ok; t += gridDim.x) {
-                const TileCoord c = tile_coord(t, MT, SW, off, cum, e, tile_rows);
+                const TileCoord c = tile_coord(t, MT, SW, off, cum, e, tile_rows, args.sched);
                 const int n0 = c.nt * BN;
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
@@ -648,11 +675,13 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
         __syncwarp();
     } else if (!W4) {
         // ------------------------------------------------ epilogue, int8: 8 warps, direct from TMEM
+        ptx::pdl_wait_primary();   // the output (and status word) are initialised by the previous kernel
+        if (warp == 2 && lane == 0 && blockIdx.x == 0 && *group_flags) atomicOr(args.status, *group_flags);
         const int q = warp & 3;
         const int col_begin = ((warp - 2) >> 2) * EPI_COLS;
         int lt = 0;
         for (int t = blockIdx.x; t < T; t += gridDim.x, ++lt) {
-            const TileCoord c = tile_coord(t, MT, SW, off, cum, e, tile_rows);
+            const TileCoord c = tile_coord(t, MT, SW, off, cum, e, tile_rows, args.sched);
             const int buf = lt & 1;
             const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
             if (!epilogue_tile_direct<EPI>(args, c, c.row0, tile_rows, tmem_base + static_cast<uint32_t>(buf * BN), q,
@@ -664,11 +693,13 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
         }
     } else if (warp < 6) {
         // ------------------------------------------------ epilogue, W4: 4 warps, staged through smem
+        ptx::pdl_wait_primary();
+        if (warp == 2 && lane == 0 && blockIdx.x == 0 && *group_flags) atomicOr(args.status, *group_flags);
         const int q = warp & 3;
         const EpiSmem sm = epi_smem(epi_stage, row_pts, row_lg, row_dst, q);
         int lt = 0;
         for (int t = blockIdx.x; t < T; t += gridDim.x, ++lt) {
-            const TileCoord c = tile_coord(t, MT, SW, off, cum, e, tile_rows);
+            const TileCoord c = tile_coord(t, MT, SW, off, cum, e, tile_rows, args.sched);
             const int buf = lt & 1;
             const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
             if (!epilogue_tile<EPI, NCHUNK>(args, c, c.row0, tile_rows, tmem_base + static_cast<uint32_t>(buf * BN), q,
@@ -801,11 +832,12 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
+    volatile uint32_t *group_flags = reinterpret_cast<volatile uint32_t *>(tmem_holder + 2);
     if (warp == 0) {
         const uint32_t flags =
-            decode_groups_warp(args.group_list, args.e, args.group_list_type, args.m, PAIR_ROWS, off, cum);
+            decode_groups_warp(args.group_list, args.e, args.group_list_type, args.m, PAIR_ROWS, args.sched, off, cum);
         if (lane == 0) {
-            if (flags && blockIdx.x == 0) atomicOr(args.status, flags);
+            *group_flags = flags;
             ptx::prefetch_tmap(&map_a);
             ptx::prefetch_tmap(&map_b);
         }
@@ -841,7 +873,9 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             uint32_t phase = 0;
             bool ok = true;
             for (int t = cluster; t < T && ok; t += nclusters) {
-                const TileCoord c = tile_coord(t, MT, SW, off, cum, e, PAIR_ROWS);
+                const TileCoord c = tile_coord(t, MT, SW, off, cum, e, PAIR_ROWS, args.sched);
+                const int my_row = c.row0 + 128 * static_cast<int>(rank);
+                const int my_col = c.nt * BN + 128 * static_cast<int>(rank);
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
                         fail();
@@ -850,10 +884,8 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
                     }
                     if (leader) ptx::mbar_arrive_expect_tx(&full[stage], TX);
                     const uint32_t fb = ptx::map_to_rank(&full[stage], 0);
-                    ptx::tma_load_2d_pair(smem_a + stage * PAIR_A_BYTES, &map_a, fb, kb * BK,
-                                          c.row0 + 128 * static_cast<int>(rank));
-                    ptx::tma_load_3d_pair(smem_b + stage * PAIR_B_BYTES, &map_b, fb,
-                                          c.nt * BN + 128 * static_cast<int>(rank), kb * BK, c.g);
+                    ptx::tma_load_2d_pair(smem_a + stage * PAIR_A_BYTES, &map_a, fb, kb * BK, my_row);
+                    ptx::tma_load_3d_pair(smem_b + stage * PAIR_B_BYTES, &map_b, fb, my_col, kb * BK, c.g);
                     ++issued[stage];
                     if (++stage == S) {
                         stage = 0;
@@ -921,6 +953,8 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue (both CTAs, own 128 rows)
+        ptx::pdl_wait_primary();   // the output (and status word) are initialised by the previous kernel
+        if (warp == 2 && lane == 0 && blockIdx.x == 0 && *group_flags) atomicOr(args.status, *group_flags);
         const int q = warp & 3;
         const int col_begin = ((warp - 2) >> 2) * EPI_COLS;
         const EpiSmem sm = epi_smem(epi_stage, row_pts, row_lg, row_dst, warp - 2);
@@ -929,7 +963,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         tempty_leader[1] = ptx::map_to_rank(&tempty[1], 0);
         int lt = 0;
         for (int t = cluster; t < T; t += nclusters, ++lt) {
-            const TileCoord c = tile_coord(t, MT, SW, off, cum, e, PAIR_ROWS);
+            const TileCoord c = tile_coord(t, MT, SW, off, cum, e, PAIR_ROWS, args.sched);
             const int buf = lt & 1;
             const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
             if (!epilogue_tile<EPI, EPI_COLS / 32>(args, c, static_cast<int64_t>(c.row0) + 128 * static_cast<int>(rank),
@@ -957,6 +991,7 @@ __global__ void output_init_kernel(float *__restrict__ out, int64_t output_bs, i
                                    const uint16_t *__restrict__ shared, int64_t shared_bs, int64_t shared_off,
                                    uint32_t *status)
 {
+    ptx::pdl_launch_dependents();   // the grouped GEMM may start its prologue and mainloop now
     if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
     const int64_t q_per_row = n / 4;
     const int64_t total = output_bs * q_per_row;
@@ -978,6 +1013,7 @@ __global__ void output_init_kernel(float *__restrict__ out, int64_t output_bs, i
 
 __global__ void clear_status_kernel(uint32_t *status)
 {
+    ptx::pdl_launch_dependents();
     *status = 0u;
 }
 
@@ -996,7 +1032,7 @@ __device__ __forceinline__ int64_t groups_total_block(const int64_t *gl, int e, 
                                                       int32_t *cum, uint32_t *status, bool report)
 {
     if (threadIdx.x < 32) {
-        const uint32_t f = decode_groups_warp(gl, e, type, m, BM, off, cum);
+        const uint32_t f = decode_groups_warp(gl, e, type, m, BM, SCHED_TILES, off, cum);
         if (threadIdx.x == 0 && report && f) atomicOr(status, f);
     }
     __syncthreads();

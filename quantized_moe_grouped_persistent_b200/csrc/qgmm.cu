@@ -216,7 +216,19 @@ qgmm_status launch_gemm_t(DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma
             dev->attr_set[EPI][W4 ? 1 : 0] = true;
         }
     }
-    kern<<<pl.grid, GemmCfg<W4>::THREADS, smem, st>>>(ma, mb, a);
+    // Programmatic dependent launch: the GEMM's prologue and mainloop may
+    // overlap the preceding output-init kernel; its epilogue waits for it.
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.grid), 1, 1);
+    cfg.blockDim = dim3(GemmCfg<W4>::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, ma, mb, a) != cudaSuccess) return QGMM_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? QGMM_OK : QGMM_ERR_CUDA;
 }
 
@@ -227,16 +239,18 @@ qgmm_status launch_pair_t(DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma
     auto kern = grouped_gemm_pair_kernel<EPI>;
     const size_t smem = PairCfg::SMEM_BYTES;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.blockDim = dim3(PairCfg::THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 1;   // the occupancy query below uses the cluster shape only
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (!dev->pair_attr_set[EPI]) {
@@ -253,6 +267,7 @@ qgmm_status launch_pair_t(DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma
     int grid = pl.grid;
     if (grid > 2 * dev->pair_clusters[EPI]) grid = 2 * dev->pair_clusters[EPI];
     cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, kern, ma, mb, a) != cudaSuccess) return QGMM_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? QGMM_OK : QGMM_ERR_CUDA;
 }
@@ -267,10 +282,28 @@ qgmm_status launch_gemm(int epi, DeviceInfo *dev, const qgmm_problem *p, const P
                      epi, int(w4), int(pl.pair), (long long)p->m, (long long)p->k, (long long)p->n, (long long)p->e,
                      pl.tile_rows, pl.slab_ntiles, pl.grid);
     if (pl.pair) {
+        // Pairs of 128-row half tiles on CTA pairs; a group's odd last half tile
+        // (its final <= 128 rows) goes to a single-CTA launch right after, so no
+        // pair tile is half empty.
+        const bool tails = env_int("QGMM_PAIR_TAILS", 1) != 0;
+        GemmArgs ap = a;
+        ap.sched = tails ? SCHED_PAIRS : SCHED_PAIRS_ALL;
+        qgmm_status s = QGMM_OK;
         switch (epi) {
-        case EPI_ATOMIC: return launch_pair_t<EPI_ATOMIC>(dev, pl, ma, mb, a, st);
-        case EPI_STORE_Y: return launch_pair_t<EPI_STORE_Y>(dev, pl, ma, mb, a, st);
-        default: return launch_pair_t<EPI_RAW_ACC>(dev, pl, ma, mb, a, st);
+        case EPI_ATOMIC: s = launch_pair_t<EPI_ATOMIC>(dev, pl, ma, mb, ap, st); break;
+        case EPI_STORE_Y: s = launch_pair_t<EPI_STORE_Y>(dev, pl, ma, mb, ap, st); break;
+        default: s = launch_pair_t<EPI_RAW_ACC>(dev, pl, ma, mb, ap, st); break;
+        }
+        if (s != QGMM_OK || !tails) return s;
+        GemmArgs at = a;
+        at.sched = SCHED_TAILS;
+        Plan pt = pl;
+        const int64_t tail_tiles = p->e * (p->n / BN);
+        pt.grid = static_cast<int>(tail_tiles < dev->sms ? tail_tiles : dev->sms);
+        switch (epi) {
+        case EPI_ATOMIC: return launch_gemm_t<EPI_ATOMIC, false>(dev, pt, ma, mb, at, st);
+        case EPI_STORE_Y: return launch_gemm_t<EPI_STORE_Y, false>(dev, pt, ma, mb, at, st);
+        default: return launch_gemm_t<EPI_RAW_ACC, false>(dev, pt, ma, mb, at, st);
         }
     }
     switch (epi) {
@@ -294,6 +327,7 @@ GemmArgs base_args(const qgmm_problem *p, const int64_t *group_list, const Plan 
     a.k = static_cast<int32_t>(p->k);
     a.n = static_cast<int32_t>(p->n);
     a.tile_rows = pl.tile_rows;
+    a.sched = SCHED_TILES;
     a.slab_ntiles = pl.slab_ntiles;
     a.row_index_type = p->row_index_type;
     a.output_bs = p->output_bs;
