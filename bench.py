@@ -166,6 +166,27 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+# ----------------------------------------------------------------------------- ranks
+def rank_seed(spec_index: int, rank: int):
+    """Seed of rank `rank`'s batch: rank 0 uses the workload's own seed, others an offset one."""
+    from synth.inputs import SEED_BASE
+    return None if rank == 0 else SEED_BASE + spec_index + 1000 * rank
+
+
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise max of per-rank timings (every rank takes part; all get the result)."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def weak_scaling_value(world: int, ops_per_rank: float, ms_max: float) -> float:
+    """Whole-job effective TOPS: every rank's work over the slowest rank's time."""
+    return world * ops_per_rank / (ms_max * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------------------- device timing
 def time_steps(d, steps, warmup, deterministic, dist=None):
     """Device time of `steps` back-to-back calls (CUDA events on the launch stream),
@@ -322,7 +343,6 @@ def reference_arm(args, p, spec_desc):
 def main():
     args = parse_args()
     from synth import CONFIGS, make_problem
-    from synth.inputs import SEED_BASE
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -351,8 +371,7 @@ def main():
         torch.cuda.set_device(0)
     dev_index = torch.cuda.current_device()
 
-    seed = SEED_BASE + spec.index + 1000 * rank
-    p = make_problem(args.workload, seed=seed if rank else None, tokens=args.tokens, e=args.experts)
+    p = make_problem(args.workload, seed=rank_seed(spec.index, rank), tokens=args.tokens, e=args.experts)
     if args.tokens or args.experts:
         spec_desc += f" (reduced: tokens={p.tokens}, e={p.e})"
     d = DeviceProblem(p)
@@ -367,11 +386,8 @@ def main():
     sampler.start()
     ms, gemm_ms = time_steps(d, args.steps, args.warmup, args.deterministic, dist)
     clocks = sampler.stop()
-    mx = torch.tensor([ms, gemm_ms], dtype=torch.float64, device="cuda")
-    if dist is not None:
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-    ms_max, gemm_max = float(mx[0]), float(mx[1])
-    value = world * ops / (ms_max * 1e-3) / 1e12
+    ms_max, gemm_max = max_over_ranks([ms, gemm_ms], dist, device="cuda")
+    value = weak_scaling_value(world, ops, ms_max)
     launches_per_step = (7 if args.deterministic else 2) + (1 if d.prologue else 0)
 
     extras = {}

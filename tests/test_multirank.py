@@ -1,0 +1,68 @@
+"""The multi-GPU plumbing of bench.py, run as two gloo ranks on the CPU.
+
+Every rank takes the same collective steps; each rank draws its own batch
+(weak scaling, no data-path collective); the reported time is the max over
+ranks and the value all ranks' work over that time.
+"""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    import datetime
+    import torch.distributed as dist
+    import bench
+    from synth import make_problem
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        mine = [1.0 + rank, 10.0 - rank]                    # different per-rank timings
+        got = bench.max_over_ranks(mine, dist, device="cpu")
+        p = make_problem("tiny", seed=bench.rank_seed(1, rank))
+        dist.barrier()
+        import hashlib
+        out.put((rank, got, hashlib.sha256(p.x1.tobytes()).hexdigest(), hashlib.sha256(p.row_index.tobytes()).hexdigest()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_reduce_max_and_draw_distinct_batches():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for pr in procs:
+        pr.start()
+    results = [q.get(timeout=120) for _ in range(world)]
+    for pr in procs:
+        pr.join(timeout=60)
+        assert pr.exitcode == 0
+    results.sort()
+    for _, got, _, _ in results:
+        assert got == [2.0, 10.0]                          # max over ranks, on every rank
+    assert results[0][2:] != results[1][2:]                # each rank its own seeded batch
+
+
+def test_weak_scaling_value_and_seeds():
+    import bench
+    assert bench.weak_scaling_value(4, 2e12, 1.0) == pytest.approx(8000.0)
+    assert bench.rank_seed(4, 0) is None
+    assert bench.rank_seed(4, 1) != bench.rank_seed(4, 2)
+    assert bench.max_over_ranks([3.0, 1.5]) == [3.0, 1.5]  # single process: unchanged
