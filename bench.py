@@ -377,7 +377,11 @@ def main():
     d = DeviceProblem(p)
     ops = int_ops(p)
     peaks = load_peaks()
-    int8_peak_sustained = 2.0 * peaks["bf16_sustained"]   # dense int8 = 2 x dense bf16 (nominal ratio)
+    # dense int8 = 2 x dense bf16 (nominal ratio).  The timed region (tens of ms)
+    # runs before the power cap pulls the clocks down, so the burst figure is the
+    # roofline denominator; the sustained one is reported beside it.
+    int8_peak = 2.0 * peaks["bf16"]
+    int8_peak_sustained = 2.0 * peaks["bf16_sustained"]
 
     sampler = ClockSampler(dev_index)
     d.run(deterministic=args.deterministic)                # first call: module load, tensor maps
@@ -439,11 +443,14 @@ def main():
                        "l2": "inputs larger than L2 (x2 %.2f GB per rank), no flush" % (p.x2.nbytes / 1e9),
                        "parallelism": f"dp{world} (independent batch per GPU)"},
             "pct_of_dense_int8_peak": {"nominal_4500": 100.0 * value / world / NOMINAL_INT8_TOPS,
+                                       "measured_burst": 100.0 * value / world / int8_peak,
                                        "measured_sustained": 100.0 * value / world / int8_peak_sustained},
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": int8_peak_sustained, "unit": "TOPS",
-                         "frac": achieved / int8_peak_sustained, "traffic": committed_traffic(args.workload),
-                         "kernel": "grouped_gemm_kernel", "kernel_ms": gemm_max,
-                         "peak_source": f"{peaks['source']} bf16 sustained x 2 (dense int8 : bf16 nominal ratio)"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TOPS",
+                         "frac": achieved / int8_peak, "traffic": committed_traffic(args.workload),
+                         "kernel": "grouped GEMM (grouped_gemm_pair_kernel + tail launch)", "kernel_ms": gemm_max,
+                         "frac_of_sustained": achieved / int8_peak_sustained,
+                         "peak_source": f"{peaks['source']} bf16 burst x 2 (dense int8 : bf16 nominal ratio), "
+                                        f"of measured"},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
             "device_status": flags,
