@@ -82,6 +82,7 @@ struct GemmArgs {
     int32_t k, n;
     int32_t tile_rows;     // rows per m-tile = TMA box height of x1 (16, 32, 64 or 128)
     int32_t sched;         // which m-tiles this launch covers (SCHED_*)
+    int32_t stall_producer;  // test hook: the producer issues no copy, so the MMA wait must run out
     int32_t slab_ntiles;   // n-tiles per slab; divides n / BN
     const float *scale, *pts, *logit, *bias;
     const void *row_index;
@@ -585,7 +586,7 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
             for (int s = 0; s < S; ++s) issued[s] = 0;
             int stage = 0;
             uint32_t phase = 0;
-            bool ok = true;
+            bool ok = args.stall_producer == 0;
             for (int t = blockIdx.x; t < T && ok; t += gridDim.x) {
                 const TileCoord c = tile_coord(t, MT, SW, off, cum, e, tile_rows, args.sched);
                 const int n0 = c.nt * BN;
@@ -871,7 +872,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             for (int s = 0; s < S; ++s) issued[s] = 0;
             int stage = 0;
             uint32_t phase = 0;
-            bool ok = true;
+            bool ok = args.stall_producer == 0;
             for (int t = cluster; t < T && ok; t += nclusters) {
                 const TileCoord c = tile_coord(t, MT, SW, off, cum, e, PAIR_ROWS, args.sched);
                 const int my_row = c.row0 + 128 * static_cast<int>(rank);

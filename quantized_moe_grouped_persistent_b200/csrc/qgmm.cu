@@ -328,6 +328,10 @@ GemmArgs base_args(const qgmm_problem *p, const int64_t *group_list, const Plan 
     a.n = static_cast<int32_t>(p->n);
     a.tile_rows = pl.tile_rows;
     a.sched = SCHED_TILES;
+    // Test hook for the failure path: with QGMM_TEST_STALL_PRODUCER=1 the GEMM's
+    // producer issues no copy, every consumer wait runs out after its one-second
+    // bound, the kernel sets QGMM_DEV_TIMEOUT, frees its TMEM and returns.
+    a.stall_producer = env_int("QGMM_TEST_STALL_PRODUCER", 0) != 0 ? 1 : 0;
     a.slab_ntiles = pl.slab_ntiles;
     a.row_index_type = p->row_index_type;
     a.output_bs = p->output_bs;

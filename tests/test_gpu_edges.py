@@ -1,0 +1,90 @@
+"""GPU parity on edge shapes: minimum sizes, the expert limit, tile-boundary group
+sizes on both the single-CTA and the CTA-pair paths, rows past the groups'
+total, and unusual k / n.  Same bars as test_gpu_parity (bit-exact int32,
+deterministic mode bitwise equal to the oracle's fixed-order f32, atomic mode
+within 2e-5 of the sum of |terms|).
+"""
+from types import SimpleNamespace
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+pytestmark = pytest.mark.gpu
+
+ATOMIC_TOL = 2e-5
+
+
+@pytest.fixture(scope="module")
+def dev(qgmm):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from quantized_moe_grouped_persistent_b200 import device
+    return device
+
+
+def _problem(seed, counts, k, n, extra_rows=0, output_bs=None, weight="int8", bias=True):
+    rng = np.random.default_rng(seed)
+    counts = np.asarray(counts, np.int64)
+    e = counts.size
+    total = int(counts.sum())
+    m = total + extra_rows
+    obs = output_bs or max(1, (total + 3) // 4)
+    x2 = (rng.integers(-127, 128, size=(e, k, n), dtype=np.int8) if weight == "int8"
+          else rng.integers(0, 2 ** 32, size=(e, k, n // 8), dtype=np.uint32).view(np.int32))
+    return SimpleNamespace(
+        m=m, k=k, n=n, e=e, output_bs=obs, weight=weight, group_list_type=1, counts=counts,
+        x1=rng.integers(-127, 128, size=(m, k), dtype=np.int8), x_bf16=None, x2=x2,
+        scale=rng.uniform(1e-3, 1e-2, size=(e, n)).astype(np.float32),
+        pertoken_scale=rng.uniform(1e-3, 1e-2, size=m).astype(np.float32),
+        group_list=counts.copy(), logit=rng.uniform(0.05, 1.0, size=m).astype(np.float32),
+        row_index=rng.integers(0, obs, size=m).astype(np.int64),
+        bias=rng.normal(0, 0.01, size=(e, n)).astype(np.float32) if bias else None,
+        shared=None, shared_offset=0)
+
+
+def _check(dev, oracle, p, hint):
+    d = dev.DeviceProblem(p, expected_m_per_expert=hint)
+    o64, sabs, o32 = oracle.problem_finalize(p)
+    det = d.run(deterministic=True).cpu().numpy()
+    assert d.status(True) == 0
+    np.testing.assert_array_equal(det, o32)
+    atom = d.run(deterministic=False).cpu().numpy()
+    assert d.status(False) == 0
+    err = np.abs(atom.astype(np.float64) - o64) / np.where(sabs > 0, sabs, 1.0)
+    assert err.max() <= ATOMIC_TOL
+    total = int(p.counts.sum())
+    acc = d.accum().cpu().numpy()
+    ref = oracle.accum(p.x1, p.x2, p.group_list, p.group_list_type, weight=p.weight)
+    np.testing.assert_array_equal(acc[:total], ref[:total])
+
+
+def test_single_row_single_expert_minimum_sizes(dev, oracle):
+    _check(dev, oracle, _problem(1, [1], 128, 256, output_bs=1), 0)
+
+
+def test_expert_limit_mostly_empty(dev, oracle):
+    counts = np.zeros(1024, np.int64)
+    counts[[0, 511, 1023]] = [3, 40, 5]
+    _check(dev, oracle, _problem(2, counts, 128, 256, bias=False), 0)
+
+
+@pytest.mark.parametrize("hint", [1, 200])     # single-CTA 16-row tiles / CTA-pair 256-row tiles + tails
+def test_tile_boundary_group_sizes(dev, oracle, hint):
+    counts = [127, 128, 129, 0, 255, 256, 257, 383, 1]
+    _check(dev, oracle, _problem(3, counts, 256, 512), hint)
+
+
+@pytest.mark.parametrize("hint", [0, 200])
+def test_rows_past_the_total_are_ignored(dev, oracle, hint):
+    _check(dev, oracle, _problem(4, [100, 0, 300], 256, 512, extra_rows=77), hint)
+
+
+@pytest.mark.parametrize("k,n", [(128, 256), (256, 1792), (4096, 256)])
+def test_unusual_k_and_n(dev, oracle, k, n):
+    _check(dev, oracle, _problem(5, [40, 260, 7], k, n), 0)
+
+
+def test_int4_on_tile_boundaries(dev, oracle):
+    _check(dev, oracle, _problem(6, [128, 129, 1, 256], 256, 512, weight="int4"), 0)
