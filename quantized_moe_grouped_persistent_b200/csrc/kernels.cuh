@@ -42,14 +42,17 @@ enum Epilogue : int { EPI_ATOMIC = 0, EPI_STORE_Y = 1, EPI_RAW_ACC = 2 };
 //                    last half tile is left to a SCHED_TAILS launch
 //   SCHED_PAIRS_ALL  ceil(h / 2) pair tiles of 256 rows, tails included
 //   SCHED_TAILS      h % 2 tiles: the group's last 128 rows when h is odd
-enum Schedule : int { SCHED_TILES = 0, SCHED_PAIRS = 1, SCHED_PAIRS_ALL = 2, SCHED_TAILS = 3 };
+//   SCHED_PAIRS_TAIL128  ceil(h / 2) pair tiles; when h is odd the last one is an
+//                    M = 128 pair tile (64 rows per CTA) over the final <= 128 rows
+enum Schedule : int { SCHED_TILES = 0, SCHED_PAIRS = 1, SCHED_PAIRS_ALL = 2, SCHED_TAILS = 3, SCHED_PAIRS_TAIL128 = 4 };
 
 __device__ __forceinline__ int32_t tiles_of_group(int64_t rows, int sched, int tile_rows)
 {
     const int64_t h = (rows + 127) / 128;
     switch (sched) {
     case SCHED_PAIRS: return static_cast<int32_t>(h / 2);
-    case SCHED_PAIRS_ALL: return static_cast<int32_t>((h + 1) / 2);
+    case SCHED_PAIRS_ALL:
+    case SCHED_PAIRS_TAIL128: return static_cast<int32_t>((h + 1) / 2);
     case SCHED_TAILS: return static_cast<int32_t>(h & 1);
     default: return static_cast<int32_t>((rows + tile_rows - 1) / tile_rows);
     }
@@ -166,6 +169,7 @@ __device__ __forceinline__ uint32_t decode_groups_warp(const int64_t *gl, int e,
 
 struct TileCoord {
     int g, row0, row_end, nt;
+    bool tail;   // SCHED_PAIRS_TAIL128: an M = 128 pair tile
 };
 
 // Tile t of the persistent walk.  Order: slab of slab_ntiles n-tiles, then
@@ -189,7 +193,13 @@ __device__ __forceinline__ TileCoord tile_coord(int t, int MT, int SW, const int
     }
     c.g = lo;
     c.row_end = off[lo + 1];
-    if (sched == SCHED_TAILS)
+    c.tail = false;
+    if (sched == SCHED_PAIRS_TAIL128) {
+        const int h = (off[lo + 1] - off[lo] + 127) / 128;
+        const int j = mt - cum[lo];
+        c.row0 = off[lo] + j * 256;
+        c.tail = (h & 1) && j == h / 2;
+    } else if (sched == SCHED_TAILS)
         c.row0 = off[lo] + 128 * ((off[lo + 1] - off[lo] + 127) / 128 - 1);
     else if (sched == SCHED_PAIRS || sched == SCHED_PAIRS_ALL)
         c.row0 = off[lo] + (mt - cum[lo]) * 256;
@@ -304,14 +314,15 @@ __device__ __forceinline__ EpiSmem epi_smem(float *epi_stage, float *row_pts, fl
 // Returns false if the wait for the accumulator ran out.
 template <int EPI, int NCH>
 __device__ __forceinline__ bool epilogue_tile(const GemmArgs &args, const TileCoord &c, int64_t row_base,
-                                              int rows_here, uint32_t tmem_acc, int q, int col_begin, int lane,
-                                              uint64_t *tfull_bar, uint32_t use, volatile int *abort_flag,
-                                              const EpiSmem &sm)
+                                              int rows_here, int row_off, uint32_t tmem_acc, int q, int tmem_col,
+                                              int glob_col, int lane, uint64_t *tfull_bar, uint32_t use,
+                                              volatile int *abort_flag, const EpiSmem &sm)
 {
     const int n = args.n;
+    const int col_begin = glob_col;       // tile column of this warp's first TMEM column
     const int sub = lane >> 3;            // row (mod 4) handled in the transposed phase
     const int col4 = (lane & 7) * 4;      // first of the 4 columns handled in the transposed phase
-    const int r_in = q * 32 + lane;
+    const int r_in = row_off + lane;
     const int64_t i = row_base + r_in;
     float pts = 1.0f, lg = 1.0f;
     long long dst = -1;
@@ -352,7 +363,7 @@ __device__ __forceinline__ bool epilogue_tile(const GemmArgs &args, const TileCo
     ptx::tc_fence_after();
     if (any) {
         const int64_t n0 = static_cast<int64_t>(c.nt) * BN + col_begin;
-        const uint32_t tbase = tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(col_begin);
+        const uint32_t tbase = tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(tmem_col);
         uint32_t ra[32], rb[32];
         ptx::tmem_ld_32x32b_x32(tbase, ra);
 #pragma unroll
@@ -703,8 +714,9 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
             const TileCoord c = tile_coord(t, MT, SW, off, cum, e, tile_rows, args.sched);
             const int buf = lt & 1;
             const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
-            if (!epilogue_tile<EPI, NCHUNK>(args, c, c.row0, tile_rows, tmem_base + static_cast<uint32_t>(buf * BN), q,
-                                            0, lane, &tfull[buf], use, abort_flag, sm)) {
+            if (!epilogue_tile<EPI, NCHUNK>(args, c, c.row0, tile_rows, q * 32,
+                                            tmem_base + static_cast<uint32_t>(buf * BN), q, 0, 0, lane, &tfull[buf],
+                                            use, abort_flag, sm)) {
                 fail();
                 break;
             }
@@ -875,7 +887,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             bool ok = args.stall_producer == 0;
             for (int t = cluster; t < T && ok; t += nclusters) {
                 const TileCoord c = tile_coord(t, MT, SW, off, cum, e, PAIR_ROWS, args.sched);
-                const int my_row = c.row0 + 128 * static_cast<int>(rank);
+                const int my_row = c.row0 + (c.tail ? 64 : 128) * static_cast<int>(rank);
                 const int my_col = c.nt * BN + 128 * static_cast<int>(rank);
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
@@ -906,12 +918,16 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (leader CTA only)
         if (lane == 0 && leader) {
-            constexpr uint32_t IDESC = ptx::idesc_i8(2 * BM, BN, true);
+            constexpr uint32_t IDESC_FULL = ptx::idesc_i8(2 * BM, BN, true);   // 256 rows: 128 per CTA
+            constexpr uint32_t IDESC_TAIL = ptx::idesc_i8(BM, BN, true);       // 128 rows: 64 per CTA
             int stage = 0;
             uint32_t phase = 0;
             int lt = 0;
             bool ok = true;
             for (int t = cluster; t < T && ok; t += nclusters, ++lt) {
+                const bool tail = args.sched == SCHED_PAIRS_TAIL128 &&
+                                  tile_coord(t, MT, SW, off, cum, e, PAIR_ROWS, args.sched).tail;
+                const uint32_t IDESC = tail ? IDESC_TAIL : IDESC_FULL;
                 const int buf = lt & 1;
                 const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
                 if (!ptx::mbar_wait(&tempty[buf], use ^ 1u, abort_flag)) {
@@ -967,9 +983,22 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             const TileCoord c = tile_coord(t, MT, SW, off, cum, e, PAIR_ROWS, args.sched);
             const int buf = lt & 1;
             const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
-            if (!epilogue_tile<EPI, EPI_COLS / 32>(args, c, static_cast<int64_t>(c.row0) + 128 * static_cast<int>(rank),
-                                                   128, tmem_base + static_cast<uint32_t>(buf * BN), q, col_begin, lane,
-                                                   &tfull[buf], use, abort_flag, sm)) {
+            const uint32_t acc = tmem_base + static_cast<uint32_t>(buf * BN);
+            bool ok;
+            if (c.tail) {
+                // M=128 pair tile: this CTA's 64 rows; TMEM lanes 0-63 hold columns 0-127,
+                // lanes 64-127 hold columns 128-255, in the buffer's first 128 columns.
+                const int half = (warp - 2) >> 2;
+                ok = epilogue_tile<EPI, 2>(args, c, static_cast<int64_t>(c.row0) + 64 * static_cast<int>(rank), 64,
+                                           32 * (q & 1), acc, q, half * 64, (q >> 1) * 128 + half * 64, lane,
+                                           &tfull[buf], use, abort_flag, sm);
+            } else {
+                ok = epilogue_tile<EPI, EPI_COLS / 32>(args, c,
+                                                       static_cast<int64_t>(c.row0) + 128 * static_cast<int>(rank), 128,
+                                                       q * 32, acc, q, col_begin, col_begin, lane, &tfull[buf], use,
+                                                       abort_flag, sm);
+            }
+            if (!ok) {
                 fail();
                 break;
             }

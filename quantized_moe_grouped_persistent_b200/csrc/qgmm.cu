@@ -282,12 +282,16 @@ qgmm_status launch_gemm(int epi, DeviceInfo *dev, const qgmm_problem *p, const P
                      epi, int(w4), int(pl.pair), (long long)p->m, (long long)p->k, (long long)p->n, (long long)p->e,
                      pl.tile_rows, pl.slab_ntiles, pl.grid);
     if (pl.pair) {
-        // Pairs of 128-row half tiles on CTA pairs; a group's odd last half tile
-        // (its final <= 128 rows) goes to a single-CTA launch right after, so no
-        // pair tile is half empty.
-        const bool tails = env_int("QGMM_PAIR_TAILS", 1) != 0;
+        // Pairs of 128-row half tiles on CTA pairs.  A group's odd last half tile
+        // (its final <= 128 rows) goes, by QGMM_PAIR_TAILS:
+        //   1 (default) to a single-CTA launch right after the pair launch;
+        //   2 to an M = 128 pair tile (64 rows per CTA) after the group's other tiles;
+        //   0 to a full 256-row pair tile padded with rows it ignores.
+        // All three give identical results; 1 measured fastest at large prefill.
+        const int tail_mode = env_int("QGMM_PAIR_TAILS", 1);
+        const bool tails = tail_mode == 1;
         GemmArgs ap = a;
-        ap.sched = tails ? SCHED_PAIRS : SCHED_PAIRS_ALL;
+        ap.sched = tail_mode == 2 ? SCHED_PAIRS_TAIL128 : tails ? SCHED_PAIRS : SCHED_PAIRS_ALL;
         qgmm_status s = QGMM_OK;
         switch (epi) {
         case EPI_ATOMIC: s = launch_pair_t<EPI_ATOMIC>(dev, pl, ma, mb, ap, st); break;

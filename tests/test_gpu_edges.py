@@ -88,3 +88,11 @@ def test_unusual_k_and_n(dev, oracle, k, n):
 
 def test_int4_on_tile_boundaries(dev, oracle):
     _check(dev, oracle, _problem(6, [128, 129, 1, 256], 256, 512, weight="int4"), 0)
+
+
+@pytest.mark.parametrize("tail_mode", ["0", "1", "2"])
+def test_pair_tail_modes_are_exact(dev, oracle, monkeypatch, tail_mode):
+    """The three ways of running a group's odd last 128 rows on the CTA-pair path
+    (padded pair tile, single-CTA launch, M=128 pair tile) give identical results."""
+    monkeypatch.setenv("QGMM_PAIR_TAILS", tail_mode)
+    _check(dev, oracle, _problem(7, [1, 128, 129, 255, 256, 300, 383, 0, 640], 256, 768), 200)
