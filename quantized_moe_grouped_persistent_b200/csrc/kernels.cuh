@@ -783,15 +783,21 @@ constexpr int PAIR_ROWS = 256;                 // rows per pair tile
 constexpr int PAIR_A_BYTES = 128 * BK;         // this CTA's rows
 constexpr int PAIR_B_BYTES = BK * 128;         // this CTA's columns (one MN-major atom)
 
+template <bool W4>
 struct PairCfg {
-    static constexpr int STAGES = 5;
-    static constexpr int THREADS = 320;        // producer, MMA, 8 epilogue warps
-    static constexpr int STAGE_BYTES = PAIR_A_BYTES + PAIR_B_BYTES;
-    static constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 1;
+    // int8: 5 stages of (x1 half 16 KB + weight half 16 KB), 8 epilogue warps.
+    // int4: 4 stages of (x1 half 16 KB + unpacked weight half 16 KB + packed half
+    //       8 KB), 4 epilogue warps and 4 unpack warps.
+    static constexpr int STAGES = W4 ? 4 : 5;
+    static constexpr int THREADS = 320;
+    static constexpr int EPI_WARPS = W4 ? 4 : 8;
+    static constexpr int P_BYTES = W4 ? PAIR_B_BYTES / 2 : 0;
+    static constexpr int STAGE_BYTES = PAIR_A_BYTES + PAIR_B_BYTES + P_BYTES;
+    static constexpr int NUM_BARS = 3 * STAGES + 2 + 2 + 1;
     static constexpr int CTRL_BYTES = (NUM_BARS * 8 + 16 + 15) / 16 * 16;
     static constexpr int TABLE_BYTES = (2 * (MAX_E + 1) * 4 + 15) / 16 * 16;
-    static constexpr int EPI_STAGE_BYTES = 8 * 32 * EPI_LD * 4;   // 8 epilogue warps x 32 rows x 32 cols (+pad)
-    static constexpr int ROWINFO_BYTES = 8 * 32 * 16;
+    static constexpr int EPI_STAGE_BYTES = EPI_WARPS * 32 * EPI_LD * 4;   // per warp 32 rows x 32 cols (+pad)
+    static constexpr int ROWINFO_BYTES = EPI_WARPS * 32 * 16;
     static constexpr size_t OFF_CTRL = size_t(STAGES) * STAGE_BYTES;
     static constexpr size_t OFF_TABLE = OFF_CTRL + CTRL_BYTES;
     static constexpr size_t OFF_EPI = OFF_TABLE + TABLE_BYTES;
@@ -800,30 +806,33 @@ struct PairCfg {
     static_assert(SMEM_BYTES <= 232448, "shared memory above the sm_100 per-block limit");
 };
 
-template <int EPI>
-__global__ void __launch_bounds__(PairCfg::THREADS, 1)
+template <int EPI, bool W4>
+__global__ void __launch_bounds__(PairCfg<W4>::THREADS, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                              const GemmArgs args)
 {
-    constexpr int S = PairCfg::STAGES;
+    using Cfg = PairCfg<W4>;
+    constexpr int S = Cfg::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *smem_a = smem;
     uint8_t *smem_b = smem_a + S * PAIR_A_BYTES;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + PairCfg::OFF_CTRL);
+    uint8_t *smem_p = smem_b + S * PAIR_B_BYTES;       // W4: packed int4 weight half
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_CTRL);
     uint64_t *full = bars;            // leader: both CTAs' operands landed
     uint64_t *empty = bars + S;       // both: pair MMAs finished reading the stage
     uint64_t *tfull = bars + 2 * S;   // both: accumulator buffer ready
     uint64_t *tempty = tfull + 2;     // leader: both CTAs' epilogues drained the buffer
     uint64_t *drain = tempty + 2;     // leader: all issued MMAs completed
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + PairCfg::NUM_BARS);
+    uint64_t *pfull = drain + 1;      // W4, both: this CTA's x1 half and packed weight half landed
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + Cfg::NUM_BARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
-    int32_t *off = reinterpret_cast<int32_t *>(smem + PairCfg::OFF_TABLE);
+    int32_t *off = reinterpret_cast<int32_t *>(smem + Cfg::OFF_TABLE);
     int32_t *cum = off + (MAX_E + 1);
-    float *epi_stage = reinterpret_cast<float *>(smem + PairCfg::OFF_EPI);
-    float *row_pts = reinterpret_cast<float *>(smem + PairCfg::OFF_ROWS);
-    float *row_lg = row_pts + 8 * 32;
-    long long *row_dst = reinterpret_cast<long long *>(row_lg + 8 * 32);
+    float *epi_stage = reinterpret_cast<float *>(smem + Cfg::OFF_EPI);
+    float *row_pts = reinterpret_cast<float *>(smem + Cfg::OFF_ROWS);
+    float *row_lg = row_pts + Cfg::EPI_WARPS * 32;
+    long long *row_dst = reinterpret_cast<long long *>(row_lg + Cfg::EPI_WARPS * 32);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -834,12 +843,13 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&full[s], W4 ? 8 : 1);   // W4: the 4 unpack warps of each CTA
             ptx::mbar_init(&empty[s], 1);
+            ptx::mbar_init(&pfull[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(&tfull[b], 1);
-            ptx::mbar_init(&tempty[b], 16);   // 8 epilogue warps in each CTA
+            ptx::mbar_init(&tempty[b], 2 * Cfg::EPI_WARPS);   // the epilogue warps of both CTAs
         }
         ptx::mbar_init(drain, 1);
         *abort_flag = 0;
@@ -895,10 +905,19 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
                         ok = false;
                         break;
                     }
-                    if (leader) ptx::mbar_arrive_expect_tx(&full[stage], TX);
-                    const uint32_t fb = ptx::map_to_rank(&full[stage], 0);
-                    ptx::tma_load_2d_pair(smem_a + stage * PAIR_A_BYTES, &map_a, fb, kb * BK, my_row);
-                    ptx::tma_load_3d_pair(smem_b + stage * PAIR_B_BYTES, &map_b, fb, my_col, kb * BK, c.g);
+                    if constexpr (W4) {
+                        // this CTA's x1 half and packed weight half, counted on its own barrier;
+                        // the unpack warps report to the leader once the int8 half is written
+                        ptx::mbar_arrive_expect_tx(&pfull[stage], PAIR_A_BYTES + Cfg::P_BYTES);
+                        ptx::tma_load_2d(smem_a + stage * PAIR_A_BYTES, &map_a, &pfull[stage], kb * BK, my_row);
+                        ptx::tma_load_3d(smem_p + stage * Cfg::P_BYTES, &map_b, &pfull[stage], my_col / 8, kb * BK,
+                                         c.g);
+                    } else {
+                        if (leader) ptx::mbar_arrive_expect_tx(&full[stage], TX);
+                        const uint32_t fb = ptx::map_to_rank(&full[stage], 0);
+                        ptx::tma_load_2d_pair(smem_a + stage * PAIR_A_BYTES, &map_a, fb, kb * BK, my_row);
+                        ptx::tma_load_3d_pair(smem_b + stage * PAIR_B_BYTES, &map_b, fb, my_col, kb * BK, c.g);
+                    }
                     ++issued[stage];
                     if (++stage == S) {
                         stage = 0;
@@ -906,11 +925,12 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
                     }
                 }
             }
-            if (!ok && leader) {
+            if (!ok && (W4 || leader)) {
+                // let the copies already in flight land before the CTA leaves
                 for (int s = 0; s < S; ++s) {
                     if (issued[s] == 0) continue;
                     volatile int never = 0;
-                    ptx::mbar_wait(&full[s], (issued[s] - 1u) & 1u, &never);
+                    ptx::mbar_wait(W4 ? &pfull[s] : &full[s], (issued[s] - 1u) & 1u, &never);
                 }
             }
         }
@@ -937,7 +957,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
                 ptx::tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!ptx::mbar_wait(&full[stage], phase, abort_flag)) {
+                    if (!ptx::mbar_wait<W4>(&full[stage], phase, abort_flag)) {
                         fail();
                         ok = false;
                         break;
@@ -968,12 +988,14 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             ptx::mbar_wait(drain, 0, &never);
         }
         __syncwarp();
-    } else {
-        // ------------------------------------------------ epilogue (both CTAs, own 128 rows)
+    } else if (warp < 2 + Cfg::EPI_WARPS) {
+        // ------------------------------------------------ epilogue (both CTAs, own rows)
         ptx::pdl_wait_primary();   // the output (and status word) are initialised by the previous kernel
         if (warp == 2 && lane == 0 && blockIdx.x == 0 && *group_flags) atomicOr(args.status, *group_flags);
         const int q = warp & 3;
-        const int col_begin = ((warp - 2) >> 2) * EPI_COLS;
+        // int8: 8 warps, two per TMEM lane quarter, 128 columns each; int4: 4 warps, 256 columns each
+        const int half = W4 ? 0 : (warp - 2) >> 2;
+        const int col_begin = half * EPI_COLS;
         const EpiSmem sm = epi_smem(epi_stage, row_pts, row_lg, row_dst, warp - 2);
         uint32_t tempty_leader[2];
         tempty_leader[0] = ptx::map_to_rank(&tempty[0], 0);
@@ -984,25 +1006,73 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             const int buf = lt & 1;
             const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
             const uint32_t acc = tmem_base + static_cast<uint32_t>(buf * BN);
+            const int64_t base_tail = static_cast<int64_t>(c.row0) + 64 * static_cast<int>(rank);
+            const int64_t base_full = static_cast<int64_t>(c.row0) + 128 * static_cast<int>(rank);
             bool ok;
             if (c.tail) {
                 // M=128 pair tile: this CTA's 64 rows; TMEM lanes 0-63 hold columns 0-127,
                 // lanes 64-127 hold columns 128-255, in the buffer's first 128 columns.
-                const int half = (warp - 2) >> 2;
-                ok = epilogue_tile<EPI, 2>(args, c, static_cast<int64_t>(c.row0) + 64 * static_cast<int>(rank), 64,
-                                           32 * (q & 1), acc, q, half * 64, (q >> 1) * 128 + half * 64, lane,
-                                           &tfull[buf], use, abort_flag, sm);
+                if constexpr (W4)
+                    ok = epilogue_tile<EPI, 4>(args, c, base_tail, 64, 32 * (q & 1), acc, q, 0, (q >> 1) * 128, lane,
+                                               &tfull[buf], use, abort_flag, sm);
+                else
+                    ok = epilogue_tile<EPI, 2>(args, c, base_tail, 64, 32 * (q & 1), acc, q, half * 64,
+                                               (q >> 1) * 128 + half * 64, lane, &tfull[buf], use, abort_flag, sm);
             } else {
-                ok = epilogue_tile<EPI, EPI_COLS / 32>(args, c,
-                                                       static_cast<int64_t>(c.row0) + 128 * static_cast<int>(rank), 128,
-                                                       q * 32, acc, q, col_begin, col_begin, lane, &tfull[buf], use,
-                                                       abort_flag, sm);
+                if constexpr (W4)
+                    ok = epilogue_tile<EPI, NCHUNK>(args, c, base_full, 128, q * 32, acc, q, 0, 0, lane, &tfull[buf],
+                                                    use, abort_flag, sm);
+                else
+                    ok = epilogue_tile<EPI, EPI_COLS / 32>(args, c, base_full, 128, q * 32, acc, q, col_begin,
+                                                           col_begin, lane, &tfull[buf], use, abort_flag, sm);
             }
             if (!ok) {
                 fail();
                 break;
             }
             if (lane == 0) ptx::mbar_arrive_cluster(tempty_leader[buf]);
+        }
+    } else if constexpr (W4) {
+        // ------------------------------------------------ int4 -> int8 unpack of this CTA's weight half
+        // Packed stage: BK rows x 64 bytes (128 columns, 8 per int32 word).  Unpacked:
+        // one 128-column MN-major atom, BK rows x 128 bytes, 128-byte swizzle.
+        const int ut = threadIdx.x - (2 + Cfg::EPI_WARPS) * 32;   // 0..127
+        const uint32_t full_leader0 = ptx::map_to_rank(&full[0], 0);
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int t = cluster; t < T && ok; t += nclusters) {
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!ptx::mbar_wait(&pfull[stage], phase, abort_flag)) {
+                    fail();
+                    ok = false;
+                    break;
+                }
+                const uint8_t *pk = smem_p + stage * Cfg::P_BYTES;
+                uint8_t *bb = smem_b + stage * PAIR_B_BYTES;
+                const int qc = ut & 3;                   // 16-byte packed chunk: columns 32*qc .. 32*qc+31
+#pragma unroll
+                for (int it = 0; it < 4; ++it) {
+                    const int kr = (ut >> 2) + 32 * it;  // k row within the stage
+                    const uint4 w = *reinterpret_cast<const uint4 *>(pk + kr * 64 + qc * 16);
+                    uint4 o0, o1;
+                    unpack_int4x8(w.x, o0.x, o0.y);
+                    unpack_int4x8(w.y, o0.z, o0.w);
+                    unpack_int4x8(w.z, o1.x, o1.y);
+                    unpack_int4x8(w.w, o1.z, o1.w);
+                    const int c0 = 2 * qc;               // 16-column chunk inside the atom
+                    uint8_t *rowp = bb + kr * 128;
+                    *reinterpret_cast<uint4 *>(rowp + ((c0 ^ (kr & 7)) << 4)) = o0;
+                    *reinterpret_cast<uint4 *>(rowp + (((c0 + 1) ^ (kr & 7)) << 4)) = o1;
+                }
+                ptx::fence_async_shared();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive_cluster_release(full_leader0 + stage * 8u);
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
         }
     }
 

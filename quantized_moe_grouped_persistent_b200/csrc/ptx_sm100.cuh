@@ -69,15 +69,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return done != 0;
 }
 
+// try_wait with cluster-scope acquire: pairs with arrives that release at
+// cluster scope from the peer CTA of a pair.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
 // Wait until the phase with parity `parity` of `bar` has completed.
 // Returns false on timeout or when *abort becomes non-zero.
+template <bool CLUSTER_ACQUIRE = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort)
 {
     const uint32_t b = smem_addr(bar);
-    if (mbar_try_wait(b, parity)) return true;
+    auto tw = [&]() { return CLUSTER_ACQUIRE ? mbar_try_wait_cluster(b, parity) : mbar_try_wait(b, parity); };
+    if (tw()) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(b, parity)) return true;
+        if (tw()) return true;
         if ((it & 63u) == 0) {
             if (*abort) return false;
             if (globaltimer() - t0 > kWaitTimeoutNs) return false;
@@ -335,6 +352,14 @@ __device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank)
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
 {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Arrive on an mbarrier given by its cluster-window address with a cluster-scope
+// release: this thread's earlier shared-memory writes (made visible to the async
+// proxy) are ordered before the arrive for the peer CTA's tensor-core reads.
+__device__ __forceinline__ void mbar_arrive_cluster_release(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // TMA tile loads into this CTA's shared memory whose completion is counted on

@@ -32,8 +32,8 @@ struct DeviceInfo {
     int sms = 0;
     int major = 0;
     bool attr_set[3][2] = {};
-    bool pair_attr_set[3] = {};
-    int pair_clusters[3] = {};   // co-resident CTA pairs of the pair kernel, per epilogue kind
+    bool pair_attr_set[3][2] = {};
+    int pair_clusters[3][2] = {};   // co-resident CTA pairs of the pair kernel, per epilogue and weight kind
 };
 
 std::mutex g_mu;
@@ -152,9 +152,12 @@ Plan make_plan(const qgmm_problem *p, int sms, int epi)
     if (forced_sw > 0 && forced_sw <= NT && NT % forced_sw == 0) sw = forced_sw;
     pl.slab_ntiles = sw;
 
-    // Full-height tiles of int8 weights run on CTA pairs; decode-sized tiles and
-    // int4 weights on single CTAs.
-    pl.pair = pl.tile_rows == 128 && p->weight_type == QGMM_W_INT8 && env_int("QGMM_PAIR", 1) != 0;
+    // Full-height tiles of int8 weights run on CTA pairs; decode-sized tiles run on
+    // single CTAs.  int4 weights run on single CTAs unless QGMM_PAIR_W4=1: the pair
+    // form (each CTA unpacks its own 128-column half) is exact but measured slower
+    // (W4A8 at 256 and 512 rows per expert: 1.22 / 2.07 ms against 0.89 / 1.64 ms).
+    pl.pair = pl.tile_rows == 128 && env_int("QGMM_PAIR", 1) != 0 &&
+              (p->weight_type == QGMM_W_INT8 || env_int("QGMM_PAIR_W4", 0) != 0);
     const int rows_per_tile = pl.pair ? 256 : pl.tile_rows;
     const int64_t max_mt = (p->m + rows_per_tile - 1) / rows_per_tile + p->e;
     const int64_t max_tiles = max_mt * NT;
@@ -164,8 +167,12 @@ Plan make_plan(const qgmm_problem *p, int sms, int epi)
     return pl;
 }
 
-qgmm_status make_maps(const qgmm_problem *p, const int8_t *x1, const void *x2, int tile_rows, CUtensorMap *ma,
-                      CUtensorMap *mb)
+// x1 map (box: 128 bytes x tile_rows) and weight map: int8 box 128 columns x BK
+// rows; packed int4 box w4_box_words int32 words (8 columns each) x BK rows --
+// 32 words (256 columns) for the single-CTA kernel, 16 (one CTA's 128 columns)
+// for the CTA pair.
+qgmm_status make_maps(const qgmm_problem *p, const int8_t *x1, const void *x2, int tile_rows, int w4_box_words,
+                      CUtensorMap *ma, CUtensorMap *mb)
 {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return QGMM_ERR_CUDA;
@@ -192,7 +199,7 @@ qgmm_status make_maps(const qgmm_problem *p, const int8_t *x1, const void *x2, i
         const cuuint64_t words = cuuint64_t(p->n / 8);
         const cuuint64_t gdim[3] = {words, cuuint64_t(p->k), cuuint64_t(p->e)};
         const cuuint64_t gstride[2] = {words * 4, words * 4 * cuuint64_t(p->k)};
-        const cuuint32_t box[3] = {32, cuuint32_t(BK), 1};
+        const cuuint32_t box[3] = {cuuint32_t(w4_box_words), cuuint32_t(BK), 1};
         const cuuint32_t es[3] = {1, 1, 1};
         if (enc(mb, CU_TENSOR_MAP_DATA_TYPE_INT32, 3, const_cast<void *>(x2), gdim, gstride, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -232,12 +239,12 @@ qgmm_status launch_gemm_t(DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma
     return cudaGetLastError() == cudaSuccess ? QGMM_OK : QGMM_ERR_CUDA;
 }
 
-template <int EPI>
+template <int EPI, bool W4>
 qgmm_status launch_pair_t(DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma, const CUtensorMap &mb,
                           const GemmArgs &a, cudaStream_t st)
 {
-    auto kern = grouped_gemm_pair_kernel<EPI>;
-    const size_t smem = PairCfg::SMEM_BYTES;
+    auto kern = grouped_gemm_pair_kernel<EPI, W4>;
+    const size_t smem = PairCfg<W4>::SMEM_BYTES;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -246,34 +253,36 @@ qgmm_status launch_pair_t(DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma
     attr[0].val.clusterDim.z = 1;
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.blockDim = dim3(PairCfg::THREADS, 1, 1);
+    cfg.blockDim = dim3(PairCfg<W4>::THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;   // the occupancy query below uses the cluster shape only
     {
         std::lock_guard<std::mutex> lk(g_mu);
-        if (!dev->pair_attr_set[EPI]) {
+        if (!dev->pair_attr_set[EPI][W4 ? 1 : 0]) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
                 return QGMM_ERR_CUDA;
             cfg.gridDim = dim3(static_cast<unsigned>(dev->sms & ~1), 1, 1);
             int clusters = 0;
             if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1)
                 return QGMM_ERR_CUDA;
-            dev->pair_clusters[EPI] = clusters;
-            dev->pair_attr_set[EPI] = true;
+            dev->pair_clusters[EPI][W4 ? 1 : 0] = clusters;
+            dev->pair_attr_set[EPI][W4 ? 1 : 0] = true;
         }
     }
     int grid = pl.grid;
-    if (grid > 2 * dev->pair_clusters[EPI]) grid = 2 * dev->pair_clusters[EPI];
+    if (grid > 2 * dev->pair_clusters[EPI][W4 ? 1 : 0]) grid = 2 * dev->pair_clusters[EPI][W4 ? 1 : 0];
     cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
     cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, kern, ma, mb, a) != cudaSuccess) return QGMM_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? QGMM_OK : QGMM_ERR_CUDA;
 }
 
+// mb: weight map of the main launch; mb_tail: weight map of the single-CTA
+// tail launch (they differ only for int4 weights on CTA pairs).
 qgmm_status launch_gemm(int epi, DeviceInfo *dev, const qgmm_problem *p, const Plan &pl, const CUtensorMap &ma,
-                        const CUtensorMap &mb, const GemmArgs &a, cudaStream_t st)
+                        const CUtensorMap &mb, const CUtensorMap &mb_tail, const GemmArgs &a, cudaStream_t st)
 {
     const bool w4 = p->weight_type == QGMM_W_INT4_PACKED_INT32;
     if (std::getenv("QGMM_LOG"))
@@ -294,9 +303,12 @@ qgmm_status launch_gemm(int epi, DeviceInfo *dev, const qgmm_problem *p, const P
         ap.sched = tail_mode == 2 ? SCHED_PAIRS_TAIL128 : tails ? SCHED_PAIRS : SCHED_PAIRS_ALL;
         qgmm_status s = QGMM_OK;
         switch (epi) {
-        case EPI_ATOMIC: s = launch_pair_t<EPI_ATOMIC>(dev, pl, ma, mb, ap, st); break;
-        case EPI_STORE_Y: s = launch_pair_t<EPI_STORE_Y>(dev, pl, ma, mb, ap, st); break;
-        default: s = launch_pair_t<EPI_RAW_ACC>(dev, pl, ma, mb, ap, st); break;
+        case EPI_ATOMIC: s = w4 ? launch_pair_t<EPI_ATOMIC, true>(dev, pl, ma, mb, ap, st)
+                                : launch_pair_t<EPI_ATOMIC, false>(dev, pl, ma, mb, ap, st); break;
+        case EPI_STORE_Y: s = w4 ? launch_pair_t<EPI_STORE_Y, true>(dev, pl, ma, mb, ap, st)
+                                 : launch_pair_t<EPI_STORE_Y, false>(dev, pl, ma, mb, ap, st); break;
+        default: s = w4 ? launch_pair_t<EPI_RAW_ACC, true>(dev, pl, ma, mb, ap, st)
+                        : launch_pair_t<EPI_RAW_ACC, false>(dev, pl, ma, mb, ap, st); break;
         }
         if (s != QGMM_OK || !tails) return s;
         GemmArgs at = a;
@@ -305,9 +317,12 @@ qgmm_status launch_gemm(int epi, DeviceInfo *dev, const qgmm_problem *p, const P
         const int64_t tail_tiles = p->e * (p->n / BN);
         pt.grid = static_cast<int>(tail_tiles < dev->sms ? tail_tiles : dev->sms);
         switch (epi) {
-        case EPI_ATOMIC: return launch_gemm_t<EPI_ATOMIC, false>(dev, pt, ma, mb, at, st);
-        case EPI_STORE_Y: return launch_gemm_t<EPI_STORE_Y, false>(dev, pt, ma, mb, at, st);
-        default: return launch_gemm_t<EPI_RAW_ACC, false>(dev, pt, ma, mb, at, st);
+        case EPI_ATOMIC: return w4 ? launch_gemm_t<EPI_ATOMIC, true>(dev, pt, ma, mb_tail, at, st)
+                                   : launch_gemm_t<EPI_ATOMIC, false>(dev, pt, ma, mb_tail, at, st);
+        case EPI_STORE_Y: return w4 ? launch_gemm_t<EPI_STORE_Y, true>(dev, pt, ma, mb_tail, at, st)
+                                    : launch_gemm_t<EPI_STORE_Y, false>(dev, pt, ma, mb_tail, at, st);
+        default: return w4 ? launch_gemm_t<EPI_RAW_ACC, true>(dev, pt, ma, mb_tail, at, st)
+                           : launch_gemm_t<EPI_RAW_ACC, false>(dev, pt, ma, mb_tail, at, st);
         }
     }
     switch (epi) {
@@ -388,8 +403,12 @@ qgmm_status finalize_impl(const qgmm_problem *p, const int8_t *x1, const void *x
     uint32_t *status = static_cast<uint32_t *>(workspace);
     const int epi = p->deterministic ? EPI_STORE_Y : EPI_ATOMIC;
     const Plan pl = make_plan(p, dev->sms, epi);
-    CUtensorMap ma, mb;
-    if ((s = make_maps(p, x1, x2, pl.tile_rows, &ma, &mb)) != QGMM_OK) return s;
+    CUtensorMap ma, mb, mb_tail;
+    if ((s = make_maps(p, x1, x2, pl.tile_rows, pl.pair ? 16 : 32, &ma, &mb)) != QGMM_OK) return s;
+    mb_tail = mb;
+    if (pl.pair && p->weight_type == QGMM_W_INT4_PACKED_INT32 &&
+        (s = make_maps(p, x1, x2, pl.tile_rows, 32, &ma, &mb_tail)) != QGMM_OK)
+        return s;
 
     GemmArgs a = base_args(p, group_list, pl, status);
     a.scale = scale;
@@ -406,7 +425,7 @@ qgmm_status finalize_impl(const qgmm_problem *p, const int8_t *x1, const void *x
         if (cudaGetLastError() != cudaSuccess) return QGMM_ERR_CUDA;
         a.out = out;
         if (ev_begin && cudaEventRecord(ev_begin, st) != cudaSuccess) return QGMM_ERR_CUDA;
-        if ((s = launch_gemm(EPI_ATOMIC, dev, p, pl, ma, mb, a, st)) != QGMM_OK) return s;
+        if ((s = launch_gemm(EPI_ATOMIC, dev, p, pl, ma, mb, mb_tail, a, st)) != QGMM_OK) return s;
         if (ev_end && cudaEventRecord(ev_end, st) != cudaSuccess) return QGMM_ERR_CUDA;
         return QGMM_OK;
     }
@@ -428,7 +447,7 @@ qgmm_status finalize_impl(const qgmm_problem *p, const int8_t *x1, const void *x
     if (cudaGetLastError() != cudaSuccess) return QGMM_ERR_CUDA;
     a.out = y;
     if (ev_begin && cudaEventRecord(ev_begin, st) != cudaSuccess) return QGMM_ERR_CUDA;
-    if ((s = launch_gemm(EPI_STORE_Y, dev, p, pl, ma, mb, a, st)) != QGMM_OK) return s;
+    if ((s = launch_gemm(EPI_STORE_Y, dev, p, pl, ma, mb, mb_tail, a, st)) != QGMM_OK) return s;
     if (ev_end && cudaEventRecord(ev_end, st) != cudaSuccess) return QGMM_ERR_CUDA;
     det_reduce_kernel<<<grid_for(p->output_bs, 1, dev->sms, 8), 256, 0, st>>>(
         out, y, static_cast<int32_t>(p->n), starts, list, p->output_bs, shared, p->shared_bs, p->shared_offset);
@@ -474,13 +493,17 @@ QGMM_API qgmm_status qgmm_debug_accum(const qgmm_problem *p, const int8_t *x1, c
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     uint32_t *status = static_cast<uint32_t *>(workspace);
     const Plan pl = make_plan(p, dev->sms, EPI_RAW_ACC);
-    CUtensorMap ma, mb;
-    if ((s = make_maps(p, x1, x2, pl.tile_rows, &ma, &mb)) != QGMM_OK) return s;
+    CUtensorMap ma, mb, mb_tail;
+    if ((s = make_maps(p, x1, x2, pl.tile_rows, pl.pair ? 16 : 32, &ma, &mb)) != QGMM_OK) return s;
+    mb_tail = mb;
+    if (pl.pair && p->weight_type == QGMM_W_INT4_PACKED_INT32 &&
+        (s = make_maps(p, x1, x2, pl.tile_rows, 32, &ma, &mb_tail)) != QGMM_OK)
+        return s;
     clear_status_kernel<<<1, 1, 0, st>>>(status);
     if (cudaGetLastError() != cudaSuccess) return QGMM_ERR_CUDA;
     GemmArgs a = base_args(p, group_list, pl, status);
     a.acc_out = acc_out;
-    return launch_gemm(EPI_RAW_ACC, dev, p, pl, ma, mb, a, st);
+    return launch_gemm(EPI_RAW_ACC, dev, p, pl, ma, mb, mb_tail, a, st);
 }
 
 QGMM_API qgmm_status qgmm_per_token_quant(const uint16_t *x_bf16, int64_t rows, int64_t k, int8_t *x1_out,

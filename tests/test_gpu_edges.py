@@ -96,3 +96,11 @@ def test_pair_tail_modes_are_exact(dev, oracle, monkeypatch, tail_mode):
     (padded pair tile, single-CTA launch, M=128 pair tile) give identical results."""
     monkeypatch.setenv("QGMM_PAIR_TAILS", tail_mode)
     _check(dev, oracle, _problem(7, [1, 128, 129, 255, 256, 300, 383, 0, 640], 256, 768), 200)
+
+
+@pytest.mark.parametrize("pair_w4", ["0", "1"])
+def test_int4_full_height_tiles_single_and_pair(dev, oracle, monkeypatch, pair_w4):
+    """int4 weights on 128-row tiles: the single-CTA kernel and the optional CTA-pair
+    kernel (each CTA unpacks its own 128-column half of the packed tile) are exact."""
+    monkeypatch.setenv("QGMM_PAIR_W4", pair_w4)
+    _check(dev, oracle, _problem(8, [1, 129, 255, 256, 300, 0, 513], 256, 768, weight="int4"), 200)
