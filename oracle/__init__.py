@@ -105,8 +105,10 @@ def finalize(x1, x2, group_list, group_list_type: int, *, weight: str = "int8",
              threads: Optional[int] = None):
     """The op's output rows ``dest_rows`` (default all ``output_bs`` rows).
 
-    Returns ``(out64, sabs64, out32)``: double value, double sum of |terms| per
-    element, and the f32 value in the fixed summation order (None if not asked).
+    Returns ``(out64, sabs64, out32)``: double value; per element the magnitude
+    that bounds rounding error, |sharedInput| + sum over contributions of
+    (|acc*scale*pts| + |bias|) * |logit|; and the f32 value in the fixed
+    summation order (None if not asked).
     """
     x1 = _c(x1, np.int8)
     w, wt = _weights(x2, weight)

@@ -259,7 +259,9 @@ static void fin_item(void *p, int64_t it, int64_t *s64, int32_t *acc, int *rc)
             if (o64 || a64) {
                 double y = (((double)acc[j] * (double)sc) * (double)pts + (double)bs) * (double)lg;
                 if (o64) o64[j] += y;
-                if (a64) a64[j] += fabs(y);
+                /* the rounding of (acc*scale*pts + bias)*logit in any f32 order is bounded by a
+                   few ulp of the summands' magnitudes, taken before the bias can cancel */
+                if (a64) a64[j] += (fabs((double)acc[j] * (double)sc * (double)pts) + fabs((double)bs)) * fabs((double)lg);
             }
             if (o32) {
                 float y = (float)acc[j];        /* round to nearest even */
@@ -275,8 +277,9 @@ static void fin_item(void *p, int64_t it, int64_t *s64, int32_t *acc, int *rc)
 
 /*
  * Output rows dest_rows[0..ndest) (dest_rows == NULL: rows 0..ndest-1) of the
- * op.  out64/sabs64 (double, may be NULL): value in double and the sum of the
- * absolute values of the terms added into each element (for error bounds).
+ * op.  out64/sabs64 (double, may be NULL): value in double, and the magnitude
+ * that bounds f32 rounding error in each element: |initial value| plus, per
+ * contribution, (|acc*scale*pts| + |bias|) * |logit|.
  * out32 (may be NULL): the same in f32 in the fixed order.  scale, pts, logit,
  * bias, row_index, shared may be NULL (1, 1, 1, 0, identity, absent).
  */

@@ -2,7 +2,8 @@
 sizes on both the single-CTA and the CTA-pair paths, rows past the groups'
 total, and unusual k / n.  Same bars as test_gpu_parity (bit-exact int32,
 deterministic mode bitwise equal to the oracle's fixed-order f32, atomic mode
-within 2e-5 of the sum of |terms|).
+within 2e-5 of the oracle's error magnitude: |sharedInput| plus, per
+contribution, (|acc*scale*pts| + |bias|) * |logit|).
 """
 from types import SimpleNamespace
 

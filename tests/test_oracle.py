@@ -126,6 +126,19 @@ def test_unit_scales_reduce_to_matmul_plus_index_add(oracle):
     np.testing.assert_array_equal(sabs, _abs_index_add(ri, acc, tokens))
 
 
+def test_error_magnitude_counts_bias_before_cancellation(oracle):
+    """One contribution (3*0.5*2 - 2.5)*4 = 2: the error magnitude is (3 + 2.5)*4 = 22,
+    not |2|, because f32 rounding acts on the parts before the bias cancels them."""
+    x1 = np.array([[1]], np.int8)
+    x2 = np.array([[[3]]], np.int8)
+    o64, sabs, o32 = oracle.finalize(
+        x1, x2, np.array([1], np.int64), 1, scale=np.array([[0.5]], np.float32),
+        pertoken_scale=np.array([2.0], np.float32), logit=np.array([4.0], np.float32),
+        bias=np.array([[-2.5]], np.float32), row_index=np.array([0], np.int64), output_bs=1)
+    assert o64[0, 0] == 2.0 and o32[0, 0] == 2.0
+    assert sabs[0, 0] == 22.0
+
+
 def _abs_index_add(ri, acc, tokens):
     out = np.zeros((tokens, acc.shape[1]), np.float64)
     np.add.at(out, ri, np.abs(acc).astype(np.float64))
