@@ -61,7 +61,9 @@ __device__ __forceinline__ int32_t tiles_of_group(int64_t rows, int sched, int t
 template <bool W4>
 struct GemmCfg {
     static constexpr int STAGES = W4 ? 3 : 4;
-    static constexpr int NUM_WARPS = 10;   // producer, MMA, then 8 epilogue (int8) or 4 epilogue + 4 unpack (W4)
+    // producer, MMA, then 8 epilogue warps (int8) or 4 epilogue + 8 unpack warps (int4:
+    // two unpack warps per SM sub-partition, measured 12% faster than one)
+    static constexpr int NUM_WARPS = W4 ? 14 : 10;
     static constexpr int EPI_WARPS = W4 ? 4 : 8;
     static constexpr int THREADS = NUM_WARPS * 32;
     static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES + (W4 ? P_STAGE_BYTES : 0);
@@ -545,7 +547,7 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            ptx::mbar_init(&full[s], W4 ? 4 : 1);
+            ptx::mbar_init(&full[s], W4 ? 8 : 1);   // W4: the 8 unpack warps
             ptx::mbar_init(&empty[s], 1);
             ptx::mbar_init(&pfull[s], 1);
         }
@@ -724,7 +726,7 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
         }
     } else if constexpr (W4) {
         // ------------------------------------------------ int4 -> int8 unpack into the MN-major B tile
-        const int ut = threadIdx.x - 6 * 32;    // 0..127
+        const int ut = threadIdx.x - 6 * 32;    // 0..255
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -739,8 +741,8 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
                 uint8_t *b = smem_b + stage * B_STAGE_BYTES;
                 const int qc = ut & 7;          // 16-byte packed chunk of the row: columns 32*qc .. 32*qc+31
 #pragma unroll
-                for (int it = 0; it < 8; ++it) {
-                    const int kr = (ut >> 3) + 16 * it;   // k row within the stage
+                for (int it = 0; it < 4; ++it) {
+                    const int kr = (ut >> 3) + 32 * it;   // k row within the stage
                     const uint4 w = *reinterpret_cast<const uint4 *>(p + kr * 128 + qc * 16);
                     uint4 o0, o1;
                     unpack_int4x8(w.x, o0.x, o0.y);
@@ -1077,28 +1079,33 @@ __global__ void __launch_bounds__(PairCfg<W4>::THREADS, 1)
 
 // ---------------------------------------------------------------- K1
 // out[r][:] = f32(shared[r - off][:]) for r in [off, off + bs), else 0.  Also
-// clears the call's status word.  One float4 (four columns) per thread step.
+// clears the call's status word.  A block walks whole rows; a thread step reads
+// 8 bf16 (16 bytes) and writes two float4.  The host launches 2 blocks of 256
+// threads per SM, which leaves room on every SM for a grouped-GEMM CTA that
+// programmatic dependent launch lets start while this kernel still runs.
 __global__ void output_init_kernel(float *__restrict__ out, int64_t output_bs, int32_t n,
                                    const uint16_t *__restrict__ shared, int64_t shared_bs, int64_t shared_off,
                                    uint32_t *status)
 {
     ptx::pdl_launch_dependents();   // the grouped GEMM may start its prologue and mainloop now
     if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
-    const int64_t q_per_row = n / 4;
-    const int64_t total = output_bs * q_per_row;
-    for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total;
-         idx += int64_t(gridDim.x) * blockDim.x) {
-        const int64_t r = idx / q_per_row;
-        const int64_t c4 = idx - r * q_per_row;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (shared && r >= shared_off && r < shared_off + shared_bs) {
-            const uint2 h = __ldg(reinterpret_cast<const uint2 *>(shared + (r - shared_off) * n) + c4);
-            v.x = __uint_as_float(h.x << 16);
-            v.y = __uint_as_float(h.x & 0xFFFF0000u);
-            v.z = __uint_as_float(h.y << 16);
-            v.w = __uint_as_float(h.y & 0xFFFF0000u);
+    const int n8 = n / 8;           // n % 256 == 0
+    for (int64_t r = blockIdx.x; r < output_bs; r += gridDim.x) {
+        float4 *dst = reinterpret_cast<float4 *>(out + r * n);
+        const bool sh = shared != nullptr && r >= shared_off && r < shared_off + shared_bs;
+        const uint4 *src = reinterpret_cast<const uint4 *>(shared + (sh ? (r - shared_off) * n : 0));
+        for (int c = threadIdx.x; c < n8; c += blockDim.x) {
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+            if (sh) {
+                const uint4 h = __ldg(src + c);   // bf16 -> f32 is exact: the bits move up 16 places
+                a = make_float4(__uint_as_float(h.x << 16), __uint_as_float(h.x & 0xFFFF0000u),
+                                __uint_as_float(h.y << 16), __uint_as_float(h.y & 0xFFFF0000u));
+                b = make_float4(__uint_as_float(h.z << 16), __uint_as_float(h.z & 0xFFFF0000u),
+                                __uint_as_float(h.w << 16), __uint_as_float(h.w & 0xFFFF0000u));
+            }
+            dst[2 * c] = a;
+            dst[2 * c + 1] = b;
         }
-        reinterpret_cast<float4 *>(out)[idx] = v;
     }
 }
 

@@ -419,8 +419,7 @@ qgmm_status finalize_impl(const qgmm_problem *p, const int8_t *x1, const void *x
     const uint16_t *shared = p->shared_bs > 0 ? shared_input : nullptr;
 
     if (!p->deterministic) {
-        const int64_t quads = p->output_bs * (p->n / 4);
-        output_init_kernel<<<grid_for(quads, 256, dev->sms, 8), 256, 0, st>>>(
+        output_init_kernel<<<grid_for(p->output_bs, 1, dev->sms, 2), 256, 0, st>>>(
             out, p->output_bs, static_cast<int32_t>(p->n), shared, p->shared_bs, p->shared_offset, status);
         if (cudaGetLastError() != cudaSuccess) return QGMM_ERR_CUDA;
         a.out = out;
