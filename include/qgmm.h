@@ -112,6 +112,18 @@ typedef struct {
 qgmm_status qgmm_finalize_workspace(const qgmm_problem *p, size_t *ws_bytes);
 
 /*
+ * How many kernels one qgmm_finalize call with `p` launches on the current
+ * device (host pointers; the plan depends on the device's SM count and on the
+ * QGMM_PAIR / QGMM_PAIR_W4 / QGMM_PAIR_TAILS environment switches, read now).
+ * Atomic mode: the output init plus the grouped GEMM launches (1, or 2 when
+ * full-height tiles run on CTA pairs and odd tails on a single-CTA launch).
+ * Deterministic mode adds the five bucketing kernels and the final reduce.
+ * The per-token quant prologue is a separate call and is not counted.
+ * Errors: NULL_PTR, SHAPE, DTYPE, UNSUPPORTED, CUDA (no usable device).
+ */
+qgmm_status qgmm_finalize_launches(const qgmm_problem *p, int32_t *launches);
+
+/*
  * Stage 2: run the operation on `cuda_stream`.
  *   x1              int8 [m, k] row-major, required
  *   x2              int8 [e, k, n] or int32 [e, k, n/8], row-major, required

@@ -47,8 +47,9 @@ QGMM_DEV_GROUP_TOTAL_GT_M = 1 << 2
 QGMM_DEV_ROW_INDEX_RANGE = 1 << 3
 QGMM_DEV_TIMEOUT = 1 << 4
 
-EXPORTS = ("qgmm_finalize_workspace", "qgmm_finalize", "qgmm_finalize_profiled", "qgmm_per_token_quant",
-           "qgmm_debug_accum", "qgmm_device_status", "qgmm_finalize_static_scratch", "qgmm_status_string")
+EXPORTS = ("qgmm_finalize_workspace", "qgmm_finalize_launches", "qgmm_finalize", "qgmm_finalize_profiled",
+           "qgmm_per_token_quant", "qgmm_debug_accum", "qgmm_device_status", "qgmm_finalize_static_scratch",
+           "qgmm_status_string")
 
 
 class QgmmProblem(C.Structure):
@@ -81,6 +82,7 @@ def lib():
         L = C.CDLL(LIB_PATH)
         P, I64, U = C.c_void_p, C.c_int64, C.c_size_t
         L.qgmm_finalize_workspace.argtypes = [C.POINTER(QgmmProblem), C.POINTER(C.c_size_t)]
+        L.qgmm_finalize_launches.argtypes = [C.POINTER(QgmmProblem), C.POINTER(C.c_int32)]
         L.qgmm_finalize.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, P, P, P, P, P, P, U, P]
         L.qgmm_finalize_profiled.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, P, P, P, P, P, P, U, P, P, P]
         L.qgmm_per_token_quant.argtypes = [P, I64, I64, P, P, P]
@@ -132,6 +134,13 @@ def _check(rc: int, what: str):
 def finalize_workspace(problem: QgmmProblem) -> int:
     out = C.c_size_t(0)
     _check(lib().qgmm_finalize_workspace(C.byref(problem), C.byref(out)), "qgmm_finalize_workspace")
+    return out.value
+
+
+def finalize_launches(problem: QgmmProblem) -> int:
+    """Number of kernels one ``finalize`` call with ``problem`` launches on the current device."""
+    out = C.c_int32(0)
+    _check(lib().qgmm_finalize_launches(C.byref(problem), C.byref(out)), "qgmm_finalize_launches")
     return out.value
 
 

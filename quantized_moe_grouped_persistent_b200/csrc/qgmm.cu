@@ -281,6 +281,11 @@ qgmm_status launch_pair_t(DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma
 
 // mb: weight map of the main launch; mb_tail: weight map of the single-CTA
 // tail launch (they differ only for int4 weights on CTA pairs).
+int pair_tail_mode() { return env_int("QGMM_PAIR_TAILS", 1); }
+
+// Kernel launches of one grouped GEMM under plan `pl` (launch_gemm below).
+int gemm_launches(const Plan &pl) { return pl.pair && pair_tail_mode() == 1 ? 2 : 1; }
+
 qgmm_status launch_gemm(int epi, DeviceInfo *dev, const qgmm_problem *p, const Plan &pl, const CUtensorMap &ma,
                         const CUtensorMap &mb, const CUtensorMap &mb_tail, const GemmArgs &a, cudaStream_t st)
 {
@@ -297,7 +302,7 @@ qgmm_status launch_gemm(int epi, DeviceInfo *dev, const qgmm_problem *p, const P
         //   2 to an M = 128 pair tile (64 rows per CTA) after the group's other tiles;
         //   0 to a full 256-row pair tile padded with rows it ignores.
         // All three give identical results; 1 measured fastest at large prefill.
-        const int tail_mode = env_int("QGMM_PAIR_TAILS", 1);
+        const int tail_mode = pair_tail_mode();
         const bool tails = tail_mode == 1;
         GemmArgs ap = a;
         ap.sched = tail_mode == 2 ? SCHED_PAIRS_TAIL128 : tails ? SCHED_PAIRS : SCHED_PAIRS_ALL;
@@ -474,6 +479,19 @@ QGMM_API qgmm_status qgmm_finalize_profiled(const qgmm_problem *p, const int8_t 
     return finalize_impl(p, x1, x2, scale, pertoken_scale, group_list, logit, row_index, bias, shared_input, out,
                          workspace, ws_bytes, cuda_stream, static_cast<cudaEvent_t>(gemm_begin_event),
                          static_cast<cudaEvent_t>(gemm_end_event));
+}
+
+QGMM_API qgmm_status qgmm_finalize_launches(const qgmm_problem *p, int32_t *launches)
+{
+    qgmm_status s = check_problem(p);
+    if (s != QGMM_OK) return s;
+    if (!launches) return QGMM_ERR_NULL_PTR;
+    DeviceInfo *dev = nullptr;
+    if ((s = device_info(&dev)) != QGMM_OK) return s;
+    const Plan pl = make_plan(p, dev->sms, p->deterministic ? EPI_STORE_Y : EPI_ATOMIC);
+    // atomic: output init; deterministic: clear, histogram, scan, fill, sort, then the reduce
+    *launches = (p->deterministic ? 6 : 1) + gemm_launches(pl);
+    return QGMM_OK;
 }
 
 QGMM_API qgmm_status qgmm_debug_accum(const qgmm_problem *p, const int8_t *x1, const void *x2,

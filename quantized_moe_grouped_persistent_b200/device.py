@@ -5,6 +5,7 @@ operation itself runs in libqgmm.so's kernels.
 """
 from __future__ import annotations
 
+import copy
 from typing import Optional
 
 import numpy as np
@@ -55,6 +56,17 @@ class DeviceProblem:
         self.shared_offset = p.shared_offset
         self.out = torch.empty((p.output_bs, p.n), dtype=torch.float32, device=dev)
         self._ws = {}
+
+    def io_copy(self) -> "DeviceProblem":
+        """Same problem with its own per-call buffers (activations, scales, routing,
+        sharedInput, output, workspace) and the same resident weights, scale and bias,
+        so that two calls can be in flight at once."""
+        c = copy.copy(self)
+        for name in ("x_bf16", "x1", "pts", "group_list", "logit", "row_index", "shared", "out"):
+            t = getattr(self, name)
+            setattr(c, name, None if t is None else torch.empty_like(t))
+        c._ws = {}
+        return c
 
     def problem(self, deterministic: bool = False):
         return make_problem(self.m, self.k, self.n, self.e, self.output_bs, weight_type=self.weight_type,

@@ -105,3 +105,15 @@ def test_int4_full_height_tiles_single_and_pair(dev, oracle, monkeypatch, pair_w
     kernel (each CTA unpacks its own 128-column half of the packed tile) are exact."""
     monkeypatch.setenv("QGMM_PAIR_W4", pair_w4)
     _check(dev, oracle, _problem(8, [1, 129, 255, 256, 300, 0, 513], 256, 768, weight="int4"), 200)
+
+
+def test_launch_count_query(dev, qgmm, monkeypatch):
+    """qgmm_finalize_launches follows the plan: pair tiles + a tail launch, or one GEMM launch."""
+    p = _problem(9, [300, 0, 40], 256, 512)
+    pair = dev.DeviceProblem(p, expected_m_per_expert=200)     # 128-row tiles: CTA pairs + tail launch
+    assert qgmm.finalize_launches(pair.problem(False)) == 3    # init, pair GEMM, tail GEMM
+    assert qgmm.finalize_launches(pair.problem(True)) == 8     # 5 bucketing kernels, 2 GEMM, reduce
+    monkeypatch.setenv("QGMM_PAIR_TAILS", "2")                 # tails as M=128 pair tiles in one launch
+    assert qgmm.finalize_launches(pair.problem(False)) == 2
+    single = dev.DeviceProblem(p, expected_m_per_expert=1)     # 16-row tiles on single CTAs
+    assert qgmm.finalize_launches(single.problem(False)) == 2
