@@ -779,8 +779,8 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
 // and 128 columns of the expert's weights, the leader issues
 // tcgen05.mma.cta_group::2 (M = 256, N = 256) that reads both CTAs' halves, and
 // each CTA's TMEM receives its own 128 accumulator rows.  Per SM this moves a
-// third fewer operand bytes per MAC than the single-CTA 128 x 256 tile, and the
-// same shared memory holds six stages instead of four.
+// third fewer operand bytes per MAC than the single-CTA 128 x 256 tile, and a
+// 32 KB stage instead of 48 KB lets the same shared memory hold five stages.
 constexpr int PAIR_ROWS = 256;                 // rows per pair tile
 constexpr int PAIR_A_BYTES = 128 * BK;         // this CTA's rows
 constexpr int PAIR_B_BYTES = BK * 128;         // this CTA's columns (one MN-major atom)
