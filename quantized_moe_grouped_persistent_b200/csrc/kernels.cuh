@@ -726,7 +726,15 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
         }
     } else if constexpr (W4) {
         // ------------------------------------------------ int4 -> int8 unpack into the MN-major B tile
+        // Each warp covers 4 k rows x 8 packed 16-byte chunks (qc: columns 32qc ..
+        // 32qc+31).  In every group of 8 lanes, lanes 0-3 take chunks 0-3 (atom 0) of
+        // one row and lanes 4-7 chunks 4-7 (atom 1) of the neighbouring row, so the 8
+        // swizzled int8 stores hit 8 different 16-byte bank groups (the two rows'
+        // chunk parities differ) and the 8 packed loads do too.
         const int ut = threadIdx.x - 6 * 32;    // 0..255
+        const int l = ut & 31;
+        const int qc = l & 7;
+        const int r0 = 4 * (ut >> 5) + ((((l >> 2) ^ (l >> 3)) & 1) | ((l >> 3) & 2));   // row offset 0..3 in the warp
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -739,10 +747,9 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
                 }
                 const uint8_t *p = smem_p + stage * P_STAGE_BYTES;
                 uint8_t *b = smem_b + stage * B_STAGE_BYTES;
-                const int qc = ut & 7;          // 16-byte packed chunk of the row: columns 32*qc .. 32*qc+31
 #pragma unroll
                 for (int it = 0; it < 4; ++it) {
-                    const int kr = (ut >> 3) + 32 * it;   // k row within the stage
+                    const int kr = r0 + 32 * it;          // k row within the stage
                     const uint4 w = *reinterpret_cast<const uint4 *>(p + kr * 128 + qc * 16);
                     uint4 o0, o1;
                     unpack_int4x8(w.x, o0.x, o0.y);
