@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
@@ -139,11 +140,14 @@ Plan make_plan(const qgmm_problem *p, int sms, int epi)
     const int NT = static_cast<int>(p->n / BN);
     int sw = NT;
     if (epi == EPI_ATOMIC) {
-        // One slab of the output (output_bs x slab columns, f32) of at most ~128 MB,
-        // the L2 size: wider slabs let the combine's reductions miss L2, narrower
-        // ones re-read x1 once per slab.
+        // Output slab (output_bs x slab columns, f32): a wider slab lets the combine's
+        // reductions miss L2, a narrower one re-reads x1 once per slab.  The budget
+        // is half of x1's bytes, clamped to [32 MB, 128 MB (about L2)]: large prefill
+        // (x1 268 MB) keeps ~117 MB slabs, W4A8 (x1 67 MB) ~29 MB slabs -- the best
+        // widths measured for each (2.29 vs 2.32-2.56 ms; 0.733 vs 0.754 ms).
         const double per_ntile = double(p->output_bs) * BN * 4.0;
-        const double budget = 128.0 * 1024 * 1024;
+        const double x1_bytes = double(p->m) * double(p->k);
+        const double budget = std::min(128.0 * 1024 * 1024, std::max(32.0 * 1024 * 1024, x1_bytes / 2));
         sw = 1;
         for (int d = 1; d <= NT; ++d)
             if (NT % d == 0 && d * per_ntile <= budget) sw = d;
