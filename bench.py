@@ -38,6 +38,7 @@ KERNEL_SOURCES = ["quantized_moe_grouped_persistent_b200/csrc/kernels.cuh",
 TRAFFIC_SUMMARY = {
     "large_prefill": "profiles/grouped_gemm_large_prefill.md",
     "decode": "profiles/grouped_gemm_decode.md",
+    "w4a8_prologue": "profiles/grouped_gemm_w4a8.md",
 }
 
 
@@ -413,7 +414,12 @@ def main():
     clocks = sampler.stop()
     ms_max, gemm_max = max_over_ranks([ms, gemm_ms], dist, device="cuda")
     value = weak_scaling_value(world, ops, ms_max)
-    launches_per_step = finalize_launches(d.problem(args.deterministic)) + (1 if d.prologue else 0)
+    op_launches = finalize_launches(d.problem(args.deterministic))
+    launches_per_step = op_launches + (1 if d.prologue else 0)
+    # the plan's GEMM launches: CTA-pair tiles plus a single-CTA tail launch, or one single-CTA launch
+    gemm_launches = op_launches - (6 if args.deterministic else 1)
+    gemm_kernel = ("grouped GEMM (grouped_gemm_pair_kernel + tail launch)" if gemm_launches == 2
+                   else "grouped_gemm_kernel")
 
     extras = {}
     if world == 1 and not args.no_extras:
@@ -468,7 +474,7 @@ def main():
                                        "measured_sustained": 100.0 * value / world / int8_peak_sustained},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TOPS",
                          "frac": achieved / int8_peak, "traffic": committed_traffic(args.workload),
-                         "kernel": "grouped GEMM (grouped_gemm_pair_kernel + tail launch)", "kernel_ms": gemm_max,
+                         "kernel": gemm_kernel, "kernel_ms": gemm_max,
                          "frac_of_sustained": achieved / int8_peak_sustained,
                          "peak_source": f"{peaks['source']} bf16 burst x 2 (dense int8 : bf16 nominal ratio), "
                                         f"of measured"},
