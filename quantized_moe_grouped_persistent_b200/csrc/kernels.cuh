@@ -1250,12 +1250,20 @@ __global__ void det_reduce_kernel(float *__restrict__ out, const float *__restri
                 acc.z = __uint_as_float(h.y << 16);
                 acc.w = __uint_as_float(h.y & 0xFFFF0000u);
             }
-            for (int32_t x = a; x < b; ++x) {
-                const float4 v = __ldg(reinterpret_cast<const float4 *>(y + int64_t(list[x]) * n) + c4);
-                acc.x = __fadd_rn(acc.x, v.x);
-                acc.y = __fadd_rn(acc.y, v.y);
-                acc.z = __fadd_rn(acc.z, v.z);
-                acc.w = __fadd_rn(acc.w, v.w);
+            // a bucket holds about topK rows: issue its loads together, then add in order
+            for (int32_t x0 = a; x0 < b; x0 += 8) {
+                float4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (x0 + u < b) v[u] = __ldg(reinterpret_cast<const float4 *>(y + int64_t(list[x0 + u]) * n) + c4);
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (x0 + u < b) {
+                        acc.x = __fadd_rn(acc.x, v[u].x);
+                        acc.y = __fadd_rn(acc.y, v[u].y);
+                        acc.z = __fadd_rn(acc.z, v[u].z);
+                        acc.w = __fadd_rn(acc.w, v[u].w);
+                    }
             }
             reinterpret_cast<float4 *>(out + r * n)[c4] = acc;
         }
