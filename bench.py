@@ -451,6 +451,24 @@ def main():
         }
         del dd
         torch.cuda.empty_cache()
+    if world == 1 and not args.no_extras and args.workload == "large_prefill":
+        # the other prefill-shaped workloads, atomic combine, with their own int8 roofline
+        for name in ("mid_prefill", "w4a8_prologue"):
+            ps = make_problem(name)
+            ds = DeviceProblem(ps)
+            ds.run()
+            torch.cuda.synchronize()
+            sms_, sgemm = time_steps(ds, max(10, args.steps), 3, False)
+            sops = int_ops(ps)
+            extras[name] = {
+                "workload": f"{name}: " + CONFIGS[name].description + "; atomic combine",
+                "value": sops / (sms_ * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": sms_, "gemm_ms": sgemm,
+                "roofline": {"bound": "tensor", "achieved": sops / (sgemm * 1e-3) / 1e12, "peak": int8_peak,
+                             "unit": "TOPS", "frac": sops / (sgemm * 1e-3) / 1e12 / int8_peak,
+                             "traffic": committed_traffic(name), "kernel_ms": sgemm},
+            }
+            del ds
+            torch.cuda.empty_cache()
 
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
