@@ -127,6 +127,7 @@ struct Plan {
     int slab_ntiles;
     int grid;
     bool pair;   // CTA-pair kernel (tcgen05 cta_group::2, 256-row tiles)
+    int tail_mode;   // pair path: where a group's odd last <= 128 rows run (launch_gemm)
 };
 
 Plan make_plan(const qgmm_problem *p, int sms, int epi)
@@ -168,6 +169,21 @@ Plan make_plan(const qgmm_problem *p, int sms, int epi)
     pl.grid = static_cast<int>(max_tiles < sms ? max_tiles : sms);
     if (pl.grid < 1) pl.grid = 1;
     if (pl.pair) pl.grid = static_cast<int>(2 * (max_tiles < sms / 2 ? max_tiles : sms / 2));
+
+    // Tail tiles (at most one per group and n-tile) cost a second launch's fill and
+    // drain in mode 1, and a pair's full weight feed for <= 128 rows in mode 2.  Mode
+    // 2 wins when the tail launch would be short (<= 8 waves of single CTAs) and so is
+    // the pair launch (<= 32 waves of pairs): measured 5-10% faster at m = 4096-16384
+    // over 32 experts, n = 7168; mode 1 is 2-5% faster at 256 experts (~30 tail waves)
+    // and ties or wins once the pair launch is longer.
+    pl.tail_mode = 1;
+    if (pl.pair) {
+        const double tail_waves = double(p->e) * NT / sms;
+        const double pair_waves = double(p->m) / 256.0 * NT / (sms / 2);
+        if (tail_waves <= 8.0 && pair_waves <= 32.0) pl.tail_mode = 2;
+    }
+    const int forced_tails = env_int("QGMM_PAIR_TAILS", -1);
+    if (forced_tails >= 0 && forced_tails <= 2) pl.tail_mode = forced_tails;
     return pl;
 }
 
@@ -283,10 +299,8 @@ qgmm_status launch_pair_t(DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma
     return cudaGetLastError() == cudaSuccess ? QGMM_OK : QGMM_ERR_CUDA;
 }
 
-int pair_tail_mode() { return env_int("QGMM_PAIR_TAILS", 1); }
-
 // Kernel launches of one grouped GEMM under plan `pl` (launch_gemm below).
-int gemm_launches(const Plan &pl) { return pl.pair && pair_tail_mode() == 1 ? 2 : 1; }
+int gemm_launches(const Plan &pl) { return pl.pair && pl.tail_mode == 1 ? 2 : 1; }
 
 // mb: weight map of the main launch; mb_tail: weight map of the single-CTA
 // tail launch (they differ only for int4 weights on CTA pairs).
@@ -301,14 +315,13 @@ qgmm_status launch_gemm(int epi, DeviceInfo *dev, const qgmm_problem *p, const P
                      pl.tile_rows, pl.slab_ntiles, pl.grid);
     if (pl.pair) {
         // Pairs of 128-row half tiles on CTA pairs.  A group's odd last half tile
-        // (its final <= 128 rows) goes, by QGMM_PAIR_TAILS:
-        //   1 (default) to a single-CTA launch right after the pair launch;
+        // (its final <= 128 rows) goes, by pl.tail_mode (make_plan's choice, or
+        // QGMM_PAIR_TAILS):
+        //   1 to a single-CTA launch right after the pair launch;
         //   2 to an M = 128 pair tile (64 rows per CTA) after the group's other tiles;
         //   0 to a full 256-row pair tile padded with rows it ignores.
-        // All three give identical results and measured within 1% of each other at
-        // large prefill (the tail launch re-reads weights from DRAM; the in-kernel
-        // forms spend a full pair-tile's operand feed on <= 128 rows).
-        const int tail_mode = pair_tail_mode();
+        // All three give identical results.
+        const int tail_mode = pl.tail_mode;
         const bool tails = tail_mode == 1;
         GemmArgs ap = a;
         ap.sched = tail_mode == 2 ? SCHED_PAIRS_TAIL128 : tails ? SCHED_PAIRS : SCHED_PAIRS_ALL;

@@ -110,6 +110,7 @@ def test_int4_full_height_tiles_single_and_pair(dev, oracle, monkeypatch, pair_w
 def test_launch_count_query(dev, qgmm, monkeypatch):
     """qgmm_finalize_launches follows the plan: pair tiles + a tail launch, or one GEMM launch."""
     p = _problem(9, [300, 0, 40], 256, 512)
+    monkeypatch.setenv("QGMM_PAIR_TAILS", "1")
     pair = dev.DeviceProblem(p, expected_m_per_expert=200)     # 128-row tiles: CTA pairs + tail launch
     assert qgmm.finalize_launches(pair.problem(False)) == 3    # init, pair GEMM, tail GEMM
     assert qgmm.finalize_launches(pair.problem(True)) == 8     # 5 bucketing kernels, 2 GEMM, reduce
@@ -117,3 +118,17 @@ def test_launch_count_query(dev, qgmm, monkeypatch):
     assert qgmm.finalize_launches(pair.problem(False)) == 2
     single = dev.DeviceProblem(p, expected_m_per_expert=1)     # 16-row tiles on single CTAs
     assert qgmm.finalize_launches(single.problem(False)) == 2
+
+
+def test_default_tail_mode_follows_wave_counts(qgmm, monkeypatch):
+    """Without QGMM_PAIR_TAILS the planner runs tails as M=128 pair tiles when both
+    launches would be short (32 experts, m = 8192, n = 7168: one GEMM launch), and as
+    a single-CTA tail launch once the pair launch is long (m = 32768) or the tails
+    are many (256 experts)."""
+    if not torch.cuda.is_available() or torch.cuda.get_device_properties(0).multi_processor_count != 148:
+        pytest.skip("wave counts are for a 148-SM B200")
+    monkeypatch.delenv("QGMM_PAIR_TAILS", raising=False)
+    launches = lambda m, e: qgmm.finalize_launches(qgmm.make_problem(m, 2048, 7168, e, m // 8))
+    assert launches(8192, 32) == 2          # output init + pair GEMM
+    assert launches(32768, 32) == 3         # output init + pair GEMM + tail GEMM
+    assert launches(131072, 256) == 3

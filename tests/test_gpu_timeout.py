@@ -5,8 +5,8 @@ grouped GEMM's producer issue no copy.  The MMA warp's wait for operands then
 runs out after its one-second bound; the kernel must set QGMM_DEV_TIMEOUT in
 the status word, release its tensor memory and return, leaving the context
 usable: the next ordinary call on the same operands matches the oracle.
-Both the single-CTA kernel and the CTA-pair kernel (plus its tail launch) are
-covered.
+The single-CTA kernel and the CTA-pair kernel are covered, the latter with its
+tail launch and with tails as M=128 pair tiles.
 """
 import time
 
@@ -26,12 +26,13 @@ def dev(qgmm):
     return device
 
 
-@pytest.mark.parametrize("case", ["single_cta", "cta_pair"])
+@pytest.mark.parametrize("case", ["single_cta", "cta_pair_tail_launch", "cta_pair_tail128"])
 def test_bounded_wait_runs_out_and_context_survives(dev, qgmm, oracle, problem_cache, monkeypatch, case):
     if case == "single_cta":
         p, hint = problem_cache("tiny"), 0                                        # 16-row tiles, one CTA
     else:
         p, hint = problem_cache("mid_prefill", tokens=96, e=8, k=512, n=768), 200   # pair tiles + tails
+        monkeypatch.setenv("QGMM_PAIR_TAILS", "1" if case == "cta_pair_tail_launch" else "2")
     d = dev.DeviceProblem(p, expected_m_per_expert=hint)
     monkeypatch.setenv("QGMM_TEST_STALL_PRODUCER", "1")
     t0 = time.time()
