@@ -217,15 +217,18 @@ __device__ __forceinline__ int64_t load_row_index(const void *ri, int type, int6
     return static_cast<int64_t>(__ldg(static_cast<const int *>(ri) + i));
 }
 
-// int4 (two's complement, lowest nibble = lowest column) -> int8, 8 values per word.
+// int4 (two's complement, lowest nibble = lowest column) -> int8 holding 16 times
+// the value, 8 values per word.  Each nibble moves to the high half of its byte,
+// and that byte read as int8 is the nibble's two's-complement value times 16, with
+// no sign fill.  The MMA then accumulates 16 * acc; the epilogue shifts it back
+// (W4_ACC_SHIFT), exactly, since |16 * acc| <= 16 * 65536 * 128 * 8 = 2^30 for k <= 65536.
+constexpr int W4_ACC_SHIFT = 4;
 __device__ __forceinline__ void unpack_int4x8(uint32_t w, uint32_t &lo_out, uint32_t &hi_out)
 {
-    uint32_t lo = w & 0x0F0F0F0Fu;          // nibbles 0, 2, 4, 6
-    uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;   // nibbles 1, 3, 5, 7
-    lo |= (lo & 0x08080808u) * 30u;         // sign bit 8 -> 0xF0 fill; no carry between bytes
-    hi |= (hi & 0x08080808u) * 30u;
-    lo_out = __byte_perm(lo, hi, 0x5140);   // columns 0..3
-    hi_out = __byte_perm(lo, hi, 0x7362);   // columns 4..7
+    const uint32_t ev = (w << 4) & 0xF0F0F0F0u;   // nibbles 0, 2, 4, 6
+    const uint32_t od = w & 0xF0F0F0F0u;          // nibbles 1, 3, 5, 7
+    lo_out = __byte_perm(ev, od, 0x5140);         // columns 0..3
+    hi_out = __byte_perm(ev, od, 0x7362);         // columns 4..7
 }
 
 // ---------------------------------------------------------------- K2 epilogue helpers
@@ -233,20 +236,21 @@ constexpr int NCHUNK = BN / 32;   // 32-column chunks per accumulator
 
 // Thread = accumulator row: write its 32 values of one chunk into the warp's
 // staging rows (f32 of the int32 value, or its raw bits for the debug output).
-template <int EPI>
+// SHIFT undoes the int4 path's x16 operand scale (arithmetic shift, exact).
+template <int EPI, int SHIFT>
 __device__ __forceinline__ void epi_stage_chunk(float *stage, int lane, const uint32_t (&r)[32])
 {
     float *srow = stage + lane * EPI_LD;
 #pragma unroll
     for (int v = 0; v < 8; ++v) {
+        int a[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) a[u] = static_cast<int>(r[4 * v + u]) >> SHIFT;
         float4 f;
         if constexpr (EPI == EPI_RAW_ACC) {
-            f = make_float4(__int_as_float(r[4 * v]), __int_as_float(r[4 * v + 1]), __int_as_float(r[4 * v + 2]),
-                            __int_as_float(r[4 * v + 3]));
+            f = make_float4(__int_as_float(a[0]), __int_as_float(a[1]), __int_as_float(a[2]), __int_as_float(a[3]));
         } else {
-            f = make_float4(__int2float_rn(static_cast<int>(r[4 * v])), __int2float_rn(static_cast<int>(r[4 * v + 1])),
-                            __int2float_rn(static_cast<int>(r[4 * v + 2])),
-                            __int2float_rn(static_cast<int>(r[4 * v + 3])));
+            f = make_float4(__int2float_rn(a[0]), __int2float_rn(a[1]), __int2float_rn(a[2]), __int2float_rn(a[3]));
         }
         *reinterpret_cast<float4 *>(srow + 4 * v) = f;
     }
@@ -313,8 +317,9 @@ __device__ __forceinline__ EpiSmem epi_smem(float *epi_stage, float *row_pts, fl
 // in the op's order ((f32(acc) * scale) * pts + bias) * logit.  Per-row data
 // and this lane's scale/bias columns are fetched before waiting for the
 // accumulator, and TMEM chunk k+1 is loaded while chunk k is written out.
-// Returns false if the wait for the accumulator ran out.
-template <int EPI, int NCH>
+// SHIFT: W4_ACC_SHIFT for int4 weights, else 0.  Returns false if the wait for
+// the accumulator ran out.
+template <int EPI, int NCH, int SHIFT>
 __device__ __forceinline__ bool epilogue_tile(const GemmArgs &args, const TileCoord &c, int64_t row_base,
                                               int rows_here, int row_off, uint32_t tmem_acc, int q, int tmem_col,
                                               int glob_col, int lane, uint64_t *tfull_bar, uint32_t use,
@@ -371,13 +376,13 @@ __device__ __forceinline__ bool epilogue_tile(const GemmArgs &args, const TileCo
 #pragma unroll
         for (int pc = 0; pc < NCH; pc += 2) {
             ptx::tmem_ld_wait(ra);
-            epi_stage_chunk<EPI>(sm.stage, lane, ra);
+            epi_stage_chunk<EPI, SHIFT>(sm.stage, lane, ra);
             ptx::tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>((pc + 1) * 32), rb);
             __syncwarp();
             epi_write_chunk<EPI>(args, sm.stage, sm.rp, sm.rl, sm.rd, sub, col4, n, n0 + pc * 32, sc[pc], bs[pc]);
             __syncwarp();
             ptx::tmem_ld_wait(rb);
-            epi_stage_chunk<EPI>(sm.stage, lane, rb);
+            epi_stage_chunk<EPI, SHIFT>(sm.stage, lane, rb);
             if (pc + 2 < NCH) ptx::tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>((pc + 2) * 32), ra);
             __syncwarp();
             epi_write_chunk<EPI>(args, sm.stage, sm.rp, sm.rl, sm.rd, sub, col4, n, n0 + (pc + 1) * 32, sc[pc + 1],
@@ -716,7 +721,7 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
             const TileCoord c = tile_coord(t, MT, SW, off, cum, e, tile_rows, args.sched);
             const int buf = lt & 1;
             const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
-            if (!epilogue_tile<EPI, NCHUNK>(args, c, c.row0, tile_rows, q * 32,
+            if (!epilogue_tile<EPI, NCHUNK, W4 ? W4_ACC_SHIFT : 0>(args, c, c.row0, tile_rows, q * 32,
                                             tmem_base + static_cast<uint32_t>(buf * BN), q, 0, 0, lane, &tfull[buf],
                                             use, abort_flag, sm)) {
                 fail();
@@ -1004,6 +1009,7 @@ __global__ void __launch_bounds__(PairCfg<W4>::THREADS, 1)
         ptx::pdl_wait_primary();   // the output (and status word) are initialised by the previous kernel
         if (warp == 2 && lane == 0 && blockIdx.x == 0 && *group_flags) atomicOr(args.status, *group_flags);
         const int q = warp & 3;   // TMEM lane quarter of this warp; it covers all 256 columns
+        constexpr int SHIFT = W4 ? W4_ACC_SHIFT : 0;
         const EpiSmem sm = epi_smem(epi_stage, row_pts, row_lg, row_dst, warp - 2);
         uint32_t tempty_leader[2];
         tempty_leader[0] = ptx::map_to_rank(&tempty[0], 0);
@@ -1020,11 +1026,11 @@ __global__ void __launch_bounds__(PairCfg<W4>::THREADS, 1)
             if (c.tail) {
                 // M=128 pair tile: this CTA's 64 rows; TMEM lanes 0-63 hold columns 0-127,
                 // lanes 64-127 hold columns 128-255, in the buffer's first 128 columns.
-                ok = epilogue_tile<EPI, 4>(args, c, base_tail, 64, 32 * (q & 1), acc, q, 0, (q >> 1) * 128, lane,
-                                           &tfull[buf], use, abort_flag, sm);
+                ok = epilogue_tile<EPI, 4, SHIFT>(args, c, base_tail, 64, 32 * (q & 1), acc, q, 0, (q >> 1) * 128,
+                                                  lane, &tfull[buf], use, abort_flag, sm);
             } else {
-                ok = epilogue_tile<EPI, NCHUNK>(args, c, base_full, 128, q * 32, acc, q, 0, 0, lane, &tfull[buf], use,
-                                                abort_flag, sm);
+                ok = epilogue_tile<EPI, NCHUNK, SHIFT>(args, c, base_full, 128, q * 32, acc, q, 0, 0, lane,
+                                                       &tfull[buf], use, abort_flag, sm);
             }
             if (!ok) {
                 fail();
