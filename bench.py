@@ -294,6 +294,15 @@ def time_e2e(d, p, steps, warmup, deterministic):
     return t0.elapsed_time(t1) / steps, h2d, d2h
 
 
+def line_unit(workload, p):
+    """The JSON line's unit, and the factor taking int8 TOPS of this workload to it:
+    decode is HBM-bound and reports algorithmic GB/s (a sample that does a fraction
+    of the ops is credited the same fraction of the workload's algorithmic bytes)."""
+    if workload == "decode":
+        return "GB/s", 1e3 * algorithmic_bytes(p) / int_ops(p)
+    return "TOPS", 1.0
+
+
 # ----------------------------------------------------------------------------- CPU oracle timing
 def oracle_sample_time(p, target_s, seed):
     """Time the oracle on a seeded sample of output rows sized to about target_s seconds."""
@@ -347,15 +356,16 @@ def reference_arm(args, p, spec_desc):
         oracle.problem_finalize(p, dest_rows=rows, want32=False, threads=threads, **kw)
         total_t += time.perf_counter() - t0
         total_ops += 2.0 * float(counts[rows].sum()) * p.k * p.n
-    value = total_ops / total_t / 1e12
+    unit, factor = line_unit(args.workload, p)
+    value = factor * total_ops / total_t / 1e12
     sample = f"{nrows} of {p.output_bs} output rows per step (every contributing source row in full), {args.steps} steps"
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
         "config": {"workload": spec_desc, "mode": "deterministic order (oracle)"},
-        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": threads, "kind": "oracle", "sample": sample},
-        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
@@ -413,7 +423,16 @@ def main():
     ms, gemm_ms = time_steps(d, args.steps, args.warmup, args.deterministic, dist)
     clocks = sampler.stop()
     ms_max, gemm_max = max_over_ranks([ms, gemm_ms], dist, device="cuda")
-    value = weak_scaling_value(world, ops, ms_max)
+    # decode is HBM-bound: its line reports algorithmic GB/s against the measured copy
+    # bandwidth; the prefill-shaped workloads report int8 TOPS against the tensor peak
+    unit, factor = line_unit(args.workload, p)
+    hbm_line = unit == "GB/s"
+    work = factor * ops / 1e12
+
+    def rate(step_ms):
+        return work / (step_ms * 1e-3)
+
+    value = world * rate(ms_max)
     op_launches = finalize_launches(d.problem(args.deterministic))
     launches_per_step = op_launches + (1 if d.prologue else 0)
     # the plan's GEMM launches: CTA-pair tiles plus a single-CTA tail launch, or one single-CTA launch
@@ -424,12 +443,11 @@ def main():
     extras = {}
     if world == 1 and not args.no_extras:
         e2e_ms, h2d, d2h = time_e2e(d, p, max(4, args.steps // 2), 2, args.deterministic)
-        extras["e2e"] = {"value": ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS", "h2d_bytes_per_step": h2d,
+        extras["e2e"] = {"value": rate(e2e_ms), "unit": unit, "h2d_bytes_per_step": h2d,
                          "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
         if not args.deterministic:
             dms, dgemm = time_steps(d, max(3, args.steps // 2), 2, True)
-            extras["deterministic"] = {"ms_per_step": dms, "value": ops / (dms * 1e-3) / 1e12, "unit": "TOPS",
-                                       "gemm_ms": dgemm}
+            extras["deterministic"] = {"ms_per_step": dms, "value": rate(dms), "unit": unit, "gemm_ms": dgemm}
     del d
     torch.cuda.empty_cache()
     if world == 1 and not args.no_extras and args.workload != "decode":
@@ -473,29 +491,38 @@ def main():
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         t, sops, nr, threads = oracle_sample_time(p, args.cpu_seconds, 4242)
-        cpu = {"value": sops / t / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
+        cpu = {"value": factor * sops / t / 1e12, "unit": unit, "cores": threads, "kind": "oracle",
                "sample": f"{nr} of {p.output_bs} output rows of the same workload (every contributing source "
                          f"row in full, double-precision dequant/combine), {t:.1f} s"}
 
     if rank == 0:
-        achieved = ops / (gemm_max * 1e-3) / 1e12
+        achieved = rate(gemm_max)
+        if hbm_line:
+            rates = {"pct_of_nominal_8tbs": 100.0 * value / world / NOMINAL_HBM_GBS}
+            roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": achieved / peaks["hbm_gbs"], "traffic": committed_traffic(args.workload),
+                        "kernel": gemm_kernel, "kernel_ms": gemm_max, "algorithmic_bytes": algorithmic_bytes(p),
+                        "peak_source": peaks["source"] + " copy bandwidth"}
+        else:
+            rates = {"pct_of_dense_int8_peak": {"nominal_4500": 100.0 * value / world / NOMINAL_INT8_TOPS,
+                                                "measured_burst": 100.0 * value / world / int8_peak,
+                                                "measured_sustained": 100.0 * value / world / int8_peak_sustained}}
+            roofline = {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TOPS",
+                        "frac": achieved / int8_peak, "traffic": committed_traffic(args.workload),
+                        "kernel": gemm_kernel, "kernel_ms": gemm_max,
+                        "frac_of_sustained": achieved / int8_peak_sustained,
+                        "peak_source": f"{peaks['source']} bf16 burst x 2 (dense int8 : bf16 nominal ratio), "
+                                       f"of measured"}
         line = {
-            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "config": {"workload": spec_desc, "tokens": p.tokens, "topk": p.topk, "m": p.m, "e": p.e, "k": p.k,
                        "n": p.n, "output_bs": p.output_bs, "mode": mode,
                        "l2": "inputs larger than L2 (x2 %.2f GB per rank), no flush" % (p.x2.nbytes / 1e9),
                        "parallelism": f"dp{world} (independent batch per GPU)"},
-            "pct_of_dense_int8_peak": {"nominal_4500": 100.0 * value / world / NOMINAL_INT8_TOPS,
-                                       "measured_burst": 100.0 * value / world / int8_peak,
-                                       "measured_sustained": 100.0 * value / world / int8_peak_sustained},
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TOPS",
-                         "frac": achieved / int8_peak, "traffic": committed_traffic(args.workload),
-                         "kernel": gemm_kernel, "kernel_ms": gemm_max,
-                         "frac_of_sustained": achieved / int8_peak_sustained,
-                         "peak_source": f"{peaks['source']} bf16 burst x 2 (dense int8 : bf16 nominal ratio), "
-                                        f"of measured"},
+            **rates,
+            "roofline": roofline,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
             "device_status": flags,

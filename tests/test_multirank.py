@@ -66,3 +66,15 @@ def test_weak_scaling_value_and_seeds():
     assert bench.rank_seed(4, 0) is None
     assert bench.rank_seed(4, 1) != bench.rank_seed(4, 2)
     assert bench.max_over_ranks([3.0, 1.5]) == [3.0, 1.5]  # single process: unchanged
+
+
+def test_line_unit_decode_is_bytes_prefill_is_tops():
+    """Decode lines report algorithmic GB/s: the factor takes the workload's int8
+    ops to its algorithmic bytes; prefill-shaped lines stay in TOPS."""
+    import bench
+    from synth import make_problem
+    p = make_problem("decode", tokens=4, e=8, k=128, n=256)
+    unit, factor = bench.line_unit("decode", p)
+    assert unit == "GB/s"
+    assert factor * bench.int_ops(p) / 1e12 == pytest.approx(bench.algorithmic_bytes(p) / 1e9)
+    assert bench.line_unit("mid_prefill", make_problem("mid_prefill", tokens=8, e=4, k=128, n=256)) == ("TOPS", 1.0)
