@@ -52,7 +52,7 @@ typedef enum {
     QGMM_OK = 0,
     QGMM_ERR_NULL_PTR = 1,            /* a required pointer is NULL                          */
     QGMM_ERR_SHAPE = 2,               /* a size is out of range (limits below)                */
-    QGMM_ERR_DTYPE = 3,               /* an unknown weight / index / group-list type code     */
+    QGMM_ERR_DTYPE = 3,               /* an unknown weight / index / group-list / scale type   */
     QGMM_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes below qgmm_finalize_workspace's answer      */
     QGMM_ERR_UNSUPPORTED = 5,         /* the device is not sm_100 or a feature is not built   */
     QGMM_ERR_CUDA = 6,                /* a CUDA runtime / driver call failed                  */
@@ -64,6 +64,7 @@ typedef enum {
 enum { QGMM_W_INT8 = 0, QGMM_W_INT4_PACKED_INT32 = 1 };   /* x2: (e,k,n) int8 | (e,k,n/8) int32 */
 enum { QGMM_IDX_INT64 = 0, QGMM_IDX_INT32 = 1 };          /* row_index element type             */
 enum { QGMM_GROUP_CUMSUM = 0, QGMM_GROUP_COUNTS = 1 };    /* group_list meaning                 */
+enum { QGMM_SCALE_F32 = 0, QGMM_SCALE_BF16 = 1 };         /* scale element type                 */
 
 /* Device-side status bits (qgmm_device_status). */
 #define QGMM_DEV_GROUP_NEGATIVE     (1u << 0)  /* a type-1 count (or type-0 end) below zero    */
@@ -93,6 +94,10 @@ enum { QGMM_GROUP_CUMSUM = 0, QGMM_GROUP_COUNTS = 1 };    /* group_list meaning 
  *   expected_m_per_expert   tiling hint, rows one expert is expected to get;
  *                   0 = use m / e.  Changes only the tile shape, never the
  *                   result.  (Page 1: tuningConfigOptional[0].)
+ *   scale_type      QGMM_SCALE_F32 (0) | QGMM_SCALE_BF16 (1): element type of
+ *                   `scale` (page 1: scaleOptional is FLOAT or BF16 on A2/A3).
+ *                   A bf16 scale is widened to f32, which is exact, and then
+ *                   enters the same f32 dequant.
  */
 typedef struct {
     int64_t m, k, n, e, output_bs;
@@ -100,6 +105,7 @@ typedef struct {
     int64_t shared_bs, shared_offset;
     int32_t deterministic;
     int64_t expected_m_per_expert;
+    int32_t scale_type;
 } qgmm_problem;
 
 /*
@@ -127,7 +133,7 @@ qgmm_status qgmm_finalize_launches(const qgmm_problem *p, int32_t *launches);
  * Stage 2: run the operation on `cuda_stream`.
  *   x1              int8 [m, k] row-major, required
  *   x2              int8 [e, k, n] or int32 [e, k, n/8], row-major, required
- *   scale           f32 [e, n] (page 1's (e, 1, n)); NULL = all ones
+ *   scale           f32 or bf16 bits [e, n] (page 1's (e, 1, n)), by scale_type; NULL = all ones
  *   pertoken_scale  f32 [m]; NULL = all ones
  *   group_list      int64 [e], required
  *   logit           f32 [m]; NULL = all ones
@@ -136,12 +142,12 @@ qgmm_status qgmm_finalize_launches(const qgmm_problem *p, int32_t *launches);
  *   shared_input    bf16 bits [shared_bs, n]; required iff shared_bs > 0
  *   out             f32 [output_bs, n], fully overwritten (no need to clear it)
  *   workspace       device memory of ws_bytes bytes, 256-byte aligned
- * x1, x2, out and shared_input must be 16-byte aligned.  Rows at or past the
- * groups' total are ignored.
+ * x1, x2, out, shared_input, scale and bias must be 16-byte aligned.  Rows at
+ * or past the groups' total are ignored.
  * Errors: NULL_PTR, SHAPE, DTYPE, ALIGNMENT, WORKSPACE_TOO_SMALL, UNSUPPORTED, CUDA.
  */
 qgmm_status qgmm_finalize(const qgmm_problem *p, const int8_t *x1, const void *x2,
-                          const float *scale, const float *pertoken_scale,
+                          const void *scale, const float *pertoken_scale,
                           const int64_t *group_list, const float *logit, const void *row_index,
                           const float *bias, const uint16_t *shared_input, float *out,
                           void *workspace, size_t ws_bytes, void *cuda_stream);
@@ -154,7 +160,7 @@ qgmm_status qgmm_finalize(const qgmm_problem *p, const int8_t *x1, const void *x
  * either event is NULL.
  */
 qgmm_status qgmm_finalize_profiled(const qgmm_problem *p, const int8_t *x1, const void *x2,
-                                   const float *scale, const float *pertoken_scale,
+                                   const void *scale, const float *pertoken_scale,
                                    const int64_t *group_list, const float *logit, const void *row_index,
                                    const float *bias, const uint16_t *shared_input, float *out,
                                    void *workspace, size_t ws_bytes, void *cuda_stream,
@@ -195,7 +201,7 @@ qgmm_status qgmm_finalize_profiled(const qgmm_problem *p, const int8_t *x1, cons
  */
 #define QGMM_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
 qgmm_status qgmm_finalize_static_scratch(const qgmm_problem *p, const int8_t *x1, const void *x2,
-                                         const float *scale, const float *pertoken_scale,
+                                         const void *scale, const float *pertoken_scale,
                                          const int64_t *group_list, const float *logit,
                                          const void *row_index, const float *bias,
                                          const uint16_t *shared_input, float *out, void *cuda_stream);

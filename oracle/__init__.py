@@ -47,7 +47,8 @@ def lib():
         L.qo_finalize.argtypes = [P, P, I32, I64, I64, I64, I64, P, I32, P, P, P, P, P, I32,
                                   P, I64, I64, I64, P, I64, P, P, P, I32]
         L.qo_per_token_quant.argtypes = [P, I64, I64, P, P]
-        for f in (L.qo_group_offsets, L.qo_accum, L.qo_finalize, L.qo_per_token_quant):
+        L.qo_bf16_to_f32.argtypes = [P, I64, P]
+        for f in (L.qo_group_offsets, L.qo_accum, L.qo_finalize, L.qo_per_token_quant, L.qo_bf16_to_f32):
             f.restype = C.c_int
         _lib = L
     return _lib
@@ -105,11 +106,15 @@ def finalize(x1, x2, group_list, group_list_type: int, *, weight: str = "int8",
              threads: Optional[int] = None):
     """The op's output rows ``dest_rows`` (default all ``output_bs`` rows).
 
+    ``scale`` is f32, or uint16 holding bf16 bits (widened exactly by the C oracle).
+
     Returns ``(out64, sabs64, out32)``: double value; per element the magnitude
     that bounds rounding error, |sharedInput| + sum over contributions of
     (|acc*scale*pts| + |bias|) * |logit|; and the f32 value in the fixed
     summation order (None if not asked).
     """
+    if scale is not None and scale.dtype == np.uint16:
+        scale = bf16_to_f32(scale)
     x1 = _c(x1, np.int8)
     w, wt = _weights(x2, weight)
     m, k = x1.shape
@@ -140,6 +145,16 @@ def finalize(x1, x2, group_list, group_list_type: int, *, weight: str = "int8",
     if rc:
         raise OracleError(rc, "finalize")
     return out64, sabs, out32
+
+
+def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    """bf16 bits (uint16, any shape) -> f32 values, exactly."""
+    b = _c(bits, np.uint16)
+    out = np.zeros(b.shape, np.float32)
+    rc = lib().qo_bf16_to_f32(_ptr(b), b.size, _ptr(out))
+    if rc:
+        raise OracleError(rc, "bf16_to_f32")
+    return out
 
 
 def per_token_quant(x_bf16: np.ndarray):

@@ -28,7 +28,10 @@
  *  - int4: the lowest nibble of each int32 word is the lowest n index, two's
  *    complement (values -8..7);
  *  - per-token quant: a = max |x|, pts = a/127, inv = 127/a (0 for a zero row),
- *    q = round-half-even(x * inv) clamped to [-127, 127].
+ *    q = round-half-even(x * inv) clamped to [-127, 127];
+ *  - a BF16 scale (page 1, parameter notes: scaleOptional is FLOAT or BF16 on
+ *    A2/A3) is widened to f32, which is exact, and then enters the same f32
+ *    dequant as a FLOAT scale (qo_bf16_to_f32).
  *
  * Precision: integer accumulation is exact (int64, checked to fit int32).
  * Two float forms of the dequant+combine are provided:
@@ -304,6 +307,14 @@ int qo_finalize(const int8_t *x1, const void *x2, int weight_type, int64_t m, in
     }
     free(off);
     return rc;
+}
+
+/* ---- bf16 -> f32 widening (a BF16 scale; exact) ------------------------- */
+int qo_bf16_to_f32(const uint16_t *in, int64_t count, float *out)
+{
+    if ((!in || !out) && count > 0) return QO_ERR_ARG;
+    for (int64_t i = 0; i < count; ++i) out[i] = bf16_to_f32(in[i]);
+    return QO_OK;
 }
 
 /* ---- per-token quantisation (f32; the decision is an integer) ----------- */

@@ -40,6 +40,8 @@ QGMM_IDX_INT64 = 0
 QGMM_IDX_INT32 = 1
 QGMM_GROUP_CUMSUM = 0
 QGMM_GROUP_COUNTS = 1
+QGMM_SCALE_F32 = 0
+QGMM_SCALE_BF16 = 1
 
 QGMM_DEV_GROUP_NEGATIVE = 1 << 0
 QGMM_DEV_GROUP_NOT_MONOTONE = 1 << 1
@@ -60,6 +62,7 @@ class QgmmProblem(C.Structure):
         ("shared_bs", C.c_int64), ("shared_offset", C.c_int64),
         ("deterministic", C.c_int32),
         ("expected_m_per_expert", C.c_int64),
+        ("scale_type", C.c_int32),
     ]
 
 
@@ -104,9 +107,9 @@ def status_string(code: int) -> str:
 def make_problem(m: int, k: int, n: int, e: int, output_bs: int, *, weight_type: int = QGMM_W_INT8,
                  group_list_type: int = QGMM_GROUP_CUMSUM, row_index_type: int = QGMM_IDX_INT64,
                  shared_bs: int = 0, shared_offset: int = 0, deterministic: bool = False,
-                 expected_m_per_expert: int = 0) -> QgmmProblem:
+                 expected_m_per_expert: int = 0, scale_type: int = QGMM_SCALE_F32) -> QgmmProblem:
     return QgmmProblem(m, k, n, e, output_bs, weight_type, group_list_type, row_index_type, shared_bs,
-                       shared_offset, int(bool(deterministic)), expected_m_per_expert)
+                       shared_offset, int(bool(deterministic)), expected_m_per_expert, scale_type)
 
 
 def _ptr(t) -> Optional[int]:

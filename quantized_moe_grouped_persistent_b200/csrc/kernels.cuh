@@ -89,7 +89,9 @@ struct GemmArgs {
     int32_t sched;         // which m-tiles this launch covers (SCHED_*)
     int32_t stall_producer;  // test hook: the producer issues no copy, so the MMA wait must run out
     int32_t slab_ntiles;   // n-tiles per slab; divides n / BN
-    const float *scale, *pts, *logit, *bias;
+    const void *scale;     // f32 [e, n], or bf16 bits when scale_bf16
+    int32_t scale_bf16;
+    const float *pts, *logit, *bias;
     const void *row_index;
     int32_t row_index_type;
     int64_t output_bs;
@@ -232,6 +234,27 @@ __device__ __forceinline__ void unpack_int4x8(uint32_t w, uint32_t &lo_out, uint
 }
 
 // ---------------------------------------------------------------- K2 epilogue helpers
+// scale[idx .. idx+3] (idx % 4 == 0) or [idx, idx+1] (idx even) as f32.  A bf16
+// scale is widened exactly: its 16 bits are the upper half of the f32.
+__device__ __forceinline__ float4 load_scale4(const GemmArgs &a, int64_t idx)
+{
+    if (a.scale_bf16) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(a.scale) + idx));
+        return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u), __uint_as_float(v.y << 16),
+                           __uint_as_float(v.y & 0xFFFF0000u));
+    }
+    return __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(a.scale) + idx));
+}
+
+__device__ __forceinline__ float2 load_scale2(const GemmArgs &a, int64_t idx)
+{
+    if (a.scale_bf16) {
+        const uint32_t v = __ldg(reinterpret_cast<const unsigned int *>(static_cast<const uint16_t *>(a.scale) + idx));
+        return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+    }
+    return __ldg(reinterpret_cast<const float2 *>(static_cast<const float *>(a.scale) + idx));
+}
+
 constexpr int NCHUNK = BN / 32;   // 32-column chunks per accumulator
 
 // Thread = accumulator row: write its 32 values of one chunk into the warp's
@@ -358,7 +381,7 @@ __device__ __forceinline__ bool epilogue_tile(const GemmArgs &args, const TileCo
         const int64_t base = static_cast<int64_t>(c.g) * n + static_cast<int64_t>(c.nt) * BN + col_begin + col4;
         if (args.scale) {
 #pragma unroll
-            for (int k = 0; k < NCH; ++k) sc[k] = __ldg(reinterpret_cast<const float4 *>(args.scale + base + k * 32));
+            for (int k = 0; k < NCH; ++k) sc[k] = load_scale4(args, base + k * 32);
         }
         if (args.bias) {
 #pragma unroll
@@ -486,7 +509,7 @@ __device__ __forceinline__ bool epilogue_tile_direct(const GemmArgs &args, const
             for (int ch = 0; ch < EPI_CHUNKS; ++ch)
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
-                    sc[ch][j] = __ldg(reinterpret_cast<const float2 *>(args.scale + base + 64 * ch + 8 * j));
+                    sc[ch][j] = load_scale2(args, base + 64 * ch + 8 * j);
         }
         if (args.bias) {
 #pragma unroll

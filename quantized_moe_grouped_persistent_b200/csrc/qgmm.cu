@@ -83,6 +83,7 @@ qgmm_status check_problem(const qgmm_problem *p)
     if (p->weight_type != QGMM_W_INT8 && p->weight_type != QGMM_W_INT4_PACKED_INT32) return QGMM_ERR_DTYPE;
     if (p->group_list_type != QGMM_GROUP_CUMSUM && p->group_list_type != QGMM_GROUP_COUNTS) return QGMM_ERR_DTYPE;
     if (p->row_index_type != QGMM_IDX_INT64 && p->row_index_type != QGMM_IDX_INT32) return QGMM_ERR_DTYPE;
+    if (p->scale_type != QGMM_SCALE_F32 && p->scale_type != QGMM_SCALE_BF16) return QGMM_ERR_DTYPE;
     if (p->m < 1 || p->m > kMaxM) return QGMM_ERR_SHAPE;
     if (p->k < BK || p->k > 65536 || p->k % BK) return QGMM_ERR_SHAPE;
     if (p->n < BN || p->n > 65536 || p->n % BN) return QGMM_ERR_SHAPE;
@@ -406,7 +407,7 @@ QGMM_API qgmm_status qgmm_finalize_workspace(const qgmm_problem *p, size_t *ws_b
 }
 
 namespace {
-qgmm_status finalize_impl(const qgmm_problem *p, const int8_t *x1, const void *x2, const float *scale,
+qgmm_status finalize_impl(const qgmm_problem *p, const int8_t *x1, const void *x2, const void *scale,
                           const float *pertoken_scale, const int64_t *group_list, const float *logit,
                           const void *row_index, const float *bias, const uint16_t *shared_input, float *out,
                           void *workspace, size_t ws_bytes, void *cuda_stream, cudaEvent_t ev_begin,
@@ -436,6 +437,7 @@ qgmm_status finalize_impl(const qgmm_problem *p, const int8_t *x1, const void *x
 
     GemmArgs a = base_args(p, group_list, pl, status);
     a.scale = scale;
+    a.scale_bf16 = p->scale_type == QGMM_SCALE_BF16;
     a.pts = pertoken_scale;
     a.logit = logit;
     a.bias = bias;
@@ -478,7 +480,7 @@ qgmm_status finalize_impl(const qgmm_problem *p, const int8_t *x1, const void *x
 }
 }  // namespace
 
-QGMM_API qgmm_status qgmm_finalize(const qgmm_problem *p, const int8_t *x1, const void *x2, const float *scale,
+QGMM_API qgmm_status qgmm_finalize(const qgmm_problem *p, const int8_t *x1, const void *x2, const void *scale,
                                    const float *pertoken_scale, const int64_t *group_list, const float *logit,
                                    const void *row_index, const float *bias, const uint16_t *shared_input,
                                    float *out, void *workspace, size_t ws_bytes, void *cuda_stream)
@@ -488,7 +490,7 @@ QGMM_API qgmm_status qgmm_finalize(const qgmm_problem *p, const int8_t *x1, cons
 }
 
 QGMM_API qgmm_status qgmm_finalize_profiled(const qgmm_problem *p, const int8_t *x1, const void *x2,
-                                            const float *scale, const float *pertoken_scale,
+                                            const void *scale, const float *pertoken_scale,
                                             const int64_t *group_list, const float *logit, const void *row_index,
                                             const float *bias, const uint16_t *shared_input, float *out,
                                             void *workspace, size_t ws_bytes, void *cuda_stream,
@@ -616,7 +618,7 @@ qgmm_status static_scratch_address(void **out)
 }  // namespace qgmm
 
 QGMM_API qgmm_status qgmm_finalize_static_scratch(const qgmm_problem *p, const int8_t *x1, const void *x2,
-                                                  const float *scale, const float *pertoken_scale,
+                                                  const void *scale, const float *pertoken_scale,
                                                   const int64_t *group_list, const float *logit,
                                                   const void *row_index, const float *bias,
                                                   const uint16_t *shared_input, float *out, void *cuda_stream)

@@ -11,8 +11,8 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (QGMM_IDX_INT32, QGMM_IDX_INT64, QGMM_W_INT4_PACKED_INT32, QGMM_W_INT8, debug_accum,
-               device_status, finalize, finalize_workspace, make_problem, per_token_quant)
+from . import (QGMM_IDX_INT32, QGMM_IDX_INT64, QGMM_SCALE_BF16, QGMM_SCALE_F32, QGMM_W_INT4_PACKED_INT32, QGMM_W_INT8,
+               debug_accum, device_status, finalize, finalize_workspace, make_problem, per_token_quant)
 
 
 def to_device(a: Optional[np.ndarray], device) -> Optional[torch.Tensor]:
@@ -47,6 +47,8 @@ class DeviceProblem:
         self.x2 = to_device(p.x2, dev)
         self.group_list = to_device(p.group_list.astype(np.int64), dev)
         self.scale = to_device(p.scale, dev) if with_optional else None
+        # a uint16 scale array holds bf16 bits
+        self.scale_type = QGMM_SCALE_BF16 if p.scale is not None and p.scale.dtype == np.uint16 else QGMM_SCALE_F32
         self.logit = to_device(p.logit, dev) if with_optional else None
         self.row_index = to_device(p.row_index, dev)
         self.row_index_type = QGMM_IDX_INT32 if p.row_index.dtype == np.int32 else QGMM_IDX_INT64
@@ -72,7 +74,8 @@ class DeviceProblem:
         return make_problem(self.m, self.k, self.n, self.e, self.output_bs, weight_type=self.weight_type,
                             group_list_type=self.group_list_type, row_index_type=self.row_index_type,
                             shared_bs=self.shared_bs, shared_offset=self.shared_offset,
-                            deterministic=deterministic, expected_m_per_expert=self.expected_m_per_expert)
+                            deterministic=deterministic, expected_m_per_expert=self.expected_m_per_expert,
+                            scale_type=self.scale_type)
 
     def workspace(self, deterministic: bool = False) -> torch.Tensor:
         key = bool(deterministic)

@@ -47,7 +47,7 @@ def test_problem_struct_layout_matches_header(qgmm, tmp_path):
 int main(void) {
   printf("size %zu\\n", sizeof(qgmm_problem));
   F(m) F(k) F(n) F(e) F(output_bs) F(weight_type) F(group_list_type) F(row_index_type)
-  F(shared_bs) F(shared_offset) F(deterministic) F(expected_m_per_expert)
+  F(shared_bs) F(shared_offset) F(deterministic) F(expected_m_per_expert) F(scale_type)
   return 0;
 }
 """)
@@ -93,6 +93,7 @@ def test_workspace_sizes(qgmm):
     (dict(shared_bs=33), "SHAPE"), (dict(shared_bs=8, shared_offset=25), "SHAPE"),
     (dict(shared_offset=-1), "SHAPE"), (dict(expected_m_per_expert=-1), "SHAPE"),
     (dict(weight_type=2), "DTYPE"), (dict(group_list_type=2), "DTYPE"), (dict(row_index_type=5), "DTYPE"),
+    (dict(scale_type=2), "DTYPE"), (dict(scale_type=-1), "DTYPE"),
 ])
 def test_stage_one_rejects(qgmm, kw, code):
     rc, _ = _ws(qgmm, _prob(qgmm, **kw))

@@ -132,3 +132,16 @@ def test_default_tail_mode_follows_wave_counts(qgmm, monkeypatch):
     assert launches(8192, 32) == 2          # output init + pair GEMM
     assert launches(32768, 32) == 3         # output init + pair GEMM + tail GEMM
     assert launches(131072, 256) == 3
+
+
+@pytest.mark.parametrize("weight,hint", [("int8", 0), ("int8", 200), ("int4", 0), ("int4", 200)])
+def test_bf16_scale(dev, oracle, weight, hint):
+    """scale given as bf16 bits (page 1: scaleOptional is FLOAT or BF16), on every
+    epilogue: 16-row tiles, CTA pairs with their tail launch, and int4 tiles.  The
+    oracle widens the same bits to f32; the bars are those of the f32 scale."""
+    p = _problem(10, [1, 129, 255, 256, 0, 300, 40], 256, 768, weight=weight)
+    rng = np.random.default_rng(11)
+    f32 = rng.uniform(1e-3, 1e-2, size=p.scale.shape).astype(np.float32)
+    p.scale = (f32.view(np.uint32) >> 16).astype(np.uint16)            # truncate to bf16 bits
+    assert dev.DeviceProblem(p, expected_m_per_expert=hint).scale_type == 1
+    _check(dev, oracle, p, hint)

@@ -58,6 +58,42 @@ def test_worked_example_exact(oracle, gtype):
     np.testing.assert_array_equal(oracle.accum(x, w, gl, gtype), [[9, 12, 15], [19, 26, 33]])
 
 
+# --- BF16 scale (page 1: scaleOptional is FLOAT or BF16) ---------------------
+def test_worked_example_with_bf16_scale(oracle):
+    """The worked example with deqScale given as bf16 bits.  1.0 = sign 0, exponent
+    127, mantissa 0 -> 0x3F80; 2.0 -> exponent 128 -> 0x4000; 3.0 = 1.5 * 2 -> exponent
+    128, mantissa 0b1000000 -> 0x4040.  The output is the printed one, exactly."""
+    g = _golden("per_token_worked_example.json")
+    assert g["deqScale"] == [1, 2, 3]
+    x = np.array(g["x"], np.int8)
+    w = np.array(g["weight"], np.int8)[None]
+    scale_bf16 = np.array([[0x3F80, 0x4000, 0x4040]], np.uint16)
+    o64, _, o32 = oracle.finalize(x, w, np.array([2], np.int64), 1, scale=scale_bf16,
+                                  pertoken_scale=np.array(g["perTokenScale"], np.float32),
+                                  row_index=np.array([0, 1], np.int64), output_bs=2)
+    expect = np.array(g["output"], np.float64)
+    np.testing.assert_array_equal(o64, expect)
+    np.testing.assert_array_equal(o32.astype(np.float64), expect)
+
+
+def test_bf16_widening_matches_the_format_definition(oracle):
+    """Every bf16 bit pattern against the format's definition: sign, 8-bit exponent
+    (bias 127), 7-bit fraction; exponent 0 is subnormal (fraction * 2^-133), 255 is
+    infinity (fraction 0) or NaN."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    with np.errstate(invalid="ignore"):                 # signalling-NaN patterns quieten in the cast
+        got = oracle.bf16_to_f32(bits).astype(np.float64)
+    b = bits.astype(np.int64)
+    sign = np.where(b >> 15, -1.0, 1.0)
+    ex, fr = (b >> 7) & 0xFF, b & 0x7F
+    normal = sign * (1.0 + fr / 128.0) * np.exp2(np.minimum(ex, 254).astype(np.float64) - 127.0)
+    sub = sign * fr * 2.0 ** -133
+    want = np.where(ex == 0, sub, np.where(ex == 255, np.where(fr == 0, sign * np.inf, np.nan), normal))
+    nan = np.isnan(want)
+    assert np.isnan(got[nan]).all()
+    np.testing.assert_array_equal(got[~nan], want[~nan])
+
+
 # --- library routine: numpy integer matmul per group ------------------------
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_accum_matches_numpy_matmul(oracle, seed):
