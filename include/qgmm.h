@@ -98,6 +98,11 @@ enum { QGMM_SCALE_F32 = 0, QGMM_SCALE_BF16 = 1 };         /* scale element type 
  *                   `scale` (page 1: scaleOptional is FLOAT or BF16 on A2/A3).
  *                   A bf16 scale is widened to f32, which is exact, and then
  *                   enters the same f32 dequant.
+ *   transpose_x2    0: int8 x2 is (e, k, n); 1: int8 x2 is (e, n, k) (page 1,
+ *                   full-quant scenario: x2 may be transposed, (e, n, k), on
+ *                   Atlas 350; A2/A3 take only the non-transposed layout).
+ *                   Same result either way.  int4 weights must be
+ *                   non-transposed (QGMM_ERR_UNSUPPORTED otherwise).
  */
 typedef struct {
     int64_t m, k, n, e, output_bs;
@@ -106,6 +111,7 @@ typedef struct {
     int32_t deterministic;
     int64_t expected_m_per_expert;
     int32_t scale_type;
+    int32_t transpose_x2;
 } qgmm_problem;
 
 /*
@@ -132,7 +138,8 @@ qgmm_status qgmm_finalize_launches(const qgmm_problem *p, int32_t *launches);
 /*
  * Stage 2: run the operation on `cuda_stream`.
  *   x1              int8 [m, k] row-major, required
- *   x2              int8 [e, k, n] or int32 [e, k, n/8], row-major, required
+ *   x2              int8 [e, k, n] (or [e, n, k] with transpose_x2) or int32
+ *                   [e, k, n/8], row-major, required
  *   scale           f32 or bf16 bits [e, n] (page 1's (e, 1, n)), by scale_type; NULL = all ones
  *   pertoken_scale  f32 [m]; NULL = all ones
  *   group_list      int64 [e], required

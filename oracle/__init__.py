@@ -75,17 +75,22 @@ def group_offsets(group_list: np.ndarray, group_list_type: int, m: int) -> np.nd
     return off
 
 
-def _weights(x2: np.ndarray, weight: str):
+def _weights(x2: np.ndarray, weight: str, transpose_x2: bool = False):
+    """The C oracle's weight layout, (e, k, n) int8 or (e, k, n/8) int32.  A transposed
+    int8 x2 (page 1, full-quant scenario: (e, n, k)) is swapped back to it."""
     if weight == "int8":
-        return _c(x2, np.int8), 0
+        return _c(np.swapaxes(x2, 1, 2) if transpose_x2 else x2, np.int8), 0
+    if transpose_x2:
+        raise ValueError("transposed x2 is int8 only")
     return _c(x2, np.int32), 1
 
 
 def accum(x1, x2, group_list, group_list_type: int, weight: str = "int8",
-          rows: Optional[np.ndarray] = None, threads: Optional[int] = None) -> np.ndarray:
+          rows: Optional[np.ndarray] = None, threads: Optional[int] = None,
+          transpose_x2: bool = False) -> np.ndarray:
     """Exact int32 accumulators ``x1[i] @ W[g(i)]`` for source rows ``rows`` (default all)."""
     x1 = _c(x1, np.int8)
-    w, wt = _weights(x2, weight)
+    w, wt = _weights(x2, weight, transpose_x2)
     m, k = x1.shape
     e = w.shape[0]
     n = w.shape[2] * (8 if wt else 1)
@@ -103,7 +108,7 @@ def finalize(x1, x2, group_list, group_list_type: int, *, weight: str = "int8",
              scale=None, pertoken_scale=None, logit=None, bias=None, row_index=None,
              shared=None, shared_offset: int = 0, output_bs: Optional[int] = None,
              dest_rows: Optional[np.ndarray] = None, want64: bool = True, want32: bool = True,
-             threads: Optional[int] = None):
+             threads: Optional[int] = None, transpose_x2: bool = False):
     """The op's output rows ``dest_rows`` (default all ``output_bs`` rows).
 
     ``scale`` is f32, or uint16 holding bf16 bits (widened exactly by the C oracle).
@@ -116,7 +121,7 @@ def finalize(x1, x2, group_list, group_list_type: int, *, weight: str = "int8",
     if scale is not None and scale.dtype == np.uint16:
         scale = bf16_to_f32(scale)
     x1 = _c(x1, np.int8)
-    w, wt = _weights(x2, weight)
+    w, wt = _weights(x2, weight, transpose_x2)
     m, k = x1.shape
     e = w.shape[0]
     n = w.shape[2] * (8 if wt else 1)
@@ -177,4 +182,5 @@ def problem_finalize(p, *, x1=None, pertoken_scale=None, dest_rows=None, want64=
                     pertoken_scale=p.pertoken_scale if pertoken_scale is None else pertoken_scale,
                     logit=p.logit, bias=p.bias, row_index=p.row_index, shared=p.shared,
                     shared_offset=p.shared_offset, output_bs=p.output_bs, dest_rows=dest_rows,
-                    want64=want64, want32=want32, threads=threads)
+                    want64=want64, want32=want32, threads=threads,
+                    transpose_x2=bool(getattr(p, "transpose_x2", False)))

@@ -63,6 +63,7 @@ class QgmmProblem(C.Structure):
         ("deterministic", C.c_int32),
         ("expected_m_per_expert", C.c_int64),
         ("scale_type", C.c_int32),
+        ("transpose_x2", C.c_int32),
     ]
 
 
@@ -107,9 +108,11 @@ def status_string(code: int) -> str:
 def make_problem(m: int, k: int, n: int, e: int, output_bs: int, *, weight_type: int = QGMM_W_INT8,
                  group_list_type: int = QGMM_GROUP_CUMSUM, row_index_type: int = QGMM_IDX_INT64,
                  shared_bs: int = 0, shared_offset: int = 0, deterministic: bool = False,
-                 expected_m_per_expert: int = 0, scale_type: int = QGMM_SCALE_F32) -> QgmmProblem:
+                 expected_m_per_expert: int = 0, scale_type: int = QGMM_SCALE_F32,
+                 transpose_x2: bool = False) -> QgmmProblem:
     return QgmmProblem(m, k, n, e, output_bs, weight_type, group_list_type, row_index_type, shared_bs,
-                       shared_offset, int(bool(deterministic)), expected_m_per_expert, scale_type)
+                       shared_offset, int(bool(deterministic)), expected_m_per_expert, scale_type,
+                       int(bool(transpose_x2)))
 
 
 def _ptr(t) -> Optional[int]:

@@ -89,6 +89,7 @@ struct GemmArgs {
     int32_t sched;         // which m-tiles this launch covers (SCHED_*)
     int32_t stall_producer;  // test hook: the producer issues no copy, so the MMA wait must run out
     int32_t slab_ntiles;   // n-tiles per slab; divides n / BN
+    int32_t b_kmajor;      // int8 x2 stored (e, n, k): K-major B tiles, the x1 tile's layout
     const void *scale;     // f32 [e, n], or bf16 bits when scale_bf16
     int32_t scale_bf16;
     const float *pts, *logit, *bias;
@@ -646,8 +647,13 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
                         ptx::mbar_arrive_expect_tx(&full[stage], a_bytes + B_STAGE_BYTES);
                         ptx::tma_load_2d(smem_a + stage * A_STAGE_BYTES, &map_a, &full[stage], kb * BK, c.row0);
                         uint8_t *b = smem_b + stage * B_STAGE_BYTES;
-                        ptx::tma_load_3d(b, &map_b, &full[stage], n0, kb * BK, c.g);
-                        ptx::tma_load_3d(b + B_ATOM_BYTES, &map_b, &full[stage], n0 + 128, kb * BK, c.g);
+                        if (args.b_kmajor) {   // 128 n-rows of 128 K bytes per box
+                            ptx::tma_load_3d(b, &map_b, &full[stage], kb * BK, n0, c.g);
+                            ptx::tma_load_3d(b + B_ATOM_BYTES, &map_b, &full[stage], kb * BK, n0 + 128, c.g);
+                        } else {               // 128 n-columns of BK k-rows per box
+                            ptx::tma_load_3d(b, &map_b, &full[stage], n0, kb * BK, c.g);
+                            ptx::tma_load_3d(b + B_ATOM_BYTES, &map_b, &full[stage], n0 + 128, kb * BK, c.g);
+                        }
                     }
                     ++issued[stage];
                     if (++stage == S) {
@@ -671,7 +677,10 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t IDESC = ptx::idesc_i8(BM, BN, true);
+            // int4 tiles are always unpacked MN-major; int8 (e, n, k) weights land K-major
+            const bool bk = !W4 && args.b_kmajor != 0;
+            const uint32_t idesc = ptx::idesc_i8(BM, BN, !bk);
+            const uint32_t b_kstep = bk ? UMMA_K : UMMA_K * 128, b_lbo = bk ? 16 : B_ATOM_BYTES;
             int stage = 0;
             uint32_t phase = 0;
             int lt = 0;
@@ -698,9 +707,10 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
                     for (int kk = 0; kk < BK / UMMA_K; ++kk) {
                         // A: K-major, 128-byte rows, 8-row groups 1024 B apart; step K by 32 bytes
                         const uint64_t adesc = ptx::smem_desc_sw128(a0 + kk * UMMA_K, 16, 1024);
-                        // B: MN-major, 128-column atoms B_ATOM_BYTES apart, 8-row K groups 1024 B apart
-                        const uint64_t bdesc = ptx::smem_desc_sw128(b0 + kk * UMMA_K * 128, B_ATOM_BYTES, 1024);
-                        ptx::mma_i8(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                        // B: MN-major, 128-column atoms B_ATOM_BYTES apart, 8-row K groups 1024 B
+                        // apart; or K-major like A, 8-row n groups 1024 B apart
+                        const uint64_t bdesc = ptx::smem_desc_sw128(b0 + kk * b_kstep, b_lbo, 1024);
+                        ptx::mma_i8(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     ptx::mma_commit(&empty[stage]);
                     if (++stage == S) {
@@ -955,7 +965,10 @@ __global__ void __launch_bounds__(PairCfg<W4>::THREADS, 1)
                         if (leader) ptx::mbar_arrive_expect_tx(&full[stage], TX);
                         const uint32_t fb = ptx::map_to_rank(&full[stage], 0);
                         ptx::tma_load_2d_pair(smem_a + stage * PAIR_A_BYTES, &map_a, fb, kb * BK, my_row);
-                        ptx::tma_load_3d_pair(smem_b + stage * PAIR_B_BYTES, &map_b, fb, my_col, kb * BK, c.g);
+                        if (args.b_kmajor)
+                            ptx::tma_load_3d_pair(smem_b + stage * PAIR_B_BYTES, &map_b, fb, kb * BK, my_col, c.g);
+                        else
+                            ptx::tma_load_3d_pair(smem_b + stage * PAIR_B_BYTES, &map_b, fb, my_col, kb * BK, c.g);
                     }
                     ++issued[stage];
                     if (++stage == S) {
@@ -977,8 +990,10 @@ __global__ void __launch_bounds__(PairCfg<W4>::THREADS, 1)
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (leader CTA only)
         if (lane == 0 && leader) {
-            constexpr uint32_t IDESC_FULL = ptx::idesc_i8(2 * BM, BN, true);   // 256 rows: 128 per CTA
-            constexpr uint32_t IDESC_TAIL = ptx::idesc_i8(BM, BN, true);       // 128 rows: 64 per CTA
+            const bool bk = args.b_kmajor != 0;
+            const uint32_t IDESC_FULL = ptx::idesc_i8(2 * BM, BN, !bk);   // 256 rows: 128 per CTA
+            const uint32_t IDESC_TAIL = ptx::idesc_i8(BM, BN, !bk);       // 128 rows: 64 per CTA
+            const uint32_t b_kstep = bk ? UMMA_K : UMMA_K * 128, b_lbo = bk ? 16 : B_ATOM_BYTES;
             int stage = 0;
             uint32_t phase = 0;
             int lt = 0;
@@ -1007,7 +1022,7 @@ __global__ void __launch_bounds__(PairCfg<W4>::THREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < BK / UMMA_K; ++kk) {
                         const uint64_t adesc = ptx::smem_desc_sw128(a0 + kk * UMMA_K, 16, 1024);
-                        const uint64_t bdesc = ptx::smem_desc_sw128(b0 + kk * UMMA_K * 128, B_ATOM_BYTES, 1024);
+                        const uint64_t bdesc = ptx::smem_desc_sw128(b0 + kk * b_kstep, b_lbo, 1024);
                         ptx::mma_i8_pair(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
                     }
                     ptx::mma_commit_pair(ptx::map_to_rank(&empty[stage], 0));

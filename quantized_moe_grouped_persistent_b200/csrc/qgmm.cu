@@ -93,6 +93,8 @@ qgmm_status check_problem(const qgmm_problem *p)
         return QGMM_ERR_SHAPE;
     if (p->deterministic != 0 && p->deterministic != 1) return QGMM_ERR_SHAPE;
     if (p->expected_m_per_expert < 0) return QGMM_ERR_SHAPE;
+    if (p->transpose_x2 != 0 && p->transpose_x2 != 1) return QGMM_ERR_SHAPE;
+    if (p->transpose_x2 && p->weight_type != QGMM_W_INT8) return QGMM_ERR_UNSUPPORTED;
     return QGMM_OK;
 }
 
@@ -189,7 +191,8 @@ Plan make_plan(const qgmm_problem *p, int sms, int epi)
 }
 
 // x1 map (box: 128 bytes x tile_rows) and weight map: int8 box 128 columns x BK
-// rows; packed int4 box w4_box_words int32 words (8 columns each) x BK rows --
+// rows (transposed int8: BK bytes x 128 n-rows); packed int4 box w4_box_words
+// int32 words (8 columns each) x BK rows --
 // 32 words (256 columns) for the single-CTA kernel, 16 (one CTA's 128 columns)
 // for the CTA pair.
 qgmm_status make_maps(const qgmm_problem *p, const int8_t *x1, const void *x2, int tile_rows, int w4_box_words,
@@ -207,7 +210,17 @@ qgmm_status make_maps(const qgmm_problem *p, const int8_t *x1, const void *x2, i
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return QGMM_ERR_CUDA;
     }
-    if (p->weight_type == QGMM_W_INT8) {
+    if (p->weight_type == QGMM_W_INT8 && p->transpose_x2) {
+        // (e, n, k): K-major B, a box of 128 K bytes x 128 n-rows -- the x1 tile's layout
+        const cuuint64_t gdim[3] = {cuuint64_t(p->k), cuuint64_t(p->n), cuuint64_t(p->e)};
+        const cuuint64_t gstride[2] = {cuuint64_t(p->k), cuuint64_t(p->k) * cuuint64_t(p->n)};
+        const cuuint32_t box[3] = {cuuint32_t(BK), 128, 1};
+        const cuuint32_t es[3] = {1, 1, 1};
+        if (enc(mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(x2), gdim, gstride, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return QGMM_ERR_CUDA;
+    } else if (p->weight_type == QGMM_W_INT8) {
         const cuuint64_t gdim[3] = {cuuint64_t(p->n), cuuint64_t(p->k), cuuint64_t(p->e)};
         const cuuint64_t gstride[2] = {cuuint64_t(p->n), cuuint64_t(p->n) * cuuint64_t(p->k)};
         const cuuint32_t box[3] = {128, cuuint32_t(BK), 1};
@@ -377,6 +390,7 @@ GemmArgs base_args(const qgmm_problem *p, const int64_t *group_list, const Plan 
     // bound, the kernel sets QGMM_DEV_TIMEOUT, frees its TMEM and returns.
     a.stall_producer = env_int("QGMM_TEST_STALL_PRODUCER", 0) != 0 ? 1 : 0;
     a.slab_ntiles = pl.slab_ntiles;
+    a.b_kmajor = p->transpose_x2;
     a.row_index_type = p->row_index_type;
     a.output_bs = p->output_bs;
     a.status = status;

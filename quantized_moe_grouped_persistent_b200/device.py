@@ -45,6 +45,7 @@ class DeviceProblem:
             self.x1 = to_device(p.x1, dev)
             self.pts = to_device(p.pertoken_scale, dev)
         self.x2 = to_device(p.x2, dev)
+        self.transpose_x2 = bool(getattr(p, "transpose_x2", False))   # int8 x2 stored (e, n, k)
         self.group_list = to_device(p.group_list.astype(np.int64), dev)
         self.scale = to_device(p.scale, dev) if with_optional else None
         # a uint16 scale array holds bf16 bits
@@ -75,7 +76,7 @@ class DeviceProblem:
                             group_list_type=self.group_list_type, row_index_type=self.row_index_type,
                             shared_bs=self.shared_bs, shared_offset=self.shared_offset,
                             deterministic=deterministic, expected_m_per_expert=self.expected_m_per_expert,
-                            scale_type=self.scale_type)
+                            scale_type=self.scale_type, transpose_x2=self.transpose_x2)
 
     def workspace(self, deterministic: bool = False) -> torch.Tensor:
         key = bool(deterministic)

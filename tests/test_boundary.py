@@ -47,7 +47,7 @@ def test_problem_struct_layout_matches_header(qgmm, tmp_path):
 int main(void) {
   printf("size %zu\\n", sizeof(qgmm_problem));
   F(m) F(k) F(n) F(e) F(output_bs) F(weight_type) F(group_list_type) F(row_index_type)
-  F(shared_bs) F(shared_offset) F(deterministic) F(expected_m_per_expert) F(scale_type)
+  F(shared_bs) F(shared_offset) F(deterministic) F(expected_m_per_expert) F(scale_type) F(transpose_x2)
   return 0;
 }
 """)
@@ -94,10 +94,19 @@ def test_workspace_sizes(qgmm):
     (dict(shared_offset=-1), "SHAPE"), (dict(expected_m_per_expert=-1), "SHAPE"),
     (dict(weight_type=2), "DTYPE"), (dict(group_list_type=2), "DTYPE"), (dict(row_index_type=5), "DTYPE"),
     (dict(scale_type=2), "DTYPE"), (dict(scale_type=-1), "DTYPE"),
+    (dict(transpose_x2=1, weight_type=1), "UNSUPPORTED"),
 ])
 def test_stage_one_rejects(qgmm, kw, code):
     rc, _ = _ws(qgmm, _prob(qgmm, **kw))
     assert rc == getattr(qgmm, "QGMM_ERR_" + code)
+
+
+def test_stage_one_rejects_unknown_layout_flag(qgmm):
+    p = _prob(qgmm)
+    p.transpose_x2 = 2                       # the struct field itself: the binding passes 0 or 1
+    assert _ws(qgmm, p)[0] == qgmm.QGMM_ERR_SHAPE
+    p.transpose_x2 = 1
+    assert _ws(qgmm, p)[0] == qgmm.QGMM_OK
 
 
 def test_stage_one_accepts_page_limits(qgmm):

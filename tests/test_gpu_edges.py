@@ -57,7 +57,8 @@ def _check(dev, oracle, p, hint):
     assert err.max() <= ATOMIC_TOL
     total = int(p.counts.sum())
     acc = d.accum().cpu().numpy()
-    ref = oracle.accum(p.x1, p.x2, p.group_list, p.group_list_type, weight=p.weight)
+    ref = oracle.accum(p.x1, p.x2, p.group_list, p.group_list_type, weight=p.weight,
+                       transpose_x2=bool(getattr(p, "transpose_x2", False)))
     np.testing.assert_array_equal(acc[:total], ref[:total])
 
 
@@ -144,4 +145,22 @@ def test_bf16_scale(dev, oracle, weight, hint):
     f32 = rng.uniform(1e-3, 1e-2, size=p.scale.shape).astype(np.float32)
     p.scale = (f32.view(np.uint32) >> 16).astype(np.uint16)            # truncate to bf16 bits
     assert dev.DeviceProblem(p, expected_m_per_expert=hint).scale_type == 1
+    _check(dev, oracle, p, hint)
+
+
+@pytest.mark.parametrize("hint,env", [
+    (1, {}),                              # 16-row tiles, single CTA
+    (200, {"QGMM_PAIR": "0"}),            # 128-row tiles, single CTA
+    (200, {"QGMM_PAIR_TAILS": "1"}),      # CTA pairs + single-CTA tail launch
+    (200, {"QGMM_PAIR_TAILS": "2"}),      # CTA pairs, tails as M=128 pair tiles
+])
+def test_transposed_int8_weights(dev, oracle, monkeypatch, hint, env):
+    """int8 x2 stored (e, n, k) (page 1, full-quant scenario: x2 may be transposed):
+    K-major weight tiles on 16-row and 128-row single-CTA tiles and on CTA pairs with
+    either tail form, in both combine modes, against the oracle on the same layout."""
+    for k_, v in env.items():
+        monkeypatch.setenv(k_, v)
+    p = _problem(12, [1, 129, 255, 256, 0, 300, 40, 17], 256, 768)
+    p.x2 = np.ascontiguousarray(np.swapaxes(p.x2, 1, 2))          # (e, n, k)
+    p.transpose_x2 = True
     _check(dev, oracle, p, hint)

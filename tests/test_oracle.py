@@ -94,6 +94,32 @@ def test_bf16_widening_matches_the_format_definition(oracle):
     np.testing.assert_array_equal(got[~nan], want[~nan])
 
 
+# --- transposed x2 (page 1, full-quant scenario: (e, n, k)) -----------------
+def test_worked_example_with_transposed_weight(oracle):
+    """The worked example with its weight [k=2, n=3] given as [n=3, k=2]."""
+    g = _golden("per_token_worked_example.json")
+    x = np.array(g["x"], np.int8)
+    wt = np.array(g["weight"], np.int8).T[None]           # (e=1, n, k)
+    o64, _, _ = oracle.finalize(x, wt, np.array([2], np.int64), 1, transpose_x2=True,
+                                scale=np.array(g["deqScale"], np.float32)[None],
+                                pertoken_scale=np.array(g["perTokenScale"], np.float32),
+                                row_index=np.array([0, 1], np.int64), output_bs=2)
+    np.testing.assert_array_equal(o64, np.array(g["output"], np.float64))
+    np.testing.assert_array_equal(oracle.accum(x, wt, np.array([2], np.int64), 1, transpose_x2=True),
+                                  [[9, 12, 15], [19, 26, 33]])
+
+
+def test_transposed_accum_matches_numpy_matmul(oracle):
+    rng = np.random.default_rng(131)
+    e, k, n = 3, 64, 24
+    counts = np.array([5, 0, 7])
+    x1, x2 = _rand_problem(rng, e, counts, k, n)
+    x2t = np.ascontiguousarray(np.swapaxes(x2, 1, 2))       # (e, n, k)
+    off = np.concatenate([[0], np.cumsum(counts)])
+    ref = np.concatenate([x1[off[g]:off[g + 1]].astype(np.int64) @ x2t[g].astype(np.int64).T for g in range(e)])
+    np.testing.assert_array_equal(oracle.accum(x1, x2t, counts, 1, transpose_x2=True).astype(np.int64), ref)
+
+
 # --- library routine: numpy integer matmul per group ------------------------
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_accum_matches_numpy_matmul(oracle, seed):
