@@ -78,3 +78,35 @@ def test_line_unit_decode_is_bytes_prefill_is_tops():
     assert unit == "GB/s"
     assert factor * bench.int_ops(p) / 1e12 == pytest.approx(bench.algorithmic_bytes(p) / 1e9)
     assert bench.line_unit("mid_prefill", make_problem("mid_prefill", tokens=8, e=4, k=128, n=256)) == ("TOPS", 1.0)
+
+
+def _run_bench(args, env_extra=None):
+    import json
+    import subprocess
+    import sys
+    env = dict(os.environ, **(env_extra or {}))
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], capture_output=True, text=True,
+                       env=env, timeout=240, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    return [json.loads(l) for l in lines]
+
+
+def test_reference_arm_line_contract():
+    """bench.py --impl reference times the oracle and prints one line with the
+    contract's keys; its cpu_baseline and e2e restate the line's own value."""
+    (line,) = _run_bench(["--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "1"])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["unit"] == "TOPS" and line["value"] > 0
+    assert line["steps"] == 2 and line["warmup"] == 1 and line["higher_is_better"] is True
+    assert line["config"]["workload"].startswith("tiny")
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_print_nothing():
+    assert _run_bench(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0"],
+                      {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
