@@ -120,6 +120,26 @@ def test_transposed_accum_matches_numpy_matmul(oracle):
     np.testing.assert_array_equal(oracle.accum(x1, x2t, counts, 1, transpose_x2=True).astype(np.int64), ref)
 
 
+# --- deterministic order: the shared value first, then ascending source rows -----
+def test_f32_sum_order_is_shared_first_then_ascending_rows(oracle):
+    """Hand-worked f32 sums whose result depends on the order.  Three rows reach
+    output row 0 with y = 2^24, 1, -2^24: in ascending order 2^24 + 1 rounds back to
+    2^24 (ties to even) and the sum is 0; descending, it would be 1.  The exact value
+    (f64) is 1.  With a shared value of 2^24 and y = 1, 1: shared first gives 2^24 twice
+    rounded back, so 2^24; contributions first would give 2^24 + 2."""
+    w = np.ones((1, 1, 1), np.int8)
+    t = float(1 << 24)
+    o64, _, o32 = oracle.finalize(np.ones((3, 1), np.int8), w, np.array([3], np.int64), 1,
+                                  pertoken_scale=np.array([t, 1.0, -t], np.float32),
+                                  row_index=np.zeros(3, np.int64), output_bs=1)
+    assert o64[0, 0] == 1.0 and o32[0, 0] == 0.0
+    shared = np.array([[0x4B80]], np.uint16)                 # bf16 2^24: exponent 151, fraction 0
+    o64, _, o32 = oracle.finalize(np.ones((2, 1), np.int8), w, np.array([2], np.int64), 1,
+                                  pertoken_scale=np.array([1.0, 1.0], np.float32),
+                                  row_index=np.zeros(2, np.int64), output_bs=1, shared=shared, shared_offset=0)
+    assert o64[0, 0] == t + 2 and o32[0, 0] == t
+
+
 # --- library routine: numpy integer matmul per group ------------------------
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_accum_matches_numpy_matmul(oracle, seed):
