@@ -294,6 +294,22 @@ def time_e2e(d, p, steps, warmup, deterministic):
     return t0.elapsed_time(t1) / steps, h2d, d2h
 
 
+def gemm_kernel_label(p, gemm_launches, env=None):
+    """Which grouped-GEMM kernel(s) a call runs, for the roofline line.  It follows the
+    library planner's rule (no size hint: m/e rows per expert; 128-row tiles above 64;
+    those run on CTA pairs for int8, or for int4 with QGMM_PAIR_W4=1, unless QGMM_PAIR=0);
+    the launch count, from the library itself, tells a tail launch from in-kernel tails."""
+    env = os.environ if env is None else env
+    full_height = -(-p.m // p.e) > 64
+    pair = (full_height and env.get("QGMM_PAIR", "1") != "0"
+            and (p.weight == "int8" or env.get("QGMM_PAIR_W4", "0") != "0"))
+    if not pair:
+        return "grouped_gemm_kernel"
+    if gemm_launches == 2:
+        return "grouped GEMM (grouped_gemm_pair_kernel + tail launch)"
+    return "grouped_gemm_pair_kernel"
+
+
 def line_unit(workload, p):
     """The JSON line's unit, and the factor taking int8 TOPS of this workload to it:
     decode is HBM-bound and reports algorithmic GB/s (a sample that does a fraction
@@ -437,8 +453,7 @@ def main():
     launches_per_step = op_launches + (1 if d.prologue else 0)
     # the plan's GEMM launches: CTA-pair tiles plus a single-CTA tail launch, or one single-CTA launch
     gemm_launches = op_launches - (6 if args.deterministic else 1)
-    gemm_kernel = ("grouped GEMM (grouped_gemm_pair_kernel + tail launch)" if gemm_launches == 2
-                   else "grouped_gemm_kernel")
+    gemm_kernel = gemm_kernel_label(p, gemm_launches)
 
     extras = {}
     if world == 1 and not args.no_extras:

@@ -110,3 +110,17 @@ def test_reference_arm_line_contract():
 def test_reference_arm_other_ranks_print_nothing():
     assert _run_bench(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0"],
                       {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
+
+
+def test_gemm_kernel_label_follows_the_plan():
+    import bench
+    from synth import make_problem
+    large = make_problem("large_prefill", tokens=256, e=2, k=128, n=256)    # topK 2: 256 rows per expert
+    assert bench.gemm_kernel_label(large, 2, {}) == "grouped GEMM (grouped_gemm_pair_kernel + tail launch)"
+    assert bench.gemm_kernel_label(large, 1, {}) == "grouped_gemm_pair_kernel"
+    assert bench.gemm_kernel_label(large, 1, {"QGMM_PAIR": "0"}) == "grouped_gemm_kernel"
+    dec = make_problem("decode", tokens=4, e=8, k=128, n=256)              # 4 rows per expert
+    assert bench.gemm_kernel_label(dec, 1, {}) == "grouped_gemm_kernel"
+    w4 = make_problem("w4a8_prologue", tokens=256, e=2, k=128, n=256)
+    assert bench.gemm_kernel_label(w4, 1, {}) == "grouped_gemm_kernel"
+    assert bench.gemm_kernel_label(w4, 2, {"QGMM_PAIR_W4": "1"}).startswith("grouped GEMM (grouped_gemm_pair")
