@@ -294,18 +294,11 @@ def time_e2e(d, p, steps, warmup, deterministic):
     return t0.elapsed_time(t1) / steps, h2d, d2h
 
 
-def gemm_kernel_label(p, gemm_launches, env=None):
-    """Which grouped-GEMM kernel(s) a call runs, for the roofline line.  It follows the
-    library planner's rule (no size hint: m/e rows per expert; 128-row tiles above 64;
-    those run on CTA pairs for int8, or for int4 with QGMM_PAIR_W4=1, unless QGMM_PAIR=0);
-    the launch count, from the library itself, tells a tail launch from in-kernel tails."""
-    env = os.environ if env is None else env
-    full_height = -(-p.m // p.e) > 64
-    pair = (full_height and env.get("QGMM_PAIR", "1") != "0"
-            and (p.weight == "int8" or env.get("QGMM_PAIR_W4", "0") != "0"))
-    if not pair:
+def gemm_kernel_label(plan):
+    """Which grouped-GEMM kernel(s) a call runs, from the library's own plan (qgmm_plan)."""
+    if not plan["pair"]:
         return "grouped_gemm_kernel"
-    if gemm_launches == 2:
+    if plan["gemm_launches"] == 2:
         return "grouped GEMM (grouped_gemm_pair_kernel + tail launch)"
     return "grouped_gemm_pair_kernel"
 
@@ -406,7 +399,7 @@ def main():
         return
 
     import torch
-    from quantized_moe_grouped_persistent_b200 import finalize_launches
+    from quantized_moe_grouped_persistent_b200 import finalize_launches, plan
     from quantized_moe_grouped_persistent_b200.device import DeviceProblem
     dist = None
     if world > 1:
@@ -451,9 +444,8 @@ def main():
     value = world * rate(ms_max)
     op_launches = finalize_launches(d.problem(args.deterministic))
     launches_per_step = op_launches + (1 if d.prologue else 0)
-    # the plan's GEMM launches: CTA-pair tiles plus a single-CTA tail launch, or one single-CTA launch
-    gemm_launches = op_launches - (6 if args.deterministic else 1)
-    gemm_kernel = gemm_kernel_label(p, gemm_launches)
+    sms = torch.cuda.get_device_properties(dev_index).multi_processor_count
+    gemm_kernel = gemm_kernel_label(plan(d.problem(args.deterministic), sms))
 
     extras = {}
     if world == 1 and not args.no_extras:

@@ -136,6 +136,29 @@ qgmm_status qgmm_finalize_workspace(const qgmm_problem *p, size_t *ws_bytes);
 qgmm_status qgmm_finalize_launches(const qgmm_problem *p, int32_t *launches);
 
 /*
+ * The grouped GEMM's plan for `p` on a device with `sms` SMs, without touching
+ * any device (host pointers; no counterpart on the pages).  The same planner
+ * qgmm_finalize runs, with the same QGMM_* environment switches read now, for
+ * the call's combine mode (p->deterministic).  Lets a caller (or a test on a
+ * machine without a GPU) see what a call would launch.
+ *   tile_rows      x1 rows per tile: 16, 32, 64 or 128 (from
+ *                  expected_m_per_expert, else m / e)
+ *   pair           1: full-height int8 tiles on CTA pairs (256 rows per tile)
+ *   tail_mode      pair path only: a group's odd last <= 128 rows run as a
+ *                  padded pair tile (0), on a single-CTA launch after the pair
+ *                  launch (1), or as an M = 128 pair tile (2)
+ *   slab_ntiles    output slab width in 256-column tiles (atomic combine)
+ *   grid           CTAs of the main GEMM launch (even on the pair path)
+ *   gemm_launches  GEMM launches per call: 2 with a tail launch, else 1
+ * Errors: NULL_PTR, SHAPE, DTYPE, UNSUPPORTED (as qgmm_finalize_workspace),
+ * and SHAPE when sms < 2.
+ */
+typedef struct {
+    int32_t tile_rows, pair, tail_mode, slab_ntiles, grid, gemm_launches;
+} qgmm_plan_info;
+qgmm_status qgmm_plan(const qgmm_problem *p, int32_t sms, qgmm_plan_info *info);
+
+/*
  * Stage 2: run the operation on `cuda_stream`.
  *   x1              int8 [m, k] row-major, required
  *   x2              int8 [e, k, n] (or [e, n, k] with transpose_x2) or int32

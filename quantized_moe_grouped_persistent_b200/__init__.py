@@ -49,7 +49,7 @@ QGMM_DEV_GROUP_TOTAL_GT_M = 1 << 2
 QGMM_DEV_ROW_INDEX_RANGE = 1 << 3
 QGMM_DEV_TIMEOUT = 1 << 4
 
-EXPORTS = ("qgmm_finalize_workspace", "qgmm_finalize_launches", "qgmm_finalize", "qgmm_finalize_profiled",
+EXPORTS = ("qgmm_finalize_workspace", "qgmm_finalize_launches", "qgmm_plan", "qgmm_finalize", "qgmm_finalize_profiled",
            "qgmm_per_token_quant", "qgmm_debug_accum", "qgmm_device_status", "qgmm_finalize_static_scratch",
            "qgmm_status_string")
 
@@ -65,6 +65,12 @@ class QgmmProblem(C.Structure):
         ("scale_type", C.c_int32),
         ("transpose_x2", C.c_int32),
     ]
+
+
+class QgmmPlanInfo(C.Structure):
+    """Mirror of ``qgmm_plan_info``."""
+    _fields_ = [(name, C.c_int32) for name in ("tile_rows", "pair", "tail_mode", "slab_ntiles", "grid",
+                                               "gemm_launches")]
 
 
 class QgmmError(RuntimeError):
@@ -87,6 +93,7 @@ def lib():
         P, I64, U = C.c_void_p, C.c_int64, C.c_size_t
         L.qgmm_finalize_workspace.argtypes = [C.POINTER(QgmmProblem), C.POINTER(C.c_size_t)]
         L.qgmm_finalize_launches.argtypes = [C.POINTER(QgmmProblem), C.POINTER(C.c_int32)]
+        L.qgmm_plan.argtypes = [C.POINTER(QgmmProblem), C.c_int32, C.POINTER(QgmmPlanInfo)]
         L.qgmm_finalize.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, P, P, P, P, P, P, U, P]
         L.qgmm_finalize_profiled.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, P, P, P, P, P, P, U, P, P, P]
         L.qgmm_per_token_quant.argtypes = [P, I64, I64, P, P, P]
@@ -148,6 +155,13 @@ def finalize_launches(problem: QgmmProblem) -> int:
     out = C.c_int32(0)
     _check(lib().qgmm_finalize_launches(C.byref(problem), C.byref(out)), "qgmm_finalize_launches")
     return out.value
+
+
+def plan(problem: QgmmProblem, sms: int) -> dict:
+    """The grouped GEMM's plan for ``problem`` on a device with ``sms`` SMs (no device needed)."""
+    info = QgmmPlanInfo()
+    _check(lib().qgmm_plan(C.byref(problem), int(sms), C.byref(info)), "qgmm_plan")
+    return {name: getattr(info, name) for name, _ in QgmmPlanInfo._fields_}
 
 
 def finalize(problem: QgmmProblem, x1, x2, scale, pertoken_scale, group_list, logit, row_index, bias,

@@ -529,6 +529,22 @@ QGMM_API qgmm_status qgmm_finalize_launches(const qgmm_problem *p, int32_t *laun
     return QGMM_OK;
 }
 
+QGMM_API qgmm_status qgmm_plan(const qgmm_problem *p, int32_t sms, qgmm_plan_info *info)
+{
+    qgmm_status s = check_problem(p);
+    if (s != QGMM_OK) return s;
+    if (!info) return QGMM_ERR_NULL_PTR;
+    if (sms < 2) return QGMM_ERR_SHAPE;
+    const Plan pl = make_plan(p, sms, p->deterministic ? EPI_STORE_Y : EPI_ATOMIC);
+    info->tile_rows = pl.tile_rows;
+    info->pair = pl.pair ? 1 : 0;
+    info->tail_mode = pl.tail_mode;
+    info->slab_ntiles = pl.slab_ntiles;
+    info->grid = pl.grid;
+    info->gemm_launches = gemm_launches(pl);
+    return QGMM_OK;
+}
+
 QGMM_API qgmm_status qgmm_debug_accum(const qgmm_problem *p, const int8_t *x1, const void *x2,
                                       const int64_t *group_list, int32_t *acc_out, void *workspace,
                                       size_t ws_bytes, void *cuda_stream)

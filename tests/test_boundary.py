@@ -24,7 +24,7 @@ def test_header_declares_the_abi():
     assert _declared_functions() == sorted([
         "qgmm_finalize_workspace", "qgmm_finalize", "qgmm_finalize_profiled", "qgmm_per_token_quant",
         "qgmm_debug_accum", "qgmm_device_status", "qgmm_finalize_static_scratch", "qgmm_status_string",
-        "qgmm_finalize_launches"])
+        "qgmm_finalize_launches", "qgmm_plan"])
 
 
 def test_library_exports_every_declared_symbol(qgmm):
@@ -177,3 +177,68 @@ def test_binding_raises_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(q, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         q.lib()
+
+
+# --- the planner, through qgmm_plan (host only: no device) --------------------
+def _plan(qgmm, m, e, n=7168, k=2048, output_bs=None, sms=148, **kw):
+    return qgmm.plan(qgmm.make_problem(m, k, n, e, output_bs or max(1, m // 8), **kw), sms)
+
+
+@pytest.mark.parametrize("rows_per_expert,tile_rows", [(1, 16), (16, 16), (17, 32), (32, 32), (33, 64), (64, 64),
+                                                      (65, 128), (4096, 128)])
+def test_plan_tile_rows_follow_rows_per_expert(qgmm, rows_per_expert, tile_rows):
+    e = 8
+    assert _plan(qgmm, rows_per_expert * e, e)["tile_rows"] == tile_rows
+    # the tuning hint (page 1: tuningConfigOptional[0]) replaces m / e
+    assert _plan(qgmm, 4096 * e, e, expected_m_per_expert=rows_per_expert)["tile_rows"] == tile_rows
+
+
+def test_plan_pairs_for_full_height_int8_tiles(qgmm, monkeypatch):
+    monkeypatch.delenv("QGMM_PAIR", raising=False)
+    monkeypatch.delenv("QGMM_PAIR_W4", raising=False)
+    assert _plan(qgmm, 131072, 256)["pair"] == 1
+    assert _plan(qgmm, 128, 256)["pair"] == 0                              # decode: 16-row tiles
+    assert _plan(qgmm, 32768, 128, weight_type=qgmm.QGMM_W_INT4_PACKED_INT32)["pair"] == 0
+    monkeypatch.setenv("QGMM_PAIR_W4", "1")
+    assert _plan(qgmm, 32768, 128, weight_type=qgmm.QGMM_W_INT4_PACKED_INT32)["pair"] == 1
+    monkeypatch.setenv("QGMM_PAIR", "0")
+    assert _plan(qgmm, 131072, 256)["pair"] == 0
+
+
+@pytest.mark.parametrize("m,e,mode", [(4096, 32, 2), (8192, 32, 2), (16384, 32, 2), (32768, 32, 1), (65536, 32, 1),
+                                      (32768, 256, 1), (131072, 256, 1)])
+def test_plan_tail_mode_by_wave_counts(qgmm, monkeypatch, m, e, mode):
+    """Tails as M=128 pair tiles when e*28 tail tiles fit 8 waves of 148 SMs and
+    m/256*28 pair tiles fit 32 waves of 74 pairs; else the single-CTA tail launch."""
+    monkeypatch.delenv("QGMM_PAIR_TAILS", raising=False)
+    p = _plan(qgmm, m, e)
+    assert p["pair"] == 1                                  # >= 128 rows per expert: CTA pairs
+    assert p["tail_mode"] == mode
+    assert p["gemm_launches"] == (2 if mode == 1 else 1)
+    monkeypatch.setenv("QGMM_PAIR_TAILS", "0")
+    assert _plan(qgmm, m, e)["tail_mode"] == 0 and _plan(qgmm, m, e)["gemm_launches"] == 1
+
+
+def test_plan_slab_width(qgmm, monkeypatch):
+    """Atomic combine: the widest slab (a divisor of n/256 tiles) within half of x1's
+    bytes, clamped to [32 MB, 128 MB]; the deterministic mode writes rows, no slab."""
+    monkeypatch.delenv("QGMM_SLAB_NTILES", raising=False)
+    assert _plan(qgmm, 131072, 256, output_bs=16384)["slab_ntiles"] == 7        # 7 x 16.8 MB <= 128 MB
+    assert _plan(qgmm, 32768, 128, output_bs=4096)["slab_ntiles"] == 7          # 7 x 4.2 MB <= 33.5 MB
+    assert _plan(qgmm, 8192, 32, output_bs=1024)["slab_ntiles"] == 28           # 28 x 1 MB <= 32 MB
+    assert _plan(qgmm, 131072, 256, output_bs=16384, deterministic=True)["slab_ntiles"] == 28
+    monkeypatch.setenv("QGMM_SLAB_NTILES", "4")
+    assert _plan(qgmm, 131072, 256, output_bs=16384)["slab_ntiles"] == 4
+    monkeypatch.setenv("QGMM_SLAB_NTILES", "5")                                 # not a divisor of 28: ignored
+    assert _plan(qgmm, 131072, 256, output_bs=16384)["slab_ntiles"] == 7
+
+
+def test_plan_grid_and_arguments(qgmm):
+    assert _plan(qgmm, 131072, 256)["grid"] == 148                              # one CTA per SM, in pairs
+    assert _plan(qgmm, 131072, 256, sms=132)["grid"] == 132
+    tiny = _plan(qgmm, 64, 4, n=512, k=256, output_bs=32)                        # 16-row tiles, 2 n-tiles
+    assert tiny["pair"] == 0 and tiny["grid"] == (64 // 16 + 4) * 2
+    p = qgmm.make_problem(64, 256, 512, 4, 32)
+    assert qgmm.lib().qgmm_plan(C.byref(p), 1, C.byref(qgmm.QgmmPlanInfo())) == qgmm.QGMM_ERR_SHAPE
+    assert qgmm.lib().qgmm_plan(C.byref(p), 148, None) == qgmm.QGMM_ERR_NULL_PTR
+    assert qgmm.lib().qgmm_plan(None, 148, C.byref(qgmm.QgmmPlanInfo())) == qgmm.QGMM_ERR_NULL_PTR

@@ -112,15 +112,13 @@ def test_reference_arm_other_ranks_print_nothing():
                       {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
 
 
-def test_gemm_kernel_label_follows_the_plan():
+def test_gemm_kernel_label_follows_the_plan(monkeypatch):
     import bench
-    from synth import make_problem
-    large = make_problem("large_prefill", tokens=256, e=2, k=128, n=256)    # topK 2: 256 rows per expert
-    assert bench.gemm_kernel_label(large, 2, {}) == "grouped GEMM (grouped_gemm_pair_kernel + tail launch)"
-    assert bench.gemm_kernel_label(large, 1, {}) == "grouped_gemm_pair_kernel"
-    assert bench.gemm_kernel_label(large, 1, {"QGMM_PAIR": "0"}) == "grouped_gemm_kernel"
-    dec = make_problem("decode", tokens=4, e=8, k=128, n=256)              # 4 rows per expert
-    assert bench.gemm_kernel_label(dec, 1, {}) == "grouped_gemm_kernel"
-    w4 = make_problem("w4a8_prologue", tokens=256, e=2, k=128, n=256)
-    assert bench.gemm_kernel_label(w4, 1, {}) == "grouped_gemm_kernel"
-    assert bench.gemm_kernel_label(w4, 2, {"QGMM_PAIR_W4": "1"}).startswith("grouped GEMM (grouped_gemm_pair")
+    import quantized_moe_grouped_persistent_b200 as q
+    monkeypatch.delenv("QGMM_PAIR_TAILS", raising=False)
+    label = lambda m, e, **kw: bench.gemm_kernel_label(q.plan(q.make_problem(m, 2048, 7168, e, max(1, m // 8), **kw),
+                                                              148))
+    assert label(131072, 256) == "grouped GEMM (grouped_gemm_pair_kernel + tail launch)"
+    assert label(8192, 32) == "grouped_gemm_pair_kernel"                    # tails inside the pair launch
+    assert label(128, 256) == "grouped_gemm_kernel"                         # decode: 16-row tiles
+    assert label(32768, 128, weight_type=q.QGMM_W_INT4_PACKED_INT32) == "grouped_gemm_kernel"
