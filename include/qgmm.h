@@ -119,7 +119,8 @@ typedef struct {
  * Checks `p` and writes the workspace bytes qgmm_finalize needs with it to
  * *ws_bytes (host pointers).  Atomic mode: 256 bytes (the status word).
  * Deterministic mode: 256 + m*n*4 (f32 rows y) + (2*output_bs + 1 + m)*4
- * rounded up to 256.  Errors: NULL_PTR, SHAPE, DTYPE.
+ * rounded up to 256.  Errors: NULL_PTR, SHAPE, DTYPE, UNSUPPORTED (transpose_x2
+ * with int4 weights).
  */
 qgmm_status qgmm_finalize_workspace(const qgmm_problem *p, size_t *ws_bytes);
 
