@@ -242,3 +242,15 @@ def test_plan_grid_and_arguments(qgmm):
     assert qgmm.lib().qgmm_plan(C.byref(p), 1, C.byref(qgmm.QgmmPlanInfo())) == qgmm.QGMM_ERR_SHAPE
     assert qgmm.lib().qgmm_plan(C.byref(p), 148, None) == qgmm.QGMM_ERR_NULL_PTR
     assert qgmm.lib().qgmm_plan(None, 148, C.byref(qgmm.QgmmPlanInfo())) == qgmm.QGMM_ERR_NULL_PTR
+
+
+def test_plan_tile_rows_override(qgmm, monkeypatch):
+    """QGMM_TILE_ROWS replaces the planner's tile height (16/32/64/128 only); CTA pairs
+    need 128-row tiles."""
+    monkeypatch.setenv("QGMM_TILE_ROWS", "64")
+    p = _plan(qgmm, 131072, 256)
+    assert p["tile_rows"] == 64 and p["pair"] == 0 and p["gemm_launches"] == 1
+    monkeypatch.setenv("QGMM_TILE_ROWS", "48")                 # not a tile height: ignored
+    assert _plan(qgmm, 131072, 256)["tile_rows"] == 128
+    monkeypatch.setenv("QGMM_TILE_ROWS", "128")
+    assert _plan(qgmm, 128, 256)["tile_rows"] == 128 and _plan(qgmm, 128, 256)["pair"] == 1
