@@ -28,7 +28,8 @@
  *  - int4: the lowest nibble of each int32 word is the lowest n index, two's
  *    complement (values -8..7);
  *  - per-token quant: a = max |x|, pts = a/127, inv = 127/a (0 for a zero row),
- *    q = round-half-even(x * inv) clamped to [-127, 127];
+ *    q = round-half-even(x * inv) clamped to [-127, 127]; non-finite inputs as
+ *    IEEE f32 has them (NaN skipped by the absmax), a NaN product gives 0;
  *  - a BF16 scale (page 1, parameter notes: scaleOptional is FLOAT or BF16 on
  *    A2/A3) is widened to f32, which is exact, and then enters the same f32
  *    dequant as a FLOAT scale (qo_bf16_to_f32).
@@ -317,7 +318,13 @@ int qo_bf16_to_f32(const uint16_t *in, int64_t count, float *out)
     return QO_OK;
 }
 
-/* ---- per-token quantisation (f32; the decision is an integer) ----------- */
+/* ---- per-token quantisation (f32; the decision is an integer) -----------
+ * Non-finite inputs (a reading; the pages do not mention them) keep IEEE f32
+ * semantics: a NaN element is not larger than anything, so the absmax skips
+ * it; an infinite element makes a = inf, pts = inf and inv = 127/inf = 0.  A
+ * product x*inv that is NaN (a NaN element, or an infinite one times the zero
+ * inverse) has no integer code and quantises to 0; an infinite product would
+ * saturate like any value past 127. */
 int qo_per_token_quant(const uint16_t *x_bf16, int64_t rows, int64_t k, int8_t *q, float *pts)
 {
     if (!x_bf16 || !q || !pts || rows < 0 || k < 1) return QO_ERR_ARG;
@@ -325,12 +332,16 @@ int qo_per_token_quant(const uint16_t *x_bf16, int64_t rows, int64_t k, int8_t *
         float a = 0.0f;
         for (int64_t j = 0; j < k; ++j) {
             float v = fabsf(bf16_to_f32(x_bf16[i * k + j]));
-            if (v > a) a = v;
+            if (v > a) a = v;               /* false for NaN: skipped */
         }
         pts[i] = a / 127.0f;
         float inv = a > 0.0f ? 127.0f / a : 0.0f;
         for (int64_t j = 0; j < k; ++j) {
             float t = bf16_to_f32(x_bf16[i * k + j]) * inv;
+            if (isnan(t)) {
+                q[i * k + j] = 0;
+                continue;
+            }
             float r = rintf(t);                 /* default mode: half to even */
             if (r > 127.0f) r = 127.0f;
             if (r < -127.0f) r = -127.0f;

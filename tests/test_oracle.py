@@ -140,6 +140,54 @@ def test_f32_sum_order_is_shared_first_then_ascending_rows(oracle):
     assert o64[0, 0] == t + 2 and o32[0, 0] == t
 
 
+def test_f32_dequant_multiplies_scale_first_then_pertoken_scale(oracle):
+    """The f32 dequant is (f32(acc) * scale) * pts, two roundings in that order (page
+    "matmul支持pertoken量化模式", 计算示例: (x.w) * deqScale * perTokenScale).  Worked
+    by hand with u = 2^-23 (spacing u in [1, 2), 2u in [2, 4)), acc = 3,
+    scale = 1 + u, pts = 1 + 3u:
+      (3 * (1+u)) = 3 + 3u, a tie between 3+2u and 3+4u -> 3+4u (even significand);
+      (3+4u) * (1+3u) = 3 + 13u + 12u^2, above the midpoint 3+13u -> 3 + 14u.
+    The other orders round to 3 + 12u: (1+u)(1+3u) = 1 + 4u + 3u^2 -> 1+4u, times 3 is
+    3+12u exactly; 3(1+3u) = 3+9u, a tie -> 3+8u, times (1+u) = 3+11u+8u^2 -> 3+12u.
+    In f32 bits 3 + 14u is 0x40400007 (3.0 is 0x40400000, seven steps of 2u)."""
+    u = 2.0 ** -23
+    o64, _, o32 = oracle.finalize(np.array([[3]], np.int8), np.ones((1, 1, 1), np.int8), np.array([1], np.int64), 1,
+                                  scale=np.array([[1 + u]], np.float32),
+                                  pertoken_scale=np.array([1 + 3 * u], np.float32), output_bs=1)
+    assert o32.view(np.uint32)[0, 0] == 0x40400007
+    assert o64[0, 0] == 3 + 12 * u + 9 * u * u        # exact in double (48 significant bits)
+    # bias comes after both scales: acc = 1, scale = 1, pts = 2, bias = 1 -> 1*1*2 + 1 = 3,
+    # where adding it before the per-token scale would give (1 + 1) * 2 = 4
+    o64, _, o32 = oracle.finalize(np.array([[1]], np.int8), np.ones((1, 1, 1), np.int8), np.array([1], np.int64), 1,
+                                  pertoken_scale=np.array([2.0], np.float32), bias=np.array([[1.0]], np.float32),
+                                  output_bs=1)
+    assert o32[0, 0] == 3.0 and o64[0, 0] == 3.0
+
+
+def test_int32_to_f32_conversion_rounds_to_nearest_even(oracle):
+    """Above 2^24 not every integer is an f32.  Hand-built accumulators, each on its own
+    row and weight column, with unit scales (so out = f32(acc)):
+      2^24 + 1 = 1040*127*127 + 127*24 + 9*1, a tie between 2^24 and 2^24+2 -> 2^24;
+      2^24 + 3 = 1040*127*127 + 127*24 + 11*1, a tie between 2^24+2 and 2^24+4 -> 2^24+4;
+      2^25 + 3 = 2080*127*127 + 127*48 + 19*1, spacing 4: nearer 2^25+4 than 2^25
+    (truncation would give 2^24, 2^24+2 and 2^25)."""
+    k = 2082
+    x1 = np.zeros((3, k), np.int8)
+    w = np.zeros((1, k, 3), np.int8)
+    x1[0, :1041], x1[0, 1041] = 127, 9
+    x1[1, :1041], x1[1, 1041] = 127, 11
+    w[0, :1040, 0], w[0, 1040, 0], w[0, 1041, 0] = 127, 24, 1
+    w[0, :, 1] = w[0, :, 0]
+    x1[2, :2081], x1[2, 2081] = 127, 19
+    w[0, :2080, 2], w[0, 2080, 2], w[0, 2081, 2] = 127, 48, 1
+    gl = np.array([3], np.int64)
+    acc = oracle.accum(x1, w, gl, 1)
+    assert [acc[c, c] for c in range(3)] == [(1 << 24) + 1, (1 << 24) + 3, (1 << 25) + 3]
+    o64, _, o32 = oracle.finalize(x1, w, gl, 1, output_bs=3)
+    assert [float(o32[c, c]) for c in range(3)] == [16777216.0, 16777220.0, 33554436.0]
+    assert [o64[c, c] for c in range(3)] == [16777217.0, 16777219.0, 33554435.0]
+
+
 # --- library routine: numpy integer matmul per group ------------------------
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_accum_matches_numpy_matmul(oracle, seed):
@@ -387,6 +435,31 @@ def test_per_token_quant_hand_cases(oracle):
     assert pts[0] == np.float32(1.0)
     assert pts[1] == np.float32(2.0) / np.float32(127.0)
     assert pts[2] == 0.0
+
+
+def test_per_token_quant_non_finite_inputs(oracle):
+    """Reading for inputs the pages do not cover, with IEEE f32 semantics: the absmax
+    skips NaN; an infinity makes absmax = pts = inf and the inverse 0; a NaN product
+    (NaN input, or inf * 0) quantises to 0.
+      row 0: 1, NaN, -2, 0.5 -> absmax 2, inverse 63.5: 63.5 -> 64 (tie to even),
+             NaN -> 0, -127, 31.75 -> 32; pts = 2/127
+      row 1: +inf, 1, -3 -> pts inf, every code 0 (inf * 0 is NaN, 1 * 0 = 0)
+      row 2: -inf, NaN, 5 -> pts inf, every code 0
+      row 3: all NaN -> absmax 0, pts 0, inverse 0, every code 0"""
+    nan, pinf, ninf = 0x7FC0, 0x7F80, 0xFF80
+    x = np.zeros((4, 8), np.uint16)
+    x[0, [0, 2, 3]] = _bf16_bits([1.0, -2.0, 0.5])
+    x[0, 1] = nan
+    x[1, 0] = pinf
+    x[1, 1:3] = _bf16_bits([1.0, -3.0])
+    x[2, :2] = [ninf, nan]
+    x[2, 2] = _bf16_bits([5.0])[0]
+    x[3, :] = nan
+    q, pts = oracle.per_token_quant(x)
+    np.testing.assert_array_equal(q[0], [64, 0, -127, 32, 0, 0, 0, 0])
+    np.testing.assert_array_equal(q[1:], 0)
+    assert pts[0] == np.float32(2.0) / np.float32(127.0)
+    assert pts[1] == np.inf and pts[2] == np.inf and pts[3] == 0.0
 
 
 def test_per_token_quant_bounds(oracle):
