@@ -189,10 +189,11 @@ def weak_scaling_value(world: int, ops_per_rank: float, ms_max: float) -> float:
 
 
 # ----------------------------------------------------------------------------- device timing
-def time_steps(d, steps, warmup, deterministic, dist=None):
+def time_steps(d, steps, warmup, deterministic, dist=None, per_step=None):
     """Device time of `steps` back-to-back calls (CUDA events on the launch stream),
     and the grouped-GEMM kernel's own average duration from events recorded by the
-    library around its launch."""
+    library around its launch.  If `per_step` is a dict it receives the median and
+    the best single-step time (events between consecutive steps)."""
     import torch
     from quantized_moe_grouped_persistent_b200 import finalize_profiled
     stream = torch.cuda.current_stream()
@@ -214,17 +215,22 @@ def time_steps(d, steps, warmup, deterministic, dist=None):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    marks[0].record(stream)
     for s in range(steps):
         step(*ev[s])
-    t1.record(stream)
+        marks[s + 1].record(stream)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1) / steps
+    ms = marks[0].elapsed_time(marks[-1]) / steps
     gemm_ms = sum(b.elapsed_time(e) for b, e in ev) / steps
+    if per_step is not None:
+        each = sorted(marks[s].elapsed_time(marks[s + 1]) for s in range(steps))
+        gemm_each = sorted(b.elapsed_time(e) for b, e in ev)
+        per_step.update(ms_median=each[len(each) // 2], ms_best=each[0],
+                        gemm_ms_median=gemm_each[len(gemm_each) // 2], gemm_ms_best=gemm_each[0])
     return ms, gemm_ms
 
 
@@ -429,7 +435,8 @@ def main():
     torch.cuda.synchronize()
     flags = d.status(args.deterministic)
     sampler.start()
-    ms, gemm_ms = time_steps(d, args.steps, args.warmup, args.deterministic, dist)
+    per_step = {}
+    ms, gemm_ms = time_steps(d, args.steps, args.warmup, args.deterministic, dist, per_step)
     clocks = sampler.stop()
     ms_max, gemm_max = max_over_ranks([ms, gemm_ms], dist, device="cuda")
     # decode is HBM-bound: its line reports algorithmic GB/s against the measured copy
@@ -522,7 +529,12 @@ def main():
                                        f"of measured"}
         line = {
             "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_max,
+            "step_ms": {"mean": ms_max, "median": per_step["ms_median"], "best": per_step["ms_best"],
+                        "value_at_median": world * rate(per_step["ms_median"]),
+                        "gemm_mean": gemm_max, "gemm_median": per_step["gemm_ms_median"],
+                        "gemm_best": per_step["gemm_ms_best"], "of_rank": rank},
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "config": {"workload": spec_desc, "tokens": p.tokens, "topk": p.topk, "m": p.m, "e": p.e, "k": p.k,
                        "n": p.n, "output_bs": p.output_bs, "mode": mode,

@@ -118,9 +118,15 @@ typedef struct {
  * Stage 1 (page 1: the GetWorkspaceSize call, which validates the inputs).
  * Checks `p` and writes the workspace bytes qgmm_finalize needs with it to
  * *ws_bytes (host pointers).  Atomic mode: 256 bytes (the status word).
- * Deterministic mode: 256 + m*n*4 (f32 rows y) + (2*output_bs + 1 + m)*4
- * rounded up to 256.  Errors: NULL_PTR, SHAPE, DTYPE, UNSUPPORTED (transpose_x2
- * with int4 weights).
+ * Deterministic mode, each part rounded up to 256 bytes:
+ *   256                        status word
+ *   + m*n*4                    f32 rows y
+ *   + S*output_bs*4            per-segment destination histograms, where
+ *                              S = min(1024, max(1, ceil(m/1024)),
+ *                                      max(1, floor(max(2^24, m*n/16) / output_bs)))
+ *   + (output_bs + 1)*4        bucket boundaries
+ *   + m*4                      source rows grouped by destination
+ * Errors: NULL_PTR, SHAPE, DTYPE, UNSUPPORTED (transpose_x2 with int4 weights).
  */
 qgmm_status qgmm_finalize_workspace(const qgmm_problem *p, size_t *ws_bytes);
 
@@ -213,8 +219,8 @@ qgmm_status qgmm_finalize_profiled(const qgmm_problem *p, const int8_t *x1, cons
  *
  *  - Limit: the problem's workspace (qgmm_finalize_workspace) must fit in
  *    16 MiB.  Atomic mode needs 256 bytes, so it always fits; deterministic
- *    mode fits while 256 + m*n*4 + (2*output_bs + 1 + m)*4, each part rounded
- *    up to 256 bytes, stays within 16 MiB (for example m = 128, n = 7168).
+ *    mode fits while its workspace (about m*n*4 bytes plus the bucket lists)
+ *    stays within 16 MiB (for example m = 128, n = 7168).
  *    Larger problems return QGMM_ERR_SCRATCH_LIMIT before anything is launched.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
@@ -251,6 +257,8 @@ qgmm_status qgmm_per_token_quant(const uint16_t *x_bf16, int64_t rows, int64_t k
                                  float *scale_out, void *cuda_stream);
 
 /*
+ * Parity hook (no counterpart on the pages): the op's exact integer stage, so a
+ * test can compare it bit for bit with an independent computation.
  * The raw int32 accumulators acc_out[i][j] = sum_kk x1[i][kk] * W(g, kk, j)
  * for every row i below the groups' total, written by the same grouped GEMM
  * that qgmm_finalize runs (no epilogue arithmetic, no combine).  Rows at or
@@ -264,6 +272,9 @@ qgmm_status qgmm_debug_accum(const qgmm_problem *p, const int8_t *x1, const void
                              size_t ws_bytes, void *cuda_stream);
 
 /*
+ * Page 1, return values of both stages: each call returns a status code (an
+ * aclnnStatus there, qgmm_status here).  Input errors only the device can see
+ * are reported through the workspace status word instead, read by this call.
  * Synchronise `cuda_stream`, then copy the workspace status word written by
  * the last qgmm_finalize / qgmm_debug_accum on that workspace to *flags (host).
  * Returns QGMM_ERR_DEVICE_INPUT when any QGMM_DEV_* bit is set, QGMM_OK when
@@ -271,7 +282,8 @@ qgmm_status qgmm_debug_accum(const qgmm_problem *p, const int8_t *x1, const void
  */
 qgmm_status qgmm_device_status(const void *workspace, uint32_t *flags, void *cuda_stream);
 
-/* A static English description of a status code. */
+/* A static English description of a status code (page 1, return values: the
+ * status code of each stage; here the qgmm_status values above). */
 const char *qgmm_status_string(qgmm_status s);
 
 #ifdef __cplusplus

@@ -614,7 +614,10 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
     const int KB = args.k / BK;
     const int tile_rows = args.tile_rows;
 
+    // The status word is cleared by the kernel this one may overlap under programmatic
+    // dependent launch: wait for that kernel before setting a bit in it.
     auto fail = [&]() {
+        ptx::pdl_wait_primary();
         atomicOr(args.status, QGMM_DEV_TIMEOUT);
         *abort_flag = 1;
     };
@@ -929,7 +932,10 @@ __global__ void __launch_bounds__(PairCfg<W4>::THREADS, 1)
     const int T = MT * NT;
     const int KB = args.k / BK;
 
+    // The status word is cleared by the kernel this one may overlap under programmatic
+    // dependent launch: wait for that kernel before setting a bit in it.
     auto fail = [&]() {
+        ptx::pdl_wait_primary();
         atomicOr(args.status, QGMM_DEV_TIMEOUT);
         *abort_flag = 1;
     };
@@ -1167,11 +1173,19 @@ __global__ void clear_status_kernel(uint32_t *status)
 }
 
 // ---------------------------------------------------------------- K3 (deterministic combine)
-// Workspace: counts[output_bs] (histogram, then fill cursor), starts[output_bs+1], list[m].
-__global__ void det_clear_kernel(int32_t *counts, int64_t output_bs, uint32_t *status)
+// The destination-sorted list of source rows is built in source-row order, so no
+// bucket is ever sorted.  The rows below the total are cut into nseg segments of
+// L = ceil(total / nseg) consecutive rows.  Workspace:
+//   counts[nseg][output_bs]  per-segment histogram of destinations, then (after
+//                            det_colscan) the segment's first slot inside each bucket
+//   starts[output_bs + 1]    bucket boundaries (exclusive scan of the bucket sizes)
+//   list[m]                  source rows grouped by destination, ascending in each
+// det_fill gives each segment to one warp, which walks its rows in ascending order,
+// so every bucket receives segment 0's rows first, each segment's rows in order.
+__global__ void det_clear_kernel(int32_t *counts, int64_t entries, uint32_t *status)
 {
     if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
-    for (int64_t r = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; r < output_bs;
+    for (int64_t r = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; r < entries;
          r += int64_t(gridDim.x) * blockDim.x)
         counts[r] = 0;
 }
@@ -1189,22 +1203,40 @@ __device__ __forceinline__ int64_t groups_total_block(const int64_t *gl, int e, 
 }
 
 __global__ void det_hist_kernel(const int64_t *gl, int e, int type, int64_t m, const void *row_index, int ri_type,
-                                int64_t output_bs, int32_t *counts, uint32_t *status)
+                                int64_t output_bs, int32_t nseg, int32_t *counts, uint32_t *status)
 {
     __shared__ int32_t off[MAX_E + 1], cum[MAX_E + 1];
     const int64_t total = groups_total_block(gl, e, type, m, off, cum, status, blockIdx.x == 0);
+    const int64_t seg_len = (total + nseg - 1) / nseg;
     for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
         const int64_t d = load_row_index(row_index, ri_type, i);
         if (d < 0 || d >= output_bs) {
             atomicOr(status, QGMM_DEV_ROW_INDEX_RANGE);
             continue;
         }
-        atomicAdd(counts + d, 1);
+        atomicAdd(counts + (i / seg_len) * output_bs + d, 1);
     }
 }
 
-// Single block: exclusive scan of counts into starts; counts becomes the fill cursor.
-__global__ void det_scan_kernel(int32_t *counts, int32_t *starts, int64_t output_bs)
+// Per destination d: counts[s][d] <- rows of d in segments before s; sizes[d] <- all rows of d.
+__global__ void det_colscan_kernel(int32_t *counts, int32_t nseg, int64_t output_bs, int32_t *sizes)
+{
+    for (int64_t d = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; d < output_bs;
+         d += int64_t(gridDim.x) * blockDim.x) {
+        int32_t run = 0;
+        for (int32_t s = 0; s < nseg; ++s) {
+            int32_t *c = counts + s * output_bs + d;
+            const int32_t v = *c;
+            *c = run;
+            run += v;
+        }
+        sizes[d] = run;
+    }
+}
+
+// Single block, in place: starts[0..output_bs) holds the bucket sizes on entry and
+// their exclusive scan on exit; starts[output_bs] = the sum.
+__global__ void det_scan_kernel(int32_t *starts, int64_t output_bs)
 {
     __shared__ int32_t warp_sums[32];
     __shared__ int32_t carry;
@@ -1213,7 +1245,7 @@ __global__ void det_scan_kernel(int32_t *counts, int32_t *starts, int64_t output
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
     for (int64_t base = 0; base < output_bs; base += blockDim.x) {
         const int64_t r = base + threadIdx.x;
-        const int32_t v = r < output_bs ? counts[r] : 0;
+        const int32_t v = r < output_bs ? starts[r] : 0;
         int32_t s = v;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
@@ -1233,10 +1265,7 @@ __global__ void det_scan_kernel(int32_t *counts, int32_t *starts, int64_t output
         }
         __syncthreads();
         const int32_t excl = carry + (w ? warp_sums[w - 1] : 0) + s - v;
-        if (r < output_bs) {
-            starts[r] = excl;
-            counts[r] = excl;
-        }
+        if (r < output_bs) starts[r] = excl;
         __syncthreads();
         if (threadIdx.x == blockDim.x - 1) carry = excl + v;
         __syncthreads();
@@ -1244,33 +1273,39 @@ __global__ void det_scan_kernel(int32_t *counts, int32_t *starts, int64_t output
     if (threadIdx.x == 0) starts[output_bs] = carry;
 }
 
+// One warp per segment, 32 source rows at a time in ascending order.  Lanes with the
+// same destination find each other with __match_any_sync and take consecutive slots
+// in lane order after the segment's cursor for that destination; the group's lowest
+// lane then advances the cursor.
 __global__ void det_fill_kernel(const int64_t *gl, int e, int type, int64_t m, const void *row_index, int ri_type,
-                                int64_t output_bs, int32_t *cursor, int32_t *list)
+                                int64_t output_bs, int32_t nseg, int32_t *cursor, const int32_t *starts,
+                                int32_t *list)
 {
     __shared__ int32_t off[MAX_E + 1], cum[MAX_E + 1];
     const int64_t total = groups_total_block(gl, e, type, m, off, cum, nullptr, false);
-    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
-        const int64_t d = load_row_index(row_index, ri_type, i);
-        if (d < 0 || d >= output_bs) continue;
-        const int32_t pos = atomicAdd(cursor + d, 1);
-        list[pos] = static_cast<int32_t>(i);
-    }
-}
-
-// Sort each destination's source rows ascending (buckets hold about topK rows).
-__global__ void det_sort_kernel(const int32_t *starts, int32_t *list, int64_t output_bs)
-{
-    for (int64_t r = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; r < output_bs;
-         r += int64_t(gridDim.x) * blockDim.x) {
-        const int32_t a = starts[r], b = starts[r + 1];
-        for (int32_t x = a + 1; x < b; ++x) {
-            const int32_t v = list[x];
-            int32_t y = x - 1;
-            while (y >= a && list[y] > v) {
-                list[y + 1] = list[y];
-                --y;
+    const int64_t seg_len = (total + nseg - 1) / nseg;
+    const int lane = threadIdx.x & 31;
+    const int wpb = blockDim.x >> 5;
+    for (int64_t s = int64_t(blockIdx.x) * wpb + (threadIdx.x >> 5); s < nseg; s += int64_t(gridDim.x) * wpb) {
+        const int64_t r0 = s * seg_len;
+        const int64_t r1 = r0 + seg_len < total ? r0 + seg_len : total;
+        for (int64_t base = r0; base < r1; base += 32) {
+            const int64_t i = base + lane;
+            long long d = -1;
+            if (i < r1) {
+                d = load_row_index(row_index, ri_type, i);
+                if (d < 0 || d >= output_bs) d = -1;
             }
-            list[y + 1] = v;
+            const uint32_t grp = __match_any_sync(0xffffffffu, d);
+            int32_t *cur = cursor + s * output_bs + (d < 0 ? 0 : d);
+            int32_t slot = 0;
+            if (d >= 0) {
+                slot = *cur;
+                list[starts[d] + slot + __popc(grp & ((1u << lane) - 1u))] = static_cast<int32_t>(i);
+            }
+            __syncwarp();
+            if (d >= 0 && lane == __ffs(grp) - 1) *cur = slot + __popc(grp);
+            __syncwarp();
         }
     }
 }
@@ -1318,6 +1353,9 @@ __global__ void det_reduce_kernel(float *__restrict__ out, const float *__restri
 // One warp per row: absmax over the row, then q = clamp(rn(x * (127/a)), +-127)
 // and scale = a / 127, all in IEEE f32 (page 4, per_token_cast: value times a
 // precomputed inverse).  k % 8 == 0; 16-byte vector loads, 8-byte stores.
+// Non-finite inputs follow IEEE f32: fmaxf skips NaN elements in the absmax, an
+// infinite element makes a = inf, scale = inf and inv = 0; a product x * inv that
+// is NaN (a NaN input, or an infinite one times a zero inverse) gives code 0.
 __global__ void per_token_quant_kernel(const uint16_t *__restrict__ x, int64_t rows, int32_t k, int8_t *__restrict__ q,
                                        float *__restrict__ scale_out)
 {
@@ -1347,12 +1385,11 @@ __global__ void per_token_quant_kernel(const uint16_t *__restrict__ x, int64_t r
             uint32_t packed[2] = {0u, 0u};
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const float f0 = __uint_as_float(w[u] << 16);
-                const float f1 = __uint_as_float(w[u] & 0xFFFF0000u);
-                float r0 = rintf(__fmul_rn(f0, inv));
-                float r1 = rintf(__fmul_rn(f1, inv));
-                r0 = fminf(fmaxf(r0, -127.0f), 127.0f);
-                r1 = fminf(fmaxf(r1, -127.0f), 127.0f);
+                const float t0 = __fmul_rn(__uint_as_float(w[u] << 16), inv);
+                const float t1 = __fmul_rn(__uint_as_float(w[u] & 0xFFFF0000u), inv);
+                // a NaN product has no integer code and becomes 0; infinities saturate
+                const float r0 = t0 != t0 ? 0.0f : fminf(fmaxf(rintf(t0), -127.0f), 127.0f);
+                const float r1 = t1 != t1 ? 0.0f : fminf(fmaxf(rintf(t1), -127.0f), 127.0f);
                 const uint32_t b0 = static_cast<uint32_t>(static_cast<int32_t>(r0)) & 0xFFu;
                 const uint32_t b1 = static_cast<uint32_t>(static_cast<int32_t>(r1)) & 0xFFu;
                 packed[u >> 1] |= (b0 | (b1 << 8)) << (16 * (u & 1));

@@ -98,6 +98,17 @@ qgmm_status check_problem(const qgmm_problem *p)
     return QGMM_OK;
 }
 
+// Segments of the deterministic mode's bucket fill (det_fill_kernel): about 1024
+// source rows each, at most 1024 segments, and the per-segment histograms
+// (segments x output_bs int32) held to max(2^24, m*n/16) entries -- a sixteenth of
+// the f32 rows y the same workspace holds.
+int64_t det_segments(const qgmm_problem *p)
+{
+    int64_t s = std::min<int64_t>(1024, std::max<int64_t>(1, (p->m + 1023) / 1024));
+    const int64_t cap = std::max<int64_t>(int64_t(1) << 24, p->m * p->n / 16);
+    return std::max<int64_t>(1, std::min<int64_t>(s, cap / p->output_bs));
+}
+
 struct DetLayout {
     size_t y, counts, starts, list, total;
 };
@@ -107,7 +118,7 @@ DetLayout det_layout(const qgmm_problem *p)
     DetLayout L;
     L.y = kAlign;
     L.counts = L.y + align_up(size_t(p->m) * size_t(p->n) * 4);
-    L.starts = L.counts + align_up(size_t(p->output_bs) * 4);
+    L.starts = L.counts + align_up(size_t(det_segments(p)) * size_t(p->output_bs) * 4);
     L.list = L.starts + align_up(size_t(p->output_bs + 1) * 4);
     L.total = L.list + align_up(size_t(p->m) * 4);
     return L;
@@ -476,13 +487,19 @@ qgmm_status finalize_impl(const qgmm_problem *p, const int8_t *x1, const void *x
     int32_t *starts = reinterpret_cast<int32_t *>(ws + L.starts);
     int32_t *list = reinterpret_cast<int32_t *>(ws + L.list);
     const int e = static_cast<int>(p->e);
-    det_clear_kernel<<<grid_for(p->output_bs, 256, dev->sms, 4), 256, 0, st>>>(counts, p->output_bs, status);
+    const int64_t nseg = det_segments(p);
+    // destination buckets of source rows, filled in ascending source-row order
+    det_clear_kernel<<<grid_for(nseg * p->output_bs, 256, dev->sms, 4), 256, 0, st>>>(counts, nseg * p->output_bs,
+                                                                                      status);
     det_hist_kernel<<<grid_for(p->m, 256, dev->sms, 4), 256, 0, st>>>(
-        group_list, e, p->group_list_type, p->m, row_index, p->row_index_type, p->output_bs, counts, status);
-    det_scan_kernel<<<1, 1024, 0, st>>>(counts, starts, p->output_bs);
-    det_fill_kernel<<<grid_for(p->m, 256, dev->sms, 4), 256, 0, st>>>(
-        group_list, e, p->group_list_type, p->m, row_index, p->row_index_type, p->output_bs, counts, list);
-    det_sort_kernel<<<grid_for(p->output_bs, 256, dev->sms, 4), 256, 0, st>>>(starts, list, p->output_bs);
+        group_list, e, p->group_list_type, p->m, row_index, p->row_index_type, p->output_bs,
+        static_cast<int32_t>(nseg), counts, status);
+    det_colscan_kernel<<<grid_for(p->output_bs, 256, dev->sms, 4), 256, 0, st>>>(counts, static_cast<int32_t>(nseg),
+                                                                                 p->output_bs, starts);
+    det_scan_kernel<<<1, 1024, 0, st>>>(starts, p->output_bs);
+    det_fill_kernel<<<grid_for(nseg, 8, dev->sms, 8), 256, 0, st>>>(
+        group_list, e, p->group_list_type, p->m, row_index, p->row_index_type, p->output_bs,
+        static_cast<int32_t>(nseg), counts, starts, list);
     if (cudaGetLastError() != cudaSuccess) return QGMM_ERR_CUDA;
     a.out = y;
     if (ev_begin && cudaEventRecord(ev_begin, st) != cudaSuccess) return QGMM_ERR_CUDA;
@@ -524,7 +541,7 @@ QGMM_API qgmm_status qgmm_finalize_launches(const qgmm_problem *p, int32_t *laun
     DeviceInfo *dev = nullptr;
     if ((s = device_info(&dev)) != QGMM_OK) return s;
     const Plan pl = make_plan(p, dev->sms, p->deterministic ? EPI_STORE_Y : EPI_ATOMIC);
-    // atomic: output init; deterministic: clear, histogram, scan, fill, sort, then the reduce
+    // atomic: output init; deterministic: clear, histogram, column scan, scan, fill, then the reduce
     *launches = (p->deterministic ? 6 : 1) + gemm_launches(pl);
     return QGMM_OK;
 }

@@ -83,6 +83,12 @@ def test_workspace_sizes(qgmm):
     assert rc == qgmm.QGMM_OK
     assert n == 256 + al(m * nn * 4) + al(obs * 4) + al((obs + 1) * 4) + al(m * 4)
     assert qgmm.finalize_workspace(_prob(qgmm, m=131072, k=2048, n=7168, e=256, output_bs=16384)) == 256
+    # deterministic: S per-segment histograms of output_bs int32 each,
+    # S = min(1024, max(1, ceil(m / 1024)), max(1, max(2^24, m*n/16) // output_bs))
+    for m, nn, obs, segs in ((131072, 7168, 16384, 128), (131072, 7168, 1, 128), (1 << 24, 256, 1 << 21, 128),
+                             (1 << 21, 65536, 1 << 20, 1024), (3000, 256, 1 << 23, 2), (1 << 21, 256, 5, 1024)):
+        got = qgmm.finalize_workspace(_prob(qgmm, m=m, k=128, n=nn, e=4, output_bs=obs, deterministic=True))
+        assert got == 256 + al(m * nn * 4) + al(segs * obs * 4) + al((obs + 1) * 4) + al(m * 4), (m, obs)
 
 
 @pytest.mark.parametrize("kw,code", [

@@ -40,22 +40,38 @@ def dev(qgmm):
 
 
 def _problems():
+    """(problem, tiling hint): decode-sized single-CTA tiles; a 200-rows-per-expert hint,
+    which plans full-height tiles on CTA pairs, here with groups of 1 to 3 half tiles of
+    128 rows (so pair tiles and odd tails); int4 weights after the per-token quant
+    prologue."""
     from synth import make_problem
-    return [make_problem("decode", tokens=16, e=64, k=512, n=1024),          # bias, many empty experts
-            make_problem("large_prefill", tokens=64, e=16, k=256, n=512)]    # bf16 sharedInput rows
+    return [(make_problem("decode", tokens=16, e=64, k=512, n=1024), 0),          # bias, many empty experts
+            (make_problem("large_prefill", tokens=64, e=16, k=256, n=512), 0),    # bf16 sharedInput rows
+            (make_problem("large_prefill", tokens=360, e=12, k=256, n=512, seed=82), 200),
+            (make_problem("w4a8_prologue", tokens=48, e=8, k=256, n=512), 0)]
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("tails", ["1", "2"])
 @pytest.mark.parametrize("deterministic", [True, False])
-def test_static_scratch_matches_workspace_entry_point(dev, qgmm, oracle, deterministic):
-    for p in _problems():
-        d = dev.DeviceProblem(p)
+def test_static_scratch_matches_workspace_entry_point(dev, qgmm, oracle, deterministic, tails, monkeypatch):
+    # odd tails of the pair path: a single-CTA launch after the pair launch (1), or
+    # M = 128 pair tiles inside it (2); the library reads the switch at each call
+    monkeypatch.setenv("QGMM_PAIR_TAILS", tails)
+    for p, hint in _problems():
+        d = dev.DeviceProblem(p, expected_m_per_expert=hint)
+        if hint:
+            assert qgmm.plan(d.problem(deterministic), 148)["pair"] == 1
         prob = d.problem(deterministic)
         assert qgmm.finalize_workspace(prob) <= qgmm.QGMM_STATIC_SCRATCH_BYTES
         ref = d.run(deterministic=deterministic).clone()
         assert d.status(deterministic) == 0
         ref_h = ref.cpu().numpy()
-        _, sabs, _ = oracle.problem_finalize(p, want32=False)
+        if p.x1 is None:                                         # prologue workload: the oracle's own codes
+            q, s = oracle.per_token_quant(p.x_bf16)
+            _, sabs, _ = oracle.problem_finalize(p, x1=q, pertoken_scale=s, want32=False)
+        else:
+            _, sabs, _ = oracle.problem_finalize(p, want32=False)
         den = np.where(sabs > 0, sabs, 1.0)
         for _ in range(2):                                       # two calls in a row share the array
             out = torch.full_like(ref, float("nan"))
