@@ -8,9 +8,13 @@ resident in HBM.  Default workload: the large prefill (tokens=16384, topK=8,
 m=131072, e=256, k=2048, n=7168, Dirichlet(0.3) routing, bf16 sharedInput),
 atomic combine.  The metric is effective INT8 TOPS = 2 * sum_g m_g * k * n / t.
 
-Multi-GPU (torchrun, one process per GPU): every rank runs its own batch
-(weak scaling, no collective on the data path); ``value`` is all ranks' work
-over the slowest rank's device time.
+Multi-GPU (torchrun, one process per GPU): the op's output columns are split
+across the GPUs (whole 256-column tiles, as evenly as the tile count allows);
+every rank holds x1 and the routing in full and its own columns of the weights,
+scale, bias and sharedInput, and computes its own output columns -- no
+collective on the data path (strong scaling: the total work is the one
+workload).  ``value`` is the whole workload's work over the slowest rank's
+device time.
 
 ``--impl reference`` times the CPU oracle instead, on a bounded sample of the
 same workload's output rows (rank 0 only).
@@ -168,10 +172,15 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- ranks
-def rank_seed(spec_index: int, rank: int):
-    """Seed of rank `rank`'s batch: rank 0 uses the workload's own seed, others an offset one."""
-    from synth.inputs import SEED_BASE
-    return None if rank == 0 else SEED_BASE + spec_index + 1000 * rank
+def rank_problem(p_full, world: int, rank: int):
+    """Rank `rank`'s share of the workload: its block of output columns (the whole
+    problem on one GPU).  Every rank draws the same seeded problem and keeps its
+    columns of x2, scale, bias and sharedInput."""
+    from quantized_moe_grouped_persistent_b200.shard import column_block, slice_columns
+    c0, c1 = column_block(p_full.n, world, rank)
+    if c1 == c0:
+        raise SystemExit(f"{world} GPUs exceed the {p_full.n // 256} column tiles of the workload")
+    return (p_full if world == 1 else slice_columns(p_full, c0, c1)), (c0, c1)
 
 
 def max_over_ranks(values, dist=None, device="cpu"):
@@ -183,9 +192,10 @@ def max_over_ranks(values, dist=None, device="cpu"):
     return [float(x) for x in t.tolist()]
 
 
-def weak_scaling_value(world: int, ops_per_rank: float, ms_max: float) -> float:
-    """Whole-job effective TOPS: every rank's work over the slowest rank's time."""
-    return world * ops_per_rank / (ms_max * 1e-3) / 1e12
+def strong_scaling_value(total_work: float, ms_max: float) -> float:
+    """Whole-job rate: the whole workload's work (ops, or bytes for the decode line)
+    over the slowest rank's time, per second, in units of 1e12."""
+    return total_work / (ms_max * 1e-3) / 1e12
 
 
 # ----------------------------------------------------------------------------- device timing
@@ -377,7 +387,7 @@ def reference_arm(args, p, spec_desc):
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
         "config": {"workload": spec_desc, "mode": "deterministic order (oracle)"},
         "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -418,9 +428,10 @@ def main():
         torch.cuda.set_device(0)
     dev_index = torch.cuda.current_device()
 
-    p = make_problem(args.workload, seed=rank_seed(spec.index, rank), tokens=args.tokens, e=args.experts)
+    p_full = make_problem(args.workload, tokens=args.tokens, e=args.experts)
     if args.tokens or args.experts:
-        spec_desc += f" (reduced: tokens={p.tokens}, e={p.e})"
+        spec_desc += f" (reduced: tokens={p_full.tokens}, e={p_full.e})"
+    p, (c0, c1) = rank_problem(p_full, world, rank)
     d = DeviceProblem(p)
     ops = int_ops(p)
     peaks = load_peaks()
@@ -439,26 +450,37 @@ def main():
     ms, gemm_ms = time_steps(d, args.steps, args.warmup, args.deterministic, dist, per_step)
     clocks = sampler.stop()
     ms_max, gemm_max = max_over_ranks([ms, gemm_ms], dist, device="cuda")
+    # the int8 tensor rate this device reaches with no memory traffic (CTA-pair
+    # kind::i8 MMAs back to back), timed right after the op on the same GPU
+    from quantized_moe_grouped_persistent_b200 import probe
+    mma_probe = probe.mma_i8_rate()
     # decode is HBM-bound: its line reports algorithmic GB/s against the measured copy
     # bandwidth; the prefill-shaped workloads report int8 TOPS against the tensor peak
-    unit, factor = line_unit(args.workload, p)
+    unit, factor = line_unit(args.workload, p_full)
     hbm_line = unit == "GB/s"
-    work = factor * ops / 1e12
+    work = factor * ops / 1e12            # this rank's columns (the whole workload on one GPU)
 
     def rate(step_ms):
         return work / (step_ms * 1e-3)
 
-    value = world * rate(ms_max)
+    value = strong_scaling_value(factor * int_ops(p_full), ms_max)
     op_launches = finalize_launches(d.problem(args.deterministic))
     launches_per_step = op_launches + (1 if d.prologue else 0)
     sms = torch.cuda.get_device_properties(dev_index).multi_processor_count
     gemm_kernel = gemm_kernel_label(plan(d.problem(args.deterministic), sms))
 
     extras = {}
-    if world == 1 and not args.no_extras:
+    if not args.no_extras:
+        # every rank copies its own inputs in and its own output columns out; the
+        # whole job's rate is over the slowest rank
         e2e_ms, h2d, d2h = time_e2e(d, p, max(4, args.steps // 2), 2, args.deterministic)
-        extras["e2e"] = {"value": rate(e2e_ms), "unit": unit, "h2d_bytes_per_step": h2d,
-                         "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+        if dist is not None:
+            dist.barrier()
+        (e2e_max,) = max_over_ranks([e2e_ms], dist, device="cuda")
+        extras["e2e"] = {"value": strong_scaling_value(factor * int_ops(p_full), e2e_max), "unit": unit,
+                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_max,
+                         "bytes_of_rank": rank}
+    if world == 1 and not args.no_extras:
         if not args.deterministic:
             dms, dgemm = time_steps(d, max(3, args.steps // 2), 2, True)
             extras["deterministic"] = {"ms_per_step": dms, "value": rate(dms), "unit": unit, "gemm_ms": dgemm}
@@ -526,20 +548,24 @@ def main():
                         "kernel": gemm_kernel, "kernel_ms": gemm_max,
                         "frac_of_sustained": achieved / int8_peak_sustained,
                         "peak_source": f"{peaks['source']} bf16 burst x 2 (dense int8 : bf16 nominal ratio), "
-                                       f"of measured"}
+                                       f"of measured",
+                        "probe_int8_tops": mma_probe["tops"], "frac_of_probe": achieved / mma_probe["tops"],
+                        "probe": dict(mma_probe, what="CTA-pair tcgen05.mma kind::i8 M=256 N=256 K=32 back to "
+                                                      "back, no memory traffic, median of launches")}
         line = {
             "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max,
             "step_ms": {"mean": ms_max, "median": per_step["ms_median"], "best": per_step["ms_best"],
-                        "value_at_median": world * rate(per_step["ms_median"]),
+                        "value_at_median": strong_scaling_value(factor * int_ops(p_full), per_step["ms_median"]),
                         "gemm_mean": gemm_max, "gemm_median": per_step["gemm_ms_median"],
                         "gemm_best": per_step["gemm_ms_best"], "of_rank": rank},
-            "higher_is_better": True, "scaling": "weak",
+            "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "config": {"workload": spec_desc, "tokens": p.tokens, "topk": p.topk, "m": p.m, "e": p.e, "k": p.k,
-                       "n": p.n, "output_bs": p.output_bs, "mode": mode,
-                       "l2": "inputs larger than L2 (x2 %.2f GB per rank), no flush" % (p.x2.nbytes / 1e9),
-                       "parallelism": f"dp{world} (independent batch per GPU)"},
+                       "n": p_full.n, "output_bs": p.output_bs, "mode": mode,
+                       "l2": "inputs larger than L2 (x2 %.2f GB on rank 0), no flush" % (p.x2.nbytes / 1e9),
+                       "parallelism": (f"column split over {world} GPUs: rank 0 owns columns [{c0}, {c1}) of "
+                                       f"{p_full.n}; no data-path collective" if world > 1 else "1 GPU")},
             **rates,
             "roofline": roofline,
             "gpu_launches": launches_per_step * args.steps,

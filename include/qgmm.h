@@ -103,6 +103,23 @@ enum { QGMM_SCALE_F32 = 0, QGMM_SCALE_BF16 = 1 };         /* scale element type 
  *                   Atlas 350; A2/A3 take only the non-transposed layout).
  *                   Same result either way.  int4 weights must be
  *                   non-transposed (QGMM_ERR_UNSUPPORTED otherwise).
+ *   ld_x2, ld_sb, ld_out, ld_shared   row strides, 0 = n (no counterpart on the pages).
+ *                   They let a call work on a block of n columns inside wider
+ *                   tensors -- the column split across GPUs, where each GPU
+ *                   owns columns [c0, c0 + n) of an N-column op and passes
+ *                   pointers advanced to column c0:
+ *                     ld_x2   columns of x2's rows: x2 element (g, kk, j) is at
+ *                             (g*k + kk)*ld_x2 + j (int8), word (g*k + kk)*ld_x2/8 + j/8
+ *                             (int4), or (g*ld_x2 + j)*k + kk (transpose_x2);
+ *                             n <= ld_x2 <= 2^23, ld_x2 % 32 == 0
+ *                     ld_sb   row stride of scale and bias: element (g, j) at
+ *                             g*ld_sb + j; n <= ld_sb <= 2^32, ld_sb % 8 == 0
+ *                     ld_out  row stride of out: element (r, j) at r*ld_out + j;
+ *                             n <= ld_out <= 2^32, ld_out % 8 == 0
+ *                     ld_shared   the same for shared_input
+ *                   Columns outside [0, n) of each row are neither read nor
+ *                   written, so calls on disjoint column blocks of the same
+ *                   tensors may run at the same time.
  */
 typedef struct {
     int64_t m, k, n, e, output_bs;
@@ -112,6 +129,7 @@ typedef struct {
     int64_t expected_m_per_expert;
     int32_t scale_type;
     int32_t transpose_x2;
+    int64_t ld_x2, ld_sb, ld_out, ld_shared;
 } qgmm_problem;
 
 /*
@@ -178,6 +196,8 @@ qgmm_status qgmm_plan(const qgmm_problem *p, int32_t sms, qgmm_plan_info *info);
  *   bias            f32 [e, n]; NULL = zeros
  *   shared_input    bf16 bits [shared_bs, n]; required iff shared_bs > 0
  *   out             f32 [output_bs, n], fully overwritten (no need to clear it)
+ * (Rows of x2, scale and bias, out, and shared_input are ld_x2, ld_sb, ld_out
+ * and ld_shared apart; the shapes above are for the default strides.)
  *   workspace       device memory of ws_bytes bytes, 256-byte aligned
  * x1, x2, out, shared_input, scale and bias must be 16-byte aligned.  Rows at
  * or past the groups' total are ignored.

@@ -64,6 +64,7 @@ class QgmmProblem(C.Structure):
         ("expected_m_per_expert", C.c_int64),
         ("scale_type", C.c_int32),
         ("transpose_x2", C.c_int32),
+        ("ld_x2", C.c_int64), ("ld_sb", C.c_int64), ("ld_out", C.c_int64), ("ld_shared", C.c_int64),
     ]
 
 
@@ -116,10 +117,11 @@ def make_problem(m: int, k: int, n: int, e: int, output_bs: int, *, weight_type:
                  group_list_type: int = QGMM_GROUP_CUMSUM, row_index_type: int = QGMM_IDX_INT64,
                  shared_bs: int = 0, shared_offset: int = 0, deterministic: bool = False,
                  expected_m_per_expert: int = 0, scale_type: int = QGMM_SCALE_F32,
-                 transpose_x2: bool = False) -> QgmmProblem:
+                 transpose_x2: bool = False, ld_x2: int = 0, ld_sb: int = 0, ld_out: int = 0,
+                 ld_shared: int = 0) -> QgmmProblem:
     return QgmmProblem(m, k, n, e, output_bs, weight_type, group_list_type, row_index_type, shared_bs,
                        shared_offset, int(bool(deterministic)), expected_m_per_expert, scale_type,
-                       int(bool(transpose_x2)))
+                       int(bool(transpose_x2)), ld_x2, ld_sb, ld_out, ld_shared)
 
 
 def _ptr(t) -> Optional[int]:

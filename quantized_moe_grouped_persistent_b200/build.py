@@ -1,4 +1,5 @@
-"""Compile the sm_100a CUDA library in-tree: quantized_moe_grouped_persistent_b200/libqgmm.so."""
+"""Compile the sm_100a CUDA libraries in-tree: quantized_moe_grouped_persistent_b200/libqgmm.so
+(the op) and libqgmm_probe.so (the int8 tensor-rate probe the benchmark reads its roofline against)."""
 from __future__ import annotations
 
 import glob
@@ -10,6 +11,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libqgmm.so")
 MAIN = os.path.join(HERE, "csrc", "qgmm.cu")
+PROBE_LIB = os.path.join(HERE, "libqgmm_probe.so")
+PROBE = os.path.join(HERE, "csrc", "probe_mma.cu")
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
     "-Xcompiler", "-fPIC,-fvisibility=hidden", "-shared",
@@ -17,20 +20,25 @@ NVCC_FLAGS = [
 
 
 def sources():
-    return sorted(glob.glob(os.path.join(HERE, "csrc", "*"))) + [os.path.join(ROOT, "include", "qgmm.h")]
+    return sorted(glob.glob(os.path.join(HERE, "csrc", "*"))) + sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
+
+
+def _compile(src: str, lib: str, force: bool, verbose: bool) -> str:
+    if not force and os.path.exists(lib):
+        newest = max(os.path.getmtime(s) for s in sources())
+        if os.path.getmtime(lib) >= newest:
+            return lib
+    nvcc = os.environ.get("NVCC", "nvcc")
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc, *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), src, "-o", tmp]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, lib)
+    return lib
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and os.path.exists(LIB):
-        newest = max(os.path.getmtime(s) for s in sources())
-        if os.path.getmtime(LIB) >= newest:
-            return LIB
-    nvcc = os.environ.get("NVCC", "nvcc")
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, *( ["-Xptxas", "-v"] if verbose else []), MAIN, "-o", tmp]
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    _compile(PROBE, PROBE_LIB, force, verbose)
+    return _compile(MAIN, LIB, force, verbose)
 
 
 if __name__ == "__main__":

@@ -90,14 +90,16 @@ struct GemmArgs {
     int32_t stall_producer;  // test hook: the producer issues no copy, so the MMA wait must run out
     int32_t slab_ntiles;   // n-tiles per slab; divides n / BN
     int32_t b_kmajor;      // int8 x2 stored (e, n, k): K-major B tiles, the x1 tile's layout
-    const void *scale;     // f32 [e, n], or bf16 bits when scale_bf16
+    const void *scale;     // f32 [e, ld_sb], or bf16 bits when scale_bf16
     int32_t scale_bf16;
+    int64_t ld_sb;         // row stride of scale and bias (elements)
     const float *pts, *logit, *bias;
     const void *row_index;
     int32_t row_index_type;
     int64_t output_bs;
-    float *out;            // EPI_ATOMIC: out [output_bs, n]; EPI_STORE_Y: y [m, n]
-    int32_t *acc_out;      // EPI_RAW_ACC: [m, n]
+    float *out;            // EPI_ATOMIC: out [output_bs, ldd]; EPI_STORE_Y: y [m, ldd]
+    int32_t *acc_out;      // EPI_RAW_ACC: [m, ldd]
+    int64_t ldd;           // row stride of the destination (out, y or acc_out)
     uint32_t *status;
 };
 
@@ -285,7 +287,7 @@ __device__ __forceinline__ void epi_stage_chunk(float *stage, int lane, const ui
 // The dequant runs here in the op's order: ((f32(acc) * scale) * pts + bias) * logit.
 template <int EPI>
 __device__ __forceinline__ void epi_write_chunk(const GemmArgs &args, const float *stage, const float *rp,
-                                                const float *rl, const long long *rd, int sub, int col4, int n,
+                                                const float *rl, const long long *rd, int sub, int col4, int64_t ldd,
                                                 int64_t chunk_col0, float4 s4, float4 b4)
 {
     const int64_t col = chunk_col0 + col4;
@@ -296,7 +298,7 @@ __device__ __forceinline__ void epi_write_chunk(const GemmArgs &args, const floa
         const float4 v = *reinterpret_cast<const float4 *>(stage + row * EPI_LD + col4);
         if (d >= 0) {
             if constexpr (EPI == EPI_RAW_ACC) {
-                *reinterpret_cast<int4 *>(args.acc_out + d * n + col) =
+                *reinterpret_cast<int4 *>(args.acc_out + d * ldd + col) =
                     make_int4(__float_as_int(v.x), __float_as_int(v.y), __float_as_int(v.z), __float_as_int(v.w));
             } else {
                 const float p = rp[row], l = rl[row];
@@ -305,9 +307,9 @@ __device__ __forceinline__ void epi_write_chunk(const GemmArgs &args, const floa
                 const float y2 = __fmul_rn(__fadd_rn(__fmul_rn(__fmul_rn(v.z, s4.z), p), b4.z), l);
                 const float y3 = __fmul_rn(__fadd_rn(__fmul_rn(__fmul_rn(v.w, s4.w), p), b4.w), l);
                 if constexpr (EPI == EPI_ATOMIC) {
-                    ptx::red_add_v4(args.out + d * n + col, y0, y1, y2, y3);
+                    ptx::red_add_v4(args.out + d * ldd + col, y0, y1, y2, y3);
                 } else {
-                    *reinterpret_cast<float4 *>(args.out + d * n + col) = make_float4(y0, y1, y2, y3);
+                    *reinterpret_cast<float4 *>(args.out + d * ldd + col) = make_float4(y0, y1, y2, y3);
                 }
             }
         }
@@ -349,7 +351,7 @@ __device__ __forceinline__ bool epilogue_tile(const GemmArgs &args, const TileCo
                                               int glob_col, int lane, uint64_t *tfull_bar, uint32_t use,
                                               volatile int *abort_flag, const EpiSmem &sm)
 {
-    const int n = args.n;
+    const int64_t ldd = args.ldd;
     const int col_begin = glob_col;       // tile column of this warp's first TMEM column
     const int sub = lane >> 3;            // row (mod 4) handled in the transposed phase
     const int col4 = (lane & 7) * 4;      // first of the 4 columns handled in the transposed phase
@@ -379,7 +381,7 @@ __device__ __forceinline__ bool epilogue_tile(const GemmArgs &args, const TileCo
         bs[k] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     if (EPI != EPI_RAW_ACC && any) {
-        const int64_t base = static_cast<int64_t>(c.g) * n + static_cast<int64_t>(c.nt) * BN + col_begin + col4;
+        const int64_t base = static_cast<int64_t>(c.g) * args.ld_sb + static_cast<int64_t>(c.nt) * BN + col_begin + col4;
         if (args.scale) {
 #pragma unroll
             for (int k = 0; k < NCH; ++k) sc[k] = load_scale4(args, base + k * 32);
@@ -403,13 +405,13 @@ __device__ __forceinline__ bool epilogue_tile(const GemmArgs &args, const TileCo
             epi_stage_chunk<EPI, SHIFT>(sm.stage, lane, ra);
             ptx::tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>((pc + 1) * 32), rb);
             __syncwarp();
-            epi_write_chunk<EPI>(args, sm.stage, sm.rp, sm.rl, sm.rd, sub, col4, n, n0 + pc * 32, sc[pc], bs[pc]);
+            epi_write_chunk<EPI>(args, sm.stage, sm.rp, sm.rl, sm.rd, sub, col4, ldd, n0 + pc * 32, sc[pc], bs[pc]);
             __syncwarp();
             ptx::tmem_ld_wait(rb);
             epi_stage_chunk<EPI, SHIFT>(sm.stage, lane, rb);
             if (pc + 2 < NCH) ptx::tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>((pc + 2) * 32), ra);
             __syncwarp();
-            epi_write_chunk<EPI>(args, sm.stage, sm.rp, sm.rl, sm.rd, sub, col4, n, n0 + (pc + 1) * 32, sc[pc + 1],
+            epi_write_chunk<EPI>(args, sm.stage, sm.rp, sm.rl, sm.rd, sub, col4, ldd, n0 + (pc + 1) * 32, sc[pc + 1],
                                  bs[pc + 1]);
             __syncwarp();
         }
@@ -434,7 +436,7 @@ constexpr int EPI_CHUNKS = EPI_COLS / 64;
 template <int EPI>
 __device__ __forceinline__ void epi_direct_rows(const GemmArgs &args, const uint32_t (&v)[32], long long dA,
                                                 long long dB, float pA, float pB, float lA, float lB,
-                                                const float2 (&sc)[8], const float2 (&bs)[8], int n, int64_t col0)
+                                                const float2 (&sc)[8], const float2 (&bs)[8], int64_t ldd, int64_t col0)
 {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -445,7 +447,7 @@ __device__ __forceinline__ void epi_direct_rows(const GemmArgs &args, const uint
             if (d < 0) continue;
             const uint32_t u0 = v[4 * j + 2 * h], u1 = v[4 * j + 2 * h + 1];
             if constexpr (EPI == EPI_RAW_ACC) {
-                *reinterpret_cast<int2 *>(args.acc_out + d * n + col) =
+                *reinterpret_cast<int2 *>(args.acc_out + d * ldd + col) =
                     make_int2(static_cast<int>(u0), static_cast<int>(u1));
             } else {
                 const float p = h ? pB : pA, l = h ? lB : lA;
@@ -454,9 +456,9 @@ __device__ __forceinline__ void epi_direct_rows(const GemmArgs &args, const uint
                 const float y1 = __fmul_rn(
                     __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(u1)), sc[j].y), p), bs[j].y), l);
                 if constexpr (EPI == EPI_ATOMIC) {
-                    ptx::red_add_v2(args.out + d * n + col, y0, y1);
+                    ptx::red_add_v2(args.out + d * ldd + col, y0, y1);
                 } else {
-                    *reinterpret_cast<float2 *>(args.out + d * n + col) = make_float2(y0, y1);
+                    *reinterpret_cast<float2 *>(args.out + d * ldd + col) = make_float2(y0, y1);
                 }
             }
         }
@@ -468,7 +470,7 @@ __device__ __forceinline__ bool epilogue_tile_direct(const GemmArgs &args, const
                                                      int rows_here, uint32_t tmem_acc, int q, int col_begin, int lane,
                                                      uint64_t *tfull_bar, uint32_t use, volatile int *abort_flag)
 {
-    const int n = args.n;
+    const int64_t ldd = args.ldd;
     const int t0 = lane & 3, t1 = lane >> 2;
     float pts[4], lg[4];
     long long dst[4];
@@ -504,7 +506,7 @@ __device__ __forceinline__ bool epilogue_tile_direct(const GemmArgs &args, const
             bs[ch][j] = make_float2(0.f, 0.f);
         }
     if (EPI != EPI_RAW_ACC && any) {
-        const int64_t base = static_cast<int64_t>(c.g) * n + n0;
+        const int64_t base = static_cast<int64_t>(c.g) * args.ld_sb + n0;
         if (args.scale) {
 #pragma unroll
             for (int ch = 0; ch < EPI_CHUNKS; ++ch)
@@ -531,9 +533,9 @@ __device__ __forceinline__ bool epilogue_tile_direct(const GemmArgs &args, const
             ptx::tmem_ld_16x256b_x8(col + (static_cast<uint32_t>(q * 32) << 16), va);
             ptx::tmem_ld_16x256b_x8(col + (static_cast<uint32_t>(q * 32 + 16) << 16), vb);
             ptx::tmem_ld_wait2(va, vb);
-            epi_direct_rows<EPI>(args, va, dst[0], dst[1], pts[0], pts[1], lg[0], lg[1], sc[ch], bs[ch], n,
+            epi_direct_rows<EPI>(args, va, dst[0], dst[1], pts[0], pts[1], lg[0], lg[1], sc[ch], bs[ch], ldd,
                                  n0 + 64 * ch);
-            epi_direct_rows<EPI>(args, vb, dst[2], dst[3], pts[2], pts[3], lg[2], lg[3], sc[ch], bs[ch], n,
+            epi_direct_rows<EPI>(args, vb, dst[2], dst[3], pts[2], pts[3], lg[2], lg[3], sc[ch], bs[ch], ldd,
                                  n0 + 64 * ch);
         }
     }
@@ -1135,22 +1137,23 @@ __global__ void __launch_bounds__(PairCfg<W4>::THREADS, 1)
 }
 
 // ---------------------------------------------------------------- K1
-// out[r][:] = f32(shared[r - off][:]) for r in [off, off + bs), else 0.  Also
-// clears the call's status word.  A block walks whole rows; a thread step reads
+// out[r][:] = f32(shared[r - off][:]) for r in [off, off + bs), else 0, over n
+// columns; out rows are ld apart, shared rows ld_sh apart.  Also clears the
+// call's status word.  A block walks whole rows; a thread step reads
 // 8 bf16 (16 bytes) and writes two float4.  The host launches 2 blocks of 256
 // threads per SM, which leaves room on every SM for a grouped-GEMM CTA that
 // programmatic dependent launch lets start while this kernel still runs.
-__global__ void output_init_kernel(float *__restrict__ out, int64_t output_bs, int32_t n,
-                                   const uint16_t *__restrict__ shared, int64_t shared_bs, int64_t shared_off,
-                                   uint32_t *status)
+__global__ void output_init_kernel(float *__restrict__ out, int64_t output_bs, int32_t n, int64_t ld,
+                                   const uint16_t *__restrict__ shared, int64_t ld_sh, int64_t shared_bs,
+                                   int64_t shared_off, uint32_t *status)
 {
     ptx::pdl_launch_dependents();   // the grouped GEMM may start its prologue and mainloop now
     if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
     const int n8 = n / 8;           // n % 256 == 0
     for (int64_t r = blockIdx.x; r < output_bs; r += gridDim.x) {
-        float4 *dst = reinterpret_cast<float4 *>(out + r * n);
+        float4 *dst = reinterpret_cast<float4 *>(out + r * ld);
         const bool sh = shared != nullptr && r >= shared_off && r < shared_off + shared_bs;
-        const uint4 *src = reinterpret_cast<const uint4 *>(shared + (sh ? (r - shared_off) * n : 0));
+        const uint4 *src = reinterpret_cast<const uint4 *>(shared + (sh ? (r - shared_off) * ld_sh : 0));
         for (int c = threadIdx.x; c < n8; c += blockDim.x) {
             float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
             if (sh) {
@@ -1311,10 +1314,11 @@ __global__ void det_fill_kernel(const int64_t *gl, int e, int type, int64_t m, c
 }
 
 // out[r][:] = shared-or-0, then += y[j][:] for the bucket's rows j in ascending order.
-__global__ void det_reduce_kernel(float *__restrict__ out, const float *__restrict__ y, int32_t n,
+// y rows are n apart, out rows ld apart, shared rows ld_sh apart.
+__global__ void det_reduce_kernel(float *__restrict__ out, const float *__restrict__ y, int32_t n, int64_t ld,
                                   const int32_t *__restrict__ starts, const int32_t *__restrict__ list,
-                                  int64_t output_bs, const uint16_t *__restrict__ shared, int64_t shared_bs,
-                                  int64_t shared_off)
+                                  int64_t output_bs, const uint16_t *__restrict__ shared, int64_t ld_sh,
+                                  int64_t shared_bs, int64_t shared_off)
 {
     const int32_t q_per_row = n / 4;
     for (int64_t r = blockIdx.x; r < output_bs; r += gridDim.x) {
@@ -1323,7 +1327,7 @@ __global__ void det_reduce_kernel(float *__restrict__ out, const float *__restri
         for (int32_t c4 = threadIdx.x; c4 < q_per_row; c4 += blockDim.x) {
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
             if (sh) {
-                const uint2 h = __ldg(reinterpret_cast<const uint2 *>(shared + (r - shared_off) * n) + c4);
+                const uint2 h = __ldg(reinterpret_cast<const uint2 *>(shared + (r - shared_off) * ld_sh) + c4);
                 acc.x = __uint_as_float(h.x << 16);
                 acc.y = __uint_as_float(h.x & 0xFFFF0000u);
                 acc.z = __uint_as_float(h.y << 16);
@@ -1344,7 +1348,7 @@ __global__ void det_reduce_kernel(float *__restrict__ out, const float *__restri
                         acc.w = __fadd_rn(acc.w, v[u].w);
                     }
             }
-            reinterpret_cast<float4 *>(out + r * n)[c4] = acc;
+            reinterpret_cast<float4 *>(out + r * ld)[c4] = acc;
         }
     }
 }

@@ -95,8 +95,23 @@ qgmm_status check_problem(const qgmm_problem *p)
     if (p->expected_m_per_expert < 0) return QGMM_ERR_SHAPE;
     if (p->transpose_x2 != 0 && p->transpose_x2 != 1) return QGMM_ERR_SHAPE;
     if (p->transpose_x2 && p->weight_type != QGMM_W_INT8) return QGMM_ERR_UNSUPPORTED;
+    if (p->ld_x2 < 0 || p->ld_sb < 0 || p->ld_out < 0 || p->ld_shared < 0) return QGMM_ERR_SHAPE;
+    if (p->ld_x2 && (p->ld_x2 < p->n || p->ld_x2 % 32)) return QGMM_ERR_SHAPE;
+    if (p->ld_sb && (p->ld_sb < p->n || p->ld_sb % 8)) return QGMM_ERR_SHAPE;
+    if (p->ld_out && (p->ld_out < p->n || p->ld_out % 8)) return QGMM_ERR_SHAPE;
+    if (p->ld_shared && (p->ld_shared < p->n || p->ld_shared % 8)) return QGMM_ERR_SHAPE;
+    // x2's per-expert stride ld_x2 * k bytes stays below the tensor map's 2^40 limit
+    if (p->ld_x2 > (int64_t(1) << 23) || p->ld_sb > (int64_t(1) << 32) || p->ld_out > (int64_t(1) << 32) ||
+        p->ld_shared > (int64_t(1) << 32))
+        return QGMM_ERR_SHAPE;
     return QGMM_OK;
 }
+
+// Column strides, 0 meaning n.
+int64_t ld_x2(const qgmm_problem *p) { return p->ld_x2 ? p->ld_x2 : p->n; }
+int64_t ld_sb(const qgmm_problem *p) { return p->ld_sb ? p->ld_sb : p->n; }
+int64_t ld_out(const qgmm_problem *p) { return p->ld_out ? p->ld_out : p->n; }
+int64_t ld_shared(const qgmm_problem *p) { return p->ld_shared ? p->ld_shared : p->n; }
 
 // Segments of the deterministic mode's bucket fill (det_fill_kernel): about 1024
 // source rows each, at most 1024 segments, and the per-segment histograms
@@ -221,10 +236,11 @@ qgmm_status make_maps(const qgmm_problem *p, const int8_t *x1, const void *x2, i
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return QGMM_ERR_CUDA;
     }
+    const cuuint64_t ld = cuuint64_t(ld_x2(p));
     if (p->weight_type == QGMM_W_INT8 && p->transpose_x2) {
         // (e, n, k): K-major B, a box of 128 K bytes x 128 n-rows -- the x1 tile's layout
         const cuuint64_t gdim[3] = {cuuint64_t(p->k), cuuint64_t(p->n), cuuint64_t(p->e)};
-        const cuuint64_t gstride[2] = {cuuint64_t(p->k), cuuint64_t(p->k) * cuuint64_t(p->n)};
+        const cuuint64_t gstride[2] = {cuuint64_t(p->k), cuuint64_t(p->k) * ld};
         const cuuint32_t box[3] = {cuuint32_t(BK), 128, 1};
         const cuuint32_t es[3] = {1, 1, 1};
         if (enc(mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(x2), gdim, gstride, box, es,
@@ -233,7 +249,7 @@ qgmm_status make_maps(const qgmm_problem *p, const int8_t *x1, const void *x2, i
             return QGMM_ERR_CUDA;
     } else if (p->weight_type == QGMM_W_INT8) {
         const cuuint64_t gdim[3] = {cuuint64_t(p->n), cuuint64_t(p->k), cuuint64_t(p->e)};
-        const cuuint64_t gstride[2] = {cuuint64_t(p->n), cuuint64_t(p->n) * cuuint64_t(p->k)};
+        const cuuint64_t gstride[2] = {ld, ld * cuuint64_t(p->k)};
         const cuuint32_t box[3] = {128, cuuint32_t(BK), 1};
         const cuuint32_t es[3] = {1, 1, 1};
         if (enc(mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(x2), gdim, gstride, box, es,
@@ -243,7 +259,7 @@ qgmm_status make_maps(const qgmm_problem *p, const int8_t *x1, const void *x2, i
     } else {
         const cuuint64_t words = cuuint64_t(p->n / 8);
         const cuuint64_t gdim[3] = {words, cuuint64_t(p->k), cuuint64_t(p->e)};
-        const cuuint64_t gstride[2] = {words * 4, words * 4 * cuuint64_t(p->k)};
+        const cuuint64_t gstride[2] = {ld / 8 * 4, ld / 8 * 4 * cuuint64_t(p->k)};
         const cuuint32_t box[3] = {cuuint32_t(w4_box_words), cuuint32_t(BK), 1};
         const cuuint32_t es[3] = {1, 1, 1};
         if (enc(mb, CU_TENSOR_MAP_DATA_TYPE_INT32, 3, const_cast<void *>(x2), gdim, gstride, box, es,
@@ -405,6 +421,8 @@ GemmArgs base_args(const qgmm_problem *p, const int64_t *group_list, const Plan 
     a.row_index_type = p->row_index_type;
     a.output_bs = p->output_bs;
     a.status = status;
+    a.ld_sb = ld_sb(p);
+    a.ldd = p->n;   // y and acc_out rows; the atomic combine's launch sets ld_out
     return a;
 }
 
@@ -471,9 +489,11 @@ qgmm_status finalize_impl(const qgmm_problem *p, const int8_t *x1, const void *x
 
     if (!p->deterministic) {
         output_init_kernel<<<grid_for(p->output_bs, 1, dev->sms, 2), 256, 0, st>>>(
-            out, p->output_bs, static_cast<int32_t>(p->n), shared, p->shared_bs, p->shared_offset, status);
+            out, p->output_bs, static_cast<int32_t>(p->n), ld_out(p), shared, ld_shared(p), p->shared_bs,
+            p->shared_offset, status);
         if (cudaGetLastError() != cudaSuccess) return QGMM_ERR_CUDA;
         a.out = out;
+        a.ldd = ld_out(p);
         if (ev_begin && cudaEventRecord(ev_begin, st) != cudaSuccess) return QGMM_ERR_CUDA;
         if ((s = launch_gemm(EPI_ATOMIC, dev, p, pl, ma, mb, mb_tail, a, st)) != QGMM_OK) return s;
         if (ev_end && cudaEventRecord(ev_end, st) != cudaSuccess) return QGMM_ERR_CUDA;
@@ -506,7 +526,8 @@ qgmm_status finalize_impl(const qgmm_problem *p, const int8_t *x1, const void *x
     if ((s = launch_gemm(EPI_STORE_Y, dev, p, pl, ma, mb, mb_tail, a, st)) != QGMM_OK) return s;
     if (ev_end && cudaEventRecord(ev_end, st) != cudaSuccess) return QGMM_ERR_CUDA;
     det_reduce_kernel<<<grid_for(p->output_bs, 1, dev->sms, 8), 256, 0, st>>>(
-        out, y, static_cast<int32_t>(p->n), starts, list, p->output_bs, shared, p->shared_bs, p->shared_offset);
+        out, y, static_cast<int32_t>(p->n), ld_out(p), starts, list, p->output_bs, shared, ld_shared(p),
+        p->shared_bs, p->shared_offset);
     return cudaGetLastError() == cudaSuccess ? QGMM_OK : QGMM_ERR_CUDA;
 }
 }  // namespace

@@ -37,6 +37,21 @@ def test_library_exports_every_declared_symbol(qgmm):
     assert {s for s in exported if s.startswith("qgmm")} == set(_declared_functions())
 
 
+def test_probe_library_exports_its_declared_symbol(qgmm):
+    """libqgmm_probe.so (include/qgmm_probe.h): the int8 tensor-rate probe; loads and
+    exports exactly what its header declares.  Argument checks need no device."""
+    text = open(os.path.join(ROOT, "include", "qgmm_probe.h")).read()
+    declared = sorted(set(re.findall(r"^int\s+(qgmm_\w+)\s*\(", text, re.M)))
+    assert declared == ["qgmm_probe_mma_i8"]
+    from quantized_moe_grouped_persistent_b200 import probe
+    out = subprocess.run(["nm", "-D", "--defined-only", probe.PROBE_LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    assert {s for s in re.findall(r" T (\w+)$", out, re.M) if s.startswith("qgmm")} == set(declared)
+    L = probe.lib()
+    assert L.qgmm_probe_mma_i8(0, 10, None, None, None) == 2        # no clusters
+    assert L.qgmm_probe_mma_i8(4, 0, None, None, None) == 2         # no iterations
+
+
 def test_problem_struct_layout_matches_header(qgmm, tmp_path):
     src = tmp_path / "layout.c"
     src.write_text("""
@@ -48,6 +63,7 @@ int main(void) {
   printf("size %zu\\n", sizeof(qgmm_problem));
   F(m) F(k) F(n) F(e) F(output_bs) F(weight_type) F(group_list_type) F(row_index_type)
   F(shared_bs) F(shared_offset) F(deterministic) F(expected_m_per_expert) F(scale_type) F(transpose_x2)
+  F(ld_x2) F(ld_sb) F(ld_out) F(ld_shared)
   return 0;
 }
 """)

@@ -1,8 +1,9 @@
 """The multi-GPU plumbing of bench.py, run as two gloo ranks on the CPU.
 
-Every rank takes the same collective steps; each rank draws its own batch
-(weak scaling, no data-path collective); the reported time is the max over
-ranks and the value all ranks' work over that time.
+Every rank takes the same collective steps; every rank draws the same seeded
+workload and keeps its own block of output columns (strong scaling, no
+data-path collective); the reported time is the max over ranks and the value
+the whole workload's work over that time.
 """
 import os
 import socket
@@ -35,15 +36,16 @@ def _rank_main(rank, world, port, out):
     try:
         mine = [1.0 + rank, 10.0 - rank]                    # different per-rank timings
         got = bench.max_over_ranks(mine, dist, device="cpu")
-        p = make_problem("tiny", seed=bench.rank_seed(1, rank))
+        p, cols = bench.rank_problem(make_problem("tiny"), world, rank)
         dist.barrier()
         import hashlib
-        out.put((rank, got, hashlib.sha256(p.x1.tobytes()).hexdigest(), hashlib.sha256(p.row_index.tobytes()).hexdigest()))
+        out.put((rank, got, cols, hashlib.sha256(p.x1.tobytes()).hexdigest(),
+                 hashlib.sha256(p.x2.tobytes()).hexdigest(), p.x2.shape))
     finally:
         dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_reduce_max_and_draw_distinct_batches():
+def test_two_gloo_ranks_reduce_max_and_split_the_columns():
     world, port = 2, _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
@@ -55,17 +57,28 @@ def test_two_gloo_ranks_reduce_max_and_draw_distinct_batches():
         pr.join(timeout=60)
         assert pr.exitcode == 0
     results.sort()
-    for _, got, _, _ in results:
+    for _, got, _, _, _, _ in results:
         assert got == [2.0, 10.0]                          # max over ranks, on every rank
-    assert results[0][2:] != results[1][2:]                # each rank its own seeded batch
+    assert [r[2] for r in results] == [(0, 256), (256, 512)]   # tiny: n = 512, one tile each
+    assert results[0][3] == results[1][3]                  # x1 (row side) replicated
+    assert results[0][4] != results[1][4]                  # x2: each rank its own columns
+    assert results[0][5] == results[1][5] == (4, 256, 256)
 
 
-def test_weak_scaling_value_and_seeds():
+def test_strong_scaling_value_and_rank_problems():
     import bench
-    assert bench.weak_scaling_value(4, 2e12, 1.0) == pytest.approx(8000.0)
-    assert bench.rank_seed(4, 0) is None
-    assert bench.rank_seed(4, 1) != bench.rank_seed(4, 2)
+    from synth import make_problem
+    assert bench.strong_scaling_value(8e12, 2.0) == pytest.approx(4000.0)
     assert bench.max_over_ranks([3.0, 1.5]) == [3.0, 1.5]  # single process: unchanged
+    p = make_problem("mid_prefill", tokens=16, e=4, k=128, n=768)
+    whole, cols = bench.rank_problem(p, 1, 0)
+    assert whole is p and cols == (0, 768)
+    blocks = [bench.rank_problem(p, 2, r) for r in range(2)]
+    assert [c for _, c in blocks] == [(0, 512), (512, 768)]
+    np.testing.assert_array_equal(np.concatenate([q.x2 for q, _ in blocks], axis=2), p.x2)
+    assert sum(bench.int_ops(q) for q, _ in blocks) == bench.int_ops(p)
+    with pytest.raises(SystemExit):
+        bench.rank_problem(p, 4, 3)                        # 3 tiles, 4 GPUs: rank 3 would get nothing
 
 
 def test_line_unit_decode_is_bytes_prefill_is_tops():
