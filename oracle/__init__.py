@@ -48,8 +48,14 @@ def lib():
                                   P, I64, I64, I64, P, I64, P, P, P, I32]
         L.qo_per_token_quant.argtypes = [P, I64, I64, P, P]
         L.qo_bf16_to_f32.argtypes = [P, I64, P]
-        for f in (L.qo_group_offsets, L.qo_accum, L.qo_finalize, L.qo_per_token_quant, L.qo_bf16_to_f32):
+        L.qo_per_token_quant_mxfp8.argtypes = [P, I64, I64, P, P]
+        for f in (L.qo_group_offsets, L.qo_accum, L.qo_finalize, L.qo_per_token_quant, L.qo_bf16_to_f32,
+                  L.qo_per_token_quant_mxfp8):
             f.restype = C.c_int
+        L.qo_e4m3_encode.argtypes = [C.c_float]
+        L.qo_e4m3_encode.restype = C.c_uint8
+        L.qo_e4m3_decode.argtypes = [C.c_uint8]
+        L.qo_e4m3_decode.restype = C.c_float
         _lib = L
     return _lib
 
@@ -184,3 +190,26 @@ def problem_finalize(p, *, x1=None, pertoken_scale=None, dest_rows=None, want64=
                     shared_offset=p.shared_offset, output_bs=p.output_bs, dest_rows=dest_rows,
                     want64=want64, want32=want32, threads=threads,
                     transpose_x2=bool(getattr(p, "transpose_x2", False)))
+
+
+def e4m3_encode(v: float) -> int:
+    """FLOAT8 E4M3FN code of an f32 value: round to nearest even, saturating at 448."""
+    return int(lib().qo_e4m3_encode(float(v)))
+
+
+def e4m3_decode(code: int) -> float:
+    """The value of an E4M3FN code (NaN for 0x7F / 0xFF)."""
+    return float(lib().qo_e4m3_decode(int(code)))
+
+
+def per_token_quant_mxfp8(x_bf16: np.ndarray):
+    """bf16 bits [rows, k] (k % 32 == 0) -> (E4M3 codes uint8 [rows, k], E8M0 scale
+    codes uint8 [rows, k / 32]); x ~= decode(q) * 2^(sf - 127) per group of 32."""
+    x = _c(x_bf16, np.uint16)
+    rows, k = x.shape
+    q = np.zeros((rows, k), np.uint8)
+    sf = np.zeros((rows, k // 32), np.uint8)
+    rc = lib().qo_per_token_quant_mxfp8(_ptr(x), rows, k, _ptr(q), _ptr(sf))
+    if rc:
+        raise OracleError(rc, "per_token_quant_mxfp8")
+    return q, sf

@@ -350,3 +350,76 @@ int qo_per_token_quant(const uint16_t *x_bf16, int64_t rows, int64_t k, int8_t *
     }
     return QO_OK;
 }
+
+/* ---- per-32-group FP8 E4M3 cast ------------------------------------------
+ * "PTOAS issue 1568", 背景: per_token_cast multiplies each bf16 value by an
+ * inverse scale factor broadcast over its group of 32 elements (a 256-element
+ * tile uses sf_inv[row, tile*8 .. tile*8+7]) and converts the product to
+ * FLOAT8 E4M3FN; the scale factors are packed ("packed SF").  The page does
+ * not say how a scale factor is chosen.  Reading (the block format that
+ * per-32 FP8 groups with packed one-byte scale factors belong to, and the one
+ * page 1's MxA8W4 mode consumes): an E8M0 power of two per group, whose
+ * exponent places the group's largest magnitude in E4M3's top binade:
+ *     amax = max |x| over the group's 32 elements (NaN skipped, as above)
+ *     sf   = max(0, biased f32 exponent of amax - 8)         (E8M0 code)
+ *     inv  = 2^(127 - sf)                                     (exact)
+ *     q    = E4M3(x * inv), round to nearest even, magnitudes past 448
+ *            (and infinities) saturate to 448, NaN gives 0x7F
+ * so x ~= q * 2^(sf - 127).  (amax 0 or an f32-subnormal amax gives sf = 0.)
+ * x * inv is exact in f32 except where it falls below 2^-126, far under
+ * E4M3's smallest subnormal 2^-9, so the one rounding is the E4M3 one. */
+
+/* E4M3FN from its definition: sign, 4 exponent bits (bias 7), 3 fraction bits;
+ * exponent 0 holds subnormals m * 2^-9; S.1111.111 is NaN; no infinities; the
+ * largest finite magnitude is 1.75 * 2^8 = 448 (S.1111.110). */
+uint8_t qo_e4m3_encode(float v)
+{
+    if (isnan(v)) return 0x7F;
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    float a = fabsf(v);
+    if (a >= 448.0f) return sign | 0x7E;
+    if (a < 0.015625f) {                       /* below 2^-6: subnormal grid m * 2^-9 */
+        float m = rintf(a * 512.0f);           /* exact product; m = 8 is 2^-6, code 8 */
+        return sign | (uint8_t)m;
+    }
+    int e = ilogbf(a);                         /* -6 .. 8 */
+    float frac = ldexpf(a, -e) - 1.0f;         /* [0, 1), exact */
+    int m = (int)rintf(frac * 8.0f);           /* exact product, then half to even */
+    if (m == 8) { m = 0; e += 1; }
+    int code = ((e + 7) << 3) | m;
+    if (code > 0x7E) code = 0x7E;              /* the tie at 464 rounds up: saturate */
+    return sign | (uint8_t)code;
+}
+
+/* the value an E4M3FN code stands for (NaN for S.1111.111) */
+float qo_e4m3_decode(uint8_t c)
+{
+    int e = (c >> 3) & 0xF, m = c & 7;
+    float s = (c & 0x80) ? -1.0f : 1.0f;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) return s * ldexpf((float)m, -9);
+    return s * ldexpf(1.0f + (float)m / 8.0f, e - 7);
+}
+
+int qo_per_token_quant_mxfp8(const uint16_t *x_bf16, int64_t rows, int64_t k, uint8_t *q, uint8_t *sf)
+{
+    if (!x_bf16 || !q || !sf || rows < 0 || k < 32 || k % 32) return QO_ERR_ARG;
+    for (int64_t i = 0; i < rows; ++i) {
+        for (int64_t g = 0; g < k / 32; ++g) {
+            const uint16_t *x = x_bf16 + i * k + g * 32;
+            float a = 0.0f;
+            for (int j = 0; j < 32; ++j) {
+                float v = fabsf(bf16_to_f32(x[j]));
+                if (v > a) a = v;               /* false for NaN: skipped */
+            }
+            uint32_t bits;
+            memcpy(&bits, &a, sizeof bits);
+            int biased = (int)((bits >> 23) & 0xFF);
+            int code = biased - 8 > 0 ? biased - 8 : 0;
+            float inv = ldexpf(1.0f, 127 - code);
+            sf[i * (k / 32) + g] = (uint8_t)code;
+            for (int j = 0; j < 32; ++j) q[i * k + g * 32 + j] = qo_e4m3_encode(bf16_to_f32(x[j]) * inv);
+        }
+    }
+    return QO_OK;
+}

@@ -450,13 +450,14 @@ def test_per_token_quant_non_finite_inputs(oracle):
     x = np.zeros((4, 8), np.uint16)
     x[0, [0, 2, 3]] = _bf16_bits([1.0, -2.0, 0.5])
     x[0, 1] = nan
+    x[0, 4] = nan                                                # a NaN after the row's max as well
     x[1, 0] = pinf
     x[1, 1:3] = _bf16_bits([1.0, -3.0])
     x[2, :2] = [ninf, nan]
     x[2, 2] = _bf16_bits([5.0])[0]
     x[3, :] = nan
     q, pts = oracle.per_token_quant(x)
-    np.testing.assert_array_equal(q[0], [64, 0, -127, 32, 0, 0, 0, 0])
+    np.testing.assert_array_equal(q[0], [64, 0, -127, 32, 0, 0, 0, 0])   # element 4 is the second NaN
     np.testing.assert_array_equal(q[1:], 0)
     assert pts[0] == np.float32(2.0) / np.float32(127.0)
     assert pts[1] == np.inf and pts[2] == np.inf and pts[3] == 0.0
@@ -473,3 +474,85 @@ def test_per_token_quant_bounds(oracle):
     np.testing.assert_array_equal(pts, (np.abs(xf).max(axis=1).astype(np.float32) / np.float32(127)))
     recon = q.astype(np.float64) * pts.astype(np.float64)[:, None]
     assert (np.abs(xf - recon) <= pts.astype(np.float64)[:, None] * 0.50002).all()
+
+
+# --- per-32-group FP8 E4M3 cast ----------------------------------------------
+def test_e4m3_codes_against_the_format_definition(oracle):
+    """E4M3FN: sign, 4 exponent bits with bias 7, 3 fraction bits, subnormals m * 2^-9
+    at exponent 0, S.1111.111 NaN, no infinities, largest finite 1.75 * 2^8 = 448.
+    Hand-known codes; every non-NaN code round-trips; the finite codes increase
+    strictly; each midpoint between neighbours rounds to the even code (the code's
+    last bit is the fraction's); and torch's float8_e4m3fn conversion (a library
+    routine, round to nearest even) agrees on random in-range values."""
+    known = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0, 0x3C: 1.5, 0x40: 2.0,
+             0x7E: 448.0, 0xB8: -1.0, 0xFE: -448.0}
+    for c, v in known.items():
+        assert oracle.e4m3_decode(c) == v and oracle.e4m3_encode(v) == c, hex(c)
+    assert np.isnan(oracle.e4m3_decode(0x7F)) and np.isnan(oracle.e4m3_decode(0xFF))
+    assert oracle.e4m3_encode(-0.0) == 0x80 and oracle.e4m3_encode(float("nan")) == 0x7F
+    finite = [c for c in range(256) if c & 0x7F != 0x7F]
+    for c in finite:
+        assert oracle.e4m3_encode(oracle.e4m3_decode(c)) == c, hex(c)
+    vals = [oracle.e4m3_decode(c) for c in range(0x7F)]
+    assert all(a < b for a, b in zip(vals, vals[1:]))
+    for c in range(0x7E):
+        mid = np.float32((vals[c] + vals[c + 1]) / 2)            # exact: one more fraction bit
+        assert oracle.e4m3_encode(float(mid)) == (c if c % 2 == 0 else c + 1), hex(c)
+    for v in (449.0, 463.9, 464.0, 1e6, float("inf")):           # saturation, not NaN
+        assert oracle.e4m3_encode(v) == 0x7E and oracle.e4m3_encode(-v) == 0xFE
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(11)
+    x = np.concatenate([rng.uniform(-448, 448, 4000), rng.standard_normal(4000) * 2.0 ** rng.integers(-12, 8, 4000),
+                        [(vals[c] + vals[c + 1]) / 2 for c in range(0x7E)]]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(float(v)) for v in x], np.uint8)
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_mxfp8_cast_hand_worked_groups(oracle):
+    """One row of four 32-element groups (reading: an E8M0 scale per group whose
+    exponent puts the group's largest magnitude in E4M3's top binade).
+      group 0: 1.0, -0.30078125, 0.5 -> amax 1 (f32 exponent 127), sf = 119, x * 2^8:
+               256 -> 0x78; -77 = -2^6 * 1.203 -> fraction 1.625/8 rounds to 2/8 -> -80 -> 0xEA;
+               128 -> 0x70
+      group 1: 3.0, 1.75, 0.00099945 -> amax 3 (exponent 128), sf = 120, x * 2^7:
+               384 = 1.5 * 2^8 -> 0x7C; 224 = 1.75 * 2^7 -> 0x76; 0.1279 = 1.023 * 2^-3 -> 0x20
+      group 2: 460 (exponent 135), sf = 127, x * 1 = 460 past 448 -> saturates to 0x7E
+      group 3: all zero -> sf = 0, codes 0"""
+    x = np.zeros((1, 128), np.uint16)
+    x[0, [0, 1, 2]] = [0x3F80, 0xBE9A, 0x3F00]
+    x[0, [32, 33, 34]] = [0x4040, 0x3FE0, 0x3A83]
+    x[0, 64] = 0x43E6                                            # 460 = 1.796875 * 2^8
+    q, sf = oracle.per_token_quant_mxfp8(x)
+    np.testing.assert_array_equal(sf[0], [119, 120, 127, 0])
+    np.testing.assert_array_equal(q[0, :3], [0x78, 0xEA, 0x70])
+    np.testing.assert_array_equal(q[0, 32:35], [0x7C, 0x76, 0x20])
+    assert q[0, 64] == 0x7E
+    assert (q[0, 3:32] == 0).all() and (q[0, 35:64] == 0).all() and (q[0, 65:] == 0).all()
+
+
+def test_mxfp8_cast_bounds_and_non_finite(oracle):
+    """Every group's largest magnitude lands in [256, 448] (E4M3's top binade, or the
+    saturated 448); |x - q * 2^(sf-127)| is at most half an E4M3 step (2^-4 of the
+    element's binade, 2^-9 on the subnormal grid) after scaling, except where the
+    top element saturated.  Non-finite inputs: NaN is skipped by the group's absmax
+    and encodes as 0x7F; an infinity makes sf = 247 (f32 exponent 255 - 8) and
+    saturates to 448 while the group's finite values scale to 0."""
+    from synth.inputs import bf16_bits_normal
+    x = bf16_bits_normal(np.random.default_rng(23), (16, 256))
+    q, sf = oracle.per_token_quant_mxfp8(x)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64).reshape(16, 8, 32)
+    dq = np.vectorize(oracle.e4m3_decode)(q).astype(np.float64).reshape(16, 8, 32)
+    scaled = xf * np.exp2(127.0 - sf.astype(np.float64))[:, :, None]
+    top = np.abs(dq).max(axis=2)
+    assert ((top >= 256) & (top <= 448)).all()
+    step = np.where(np.abs(scaled) < 2.0 ** -6, 2.0 ** -9, np.exp2(np.floor(np.log2(np.maximum(np.abs(scaled),
+                                                                                            1e-300))) - 3))
+    ok = (np.abs(scaled - dq) <= step / 2) | (np.abs(dq) == 448)
+    assert ok.all()
+    y = np.zeros((1, 64), np.uint16)
+    y[0, :4] = [0x7FC0, 0x3F80, 0xC000, 0x7FC0]                   # NaN, 1, -2, NaN (after the max too)
+    y[0, 32:34] = [0x7F80, 0x3F80]                                # +inf, 1
+    q, sf = oracle.per_token_quant_mxfp8(y)
+    assert sf[0, 0] == 120 and q[0, 0] == 0x7F and q[0, 1] == 0x70 and q[0, 2] == 0xF8 and q[0, 3] == 0x7F
+    assert sf[0, 1] == 247 and q[0, 32] == 0x7E and q[0, 33] == 0
