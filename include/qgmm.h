@@ -277,6 +277,27 @@ qgmm_status qgmm_per_token_quant(const uint16_t *x_bf16, int64_t rows, int64_t k
                                  float *scale_out, void *cuda_stream);
 
 /*
+ * Per-32-group FP8 cast (page 4, "PTOAS issue 1568", 背景: per_token_cast
+ * multiplies the bf16 values of a 256-element tile by inverse scale factors
+ * broadcast over groups of 32 and converts the products to FLOAT8 E4M3FN, with
+ * packed scale factors).  How a scale factor is chosen is not on the page; the
+ * library takes one E8M0 power of two per group of 32, which puts the group's
+ * largest magnitude in E4M3's top binade (the per-32 scale format that page 1's
+ * MxA8W4 mode reads):
+ *   a        = max_j |x[i][32g + j]| over the group (NaN skipped)
+ *   sf[i][g] = max(0, biased f32 exponent of a - 8)      (E8M0 code: 2^(sf - 127))
+ *   q[i][c]  = E4M3(x[i][c] * 2^(127 - sf[i][c/32])), round to nearest even,
+ *              magnitudes past 448 (infinities too) saturate to 448, NaN -> 0x7F
+ * so x ~= q * 2^(sf - 127); the product is exact, the conversion the only
+ * rounding.  x_bf16: bf16 bits [rows, k]; q_out: E4M3 bytes [rows, k]; sf_out:
+ * E8M0 bytes [rows, k/32] (four per 32-bit word: the packed layout).
+ * 1 <= rows <= 2^31-1, k % 32 == 0, 32 <= k <= 65536; x_bf16 16-byte and q_out
+ * 8-byte aligned.  Errors: NULL_PTR, SHAPE, ALIGNMENT, UNSUPPORTED, CUDA.
+ */
+qgmm_status qgmm_per_token_quant_mxfp8(const uint16_t *x_bf16, int64_t rows, int64_t k, uint8_t *q_out,
+                                       uint8_t *sf_out, void *cuda_stream);
+
+/*
  * Parity hook (no counterpart on the pages): the op's exact integer stage, so a
  * test can compare it bit for bit with an independent computation.
  * The raw int32 accumulators acc_out[i][j] = sum_kk x1[i][kk] * W(g, kk, j)

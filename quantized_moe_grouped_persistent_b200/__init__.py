@@ -50,8 +50,8 @@ QGMM_DEV_ROW_INDEX_RANGE = 1 << 3
 QGMM_DEV_TIMEOUT = 1 << 4
 
 EXPORTS = ("qgmm_finalize_workspace", "qgmm_finalize_launches", "qgmm_plan", "qgmm_finalize", "qgmm_finalize_profiled",
-           "qgmm_per_token_quant", "qgmm_debug_accum", "qgmm_device_status", "qgmm_finalize_static_scratch",
-           "qgmm_status_string")
+           "qgmm_per_token_quant", "qgmm_per_token_quant_mxfp8", "qgmm_debug_accum", "qgmm_device_status",
+           "qgmm_finalize_static_scratch", "qgmm_status_string")
 
 
 class QgmmProblem(C.Structure):
@@ -98,6 +98,7 @@ def lib():
         L.qgmm_finalize.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, P, P, P, P, P, P, U, P]
         L.qgmm_finalize_profiled.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, P, P, P, P, P, P, U, P, P, P]
         L.qgmm_per_token_quant.argtypes = [P, I64, I64, P, P, P]
+        L.qgmm_per_token_quant_mxfp8.argtypes = [P, I64, I64, P, P, P]
         L.qgmm_debug_accum.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, U, P]
         L.qgmm_device_status.argtypes = [P, C.POINTER(C.c_uint32), P]
         L.qgmm_finalize_static_scratch.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, P, P, P, P, P, P]
@@ -198,6 +199,15 @@ def per_token_quant(x_bf16, x1_out, scale_out, rows: Optional[int] = None, k: Op
         rows, k = x_bf16.shape
     rc = lib().qgmm_per_token_quant(_ptr(x_bf16), rows, k, _ptr(x1_out), _ptr(scale_out), _stream(stream))
     _check(rc, "qgmm_per_token_quant")
+
+
+def per_token_quant_mxfp8(x_bf16, q_out, sf_out, rows: Optional[int] = None, k: Optional[int] = None,
+                          stream=None) -> None:
+    """Per-32-group FP8 cast: E4M3 codes into ``q_out`` [rows, k], E8M0 scale codes into ``sf_out`` [rows, k/32]."""
+    if rows is None:
+        rows, k = x_bf16.shape
+    rc = lib().qgmm_per_token_quant_mxfp8(_ptr(x_bf16), rows, k, _ptr(q_out), _ptr(sf_out), _stream(stream))
+    _check(rc, "qgmm_per_token_quant_mxfp8")
 
 
 def debug_accum(problem: QgmmProblem, x1, x2, group_list, acc_out, workspace, ws_bytes: Optional[int] = None,

@@ -1403,4 +1403,63 @@ __global__ void per_token_quant_kernel(const uint16_t *__restrict__ x, int64_t r
     }
 }
 
+// ---------------------------------------------------------------- K0, FP8 form
+// Per-32-group FP8 E4M3 cast (page 4, per_token_cast: the bf16 values times the
+// group's broadcast inverse scale, converted to FLOAT8 E4M3FN).  Scale factors are
+// E8M0 codes, one per 32 elements:
+//   sf = max(0, biased f32 exponent of max|x| - 8),  inv = 2^(127 - sf)  (exact)
+//   q  = E4M3(x * inv), round to nearest even, saturating at 448; NaN -> 0x7F
+// x * inv is exact (a power of two), so the conversion is the only rounding.  One
+// thread takes 8 bf16 (16 bytes), four neighbouring lanes a group, a warp 256
+// elements of one row; k % 32 == 0.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    uint32_t v = r;
+    if (lo != lo) v = (v & 0xFF00u) | 0x7Fu;          // a NaN element codes as 0x7F
+    if (hi != hi) v = (v & 0x00FFu) | 0x7F00u;
+    return v;
+}
+
+__global__ void per_token_quant_mxfp8_kernel(const uint16_t *__restrict__ x, int64_t rows, int32_t k,
+                                             uint8_t *__restrict__ q, uint8_t *__restrict__ sf)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warps_total = int64_t(gridDim.x) * (blockDim.x >> 5);
+    const int32_t chunks_per_row = (k + 255) / 256;
+    const int64_t chunks = rows * chunks_per_row;
+    for (int64_t c = blockIdx.x * int64_t(blockDim.x >> 5) + (threadIdx.x >> 5); c < chunks; c += warps_total) {
+        const int64_t row = c / chunks_per_row;
+        const int32_t col = static_cast<int32_t>(c - row * chunks_per_row) * 256 + lane * 8;
+        const bool valid = col < k;                    // k % 32 == 0: a group is all valid or all not
+        uint4 h = make_uint4(0u, 0u, 0u, 0u);
+        if (valid) h = __ldg(reinterpret_cast<const uint4 *>(x + row * k + col));
+        const uint32_t w[4] = {h.x, h.y, h.z, h.w};
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            v[2 * u] = __uint_as_float(w[u] << 16);
+            v[2 * u + 1] = __uint_as_float(w[u] & 0xFFFF0000u);
+        }
+        float a = 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) a = fmaxf(a, fabsf(v[u]));   // fmaxf skips NaN
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+        const int biased = static_cast<int>((__float_as_uint(a) >> 23) & 0xFFu);
+        const int code = biased > 8 ? biased - 8 : 0;
+        const float inv = __uint_as_float(static_cast<uint32_t>(254 - code) << 23);
+        if (!valid) continue;
+        uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            lo |= e4m3x2(__fmul_rn(v[2 * u], inv), __fmul_rn(v[2 * u + 1], inv)) << (16 * u);
+            hi |= e4m3x2(__fmul_rn(v[4 + 2 * u], inv), __fmul_rn(v[5 + 2 * u], inv)) << (16 * u);
+        }
+        *reinterpret_cast<uint2 *>(q + row * k + col) = make_uint2(lo, hi);
+        if ((lane & 3) == 0) sf[row * (k / 32) + col / 32] = static_cast<uint8_t>(code);
+    }
+}
+
 }  // namespace qgmm

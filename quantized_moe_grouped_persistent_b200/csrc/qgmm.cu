@@ -627,6 +627,22 @@ QGMM_API qgmm_status qgmm_per_token_quant(const uint16_t *x_bf16, int64_t rows, 
     return cudaGetLastError() == cudaSuccess ? QGMM_OK : QGMM_ERR_CUDA;
 }
 
+QGMM_API qgmm_status qgmm_per_token_quant_mxfp8(const uint16_t *x_bf16, int64_t rows, int64_t k, uint8_t *q_out,
+                                                uint8_t *sf_out, void *cuda_stream)
+{
+    if (!x_bf16 || !q_out || !sf_out) return QGMM_ERR_NULL_PTR;
+    if (rows < 1 || rows > (int64_t(1) << 31) - 1 || k < 32 || k > 65536 || k % 32) return QGMM_ERR_SHAPE;
+    if (!aligned16(x_bf16) || (reinterpret_cast<uintptr_t>(q_out) & 7u)) return QGMM_ERR_ALIGNMENT;
+    DeviceInfo *dev = nullptr;
+    qgmm_status s = device_info(&dev);
+    if (s != QGMM_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    const int64_t chunks = rows * ((k + 255) / 256);
+    per_token_quant_mxfp8_kernel<<<grid_for(chunks, 8, dev->sms, 8), 256, 0, st>>>(
+        x_bf16, rows, static_cast<int32_t>(k), q_out, sf_out);
+    return cudaGetLastError() == cudaSuccess ? QGMM_OK : QGMM_ERR_CUDA;
+}
+
 QGMM_API qgmm_status qgmm_device_status(const void *workspace, uint32_t *flags, void *cuda_stream)
 {
     if (!workspace || !flags) return QGMM_ERR_NULL_PTR;

@@ -23,7 +23,8 @@ def _declared_functions():
 def test_header_declares_the_abi():
     assert _declared_functions() == sorted([
         "qgmm_finalize_workspace", "qgmm_finalize", "qgmm_finalize_profiled", "qgmm_per_token_quant",
-        "qgmm_debug_accum", "qgmm_device_status", "qgmm_finalize_static_scratch", "qgmm_status_string",
+        "qgmm_per_token_quant_mxfp8", "qgmm_debug_accum", "qgmm_device_status", "qgmm_finalize_static_scratch",
+        "qgmm_status_string",
         "qgmm_finalize_launches", "qgmm_plan"])
 
 

@@ -321,3 +321,25 @@ def test_per_token_quant_bit_exact(dev, oracle, qgmm):
     qs, ss = q.cpu().numpy(), s.cpu().numpy()
     assert qs[9, 3] == 0 and np.isfinite(ss[9]) and ss[9] > 0
     assert ss[10] == np.inf and ss[11] == np.inf and (qs[10:13] == 0).all() and ss[12] == 0
+
+
+def test_per_token_quant_mxfp8_bit_exact(dev, oracle, qgmm):
+    """Per-32-group FP8 cast: E4M3 codes and E8M0 scale codes bit for bit, on normal
+    rows, a k that is not a multiple of 256, and hand-made groups: zero, NaN, +-inf,
+    bf16 subnormals, a saturating top element, round-half-even ties."""
+    from synth.inputs import bf16_bits_normal
+    rng = np.random.default_rng(81)
+    for rows, k in ((300, 2048), (37, 96)):
+        x = bf16_bits_normal(rng, (rows, k))
+        x[1, :32] = 0                                             # zero group
+        x[2, 3], x[3, 40], x[4, 7], x[5, :32] = 0x7FC0, 0x7F80, 0xFF80, 0x7FC0
+        x[6, :32] = rng.integers(1, 0x80, 32, dtype=np.uint16)    # bf16 subnormals
+        x[7, 0] = 0x43E6                                          # 460: saturates
+        x[8, :4] = [0x3F80, 0x3D88, 0x3D98, 0xBD88]               # amax 1, times 2^8: ties 17 -> 16, 19 -> 20
+        xd = torch.from_numpy(x.view(np.int16)).cuda()
+        q = torch.empty((rows, k), dtype=torch.uint8, device="cuda")
+        sf = torch.empty((rows, k // 32), dtype=torch.uint8, device="cuda")
+        qgmm.per_token_quant_mxfp8(xd, q, sf)
+        rq, rsf = oracle.per_token_quant_mxfp8(x)
+        np.testing.assert_array_equal(sf.cpu().numpy(), rsf)
+        np.testing.assert_array_equal(q.cpu().numpy(), rq)
