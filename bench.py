@@ -105,7 +105,7 @@ def algorithmic_bytes(p):
     scale/bias rows), x1 (or the bf16 activations), the per-row vectors, the output
     written once, and the sharedInput read once."""
     used = int((p.counts > 0).sum())
-    w_bytes = p.k * p.n if p.weight == "int8" else p.k * p.n // 2
+    w_bytes = p.k * p.n // 2 if p.weight == "int4" else p.k * p.n
     per_expert = w_bytes + 4 * p.n + (4 * p.n if p.bias is not None else 0)
     b = used * per_expert
     m = total_rows(p)
@@ -325,6 +325,8 @@ def line_unit(workload, p):
     of the ops is credited the same fraction of the workload's algorithmic bytes)."""
     if workload == "decode":
         return "GB/s", 1e3 * algorithmic_bytes(p) / int_ops(p)
+    if p.weight == "fp8":
+        return "TFLOPS", 1.0
     return "TOPS", 1.0
 
 

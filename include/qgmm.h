@@ -16,7 +16,8 @@
  *
  * W(g, kk, j) is x2[g][kk][j] (int8, layout (e, k, n), n contiguous), or for
  * int4 weights the signed nibble j%8 (lowest nibble = lowest j) of the int32
- * word x2[g][kk][j/8] (layout (e, k, n/8)).  Every f32 step rounds to nearest
+ * word x2[g][kk][j/8] (layout (e, k, n/8)), or for E4M3 operands the value of
+ * the FLOAT8 E4M3FN byte x2[g][kk][j] (x1 is then E4M3 too).  Every f32 step rounds to nearest
  * even; nothing is fused into an FMA.  Where the pages leave the formula open
  * (bias position, unweighted sharedInput, nibble order, summation order) the
  * library takes the readings written above.
@@ -61,7 +62,9 @@ typedef enum {
     QGMM_ERR_SCRATCH_LIMIT = 9        /* qgmm_finalize_static_scratch: scratch above its cap  */
 } qgmm_status;
 
-enum { QGMM_W_INT8 = 0, QGMM_W_INT4_PACKED_INT32 = 1 };   /* x2: (e,k,n) int8 | (e,k,n/8) int32 */
+/* x2 (and x1) element type: int8 x2 (e,k,n) | int4 packed in int32 (e,k,n/8) |
+ * FLOAT8 E4M3FN x1 and x2 (e,k,n), page 1's Atlas 350 per-token / per-channel mode */
+enum { QGMM_W_INT8 = 0, QGMM_W_INT4_PACKED_INT32 = 1, QGMM_W_FP8_E4M3 = 2 };
 enum { QGMM_IDX_INT64 = 0, QGMM_IDX_INT32 = 1 };          /* row_index element type             */
 enum { QGMM_GROUP_CUMSUM = 0, QGMM_GROUP_COUNTS = 1 };    /* group_list meaning                 */
 enum { QGMM_SCALE_F32 = 0, QGMM_SCALE_BF16 = 1 };         /* scale element type                 */
@@ -80,7 +83,12 @@ enum { QGMM_SCALE_F32 = 0, QGMM_SCALE_BF16 = 1 };         /* scale element type 
  *   n       output columns, 256 <= n <= 65536, n % 256 == 0 (page 1 fixes n = 7168)
  *   e       experts, 1 <= e <= 1024 (page 1: [1, 256] on A2/A3, [1, 1024] on Atlas 350)
  *   output_bs   rows of out, >= 1
- *   weight_type     QGMM_W_INT8 | QGMM_W_INT4_PACKED_INT32
+ *   weight_type     QGMM_W_INT8 | QGMM_W_INT4_PACKED_INT32 | QGMM_W_FP8_E4M3.  With
+ *                   QGMM_W_FP8_E4M3 both x1 and x2 hold FLOAT8 E4M3FN bytes (page 1,
+ *                   Atlas 350: x1 and x2 FLOAT8_E4M3FN with a per-channel scale and a
+ *                   per-token pertokenScale); acc is then the tensor core's f32 sum
+ *                   of the E4M3 products (not exact: rounded once per K = 32 step
+ *                   at most), and the dequant below starts from that f32 value.
  *   group_list_type QGMM_GROUP_CUMSUM (0) | QGMM_GROUP_COUNTS (1)
  *   row_index_type  QGMM_IDX_INT64 | QGMM_IDX_INT32
  *   shared_bs, shared_offset   sharedInput rows and where they land;
@@ -101,8 +109,8 @@ enum { QGMM_SCALE_F32 = 0, QGMM_SCALE_BF16 = 1 };         /* scale element type 
  *   transpose_x2    0: int8 x2 is (e, k, n); 1: int8 x2 is (e, n, k) (page 1,
  *                   full-quant scenario: x2 may be transposed, (e, n, k), on
  *                   Atlas 350; A2/A3 take only the non-transposed layout).
- *                   Same result either way.  int4 weights must be
- *                   non-transposed (QGMM_ERR_UNSUPPORTED otherwise).
+ *                   Same result either way (int8 and E4M3).  int4 weights must
+ *                   be non-transposed (QGMM_ERR_UNSUPPORTED otherwise).
  *   ld_x2, ld_sb, ld_out, ld_shared   row strides, 0 = n (no counterpart on the pages).
  *                   They let a call work on a block of n columns inside wider
  *                   tensors -- the column split across GPUs, where each GPU
@@ -300,7 +308,8 @@ qgmm_status qgmm_per_token_quant_mxfp8(const uint16_t *x_bf16, int64_t rows, int
 /*
  * Parity hook (no counterpart on the pages): the op's exact integer stage, so a
  * test can compare it bit for bit with an independent computation.
- * The raw int32 accumulators acc_out[i][j] = sum_kk x1[i][kk] * W(g, kk, j)
+ * The raw accumulators acc_out[i][j] = sum_kk x1[i][kk] * W(g, kk, j) -- int32, or
+ * for QGMM_W_FP8_E4M3 the f32 accumulator's bits in the same 4-byte slots --
  * for every row i below the groups' total, written by the same grouped GEMM
  * that qgmm_finalize runs (no epilogue arithmetic, no combine).  Rows at or
  * past the total are not written.  acc_out: int32 [m, n], 16-byte aligned.

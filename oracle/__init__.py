@@ -49,6 +49,8 @@ def lib():
         L.qo_per_token_quant.argtypes = [P, I64, I64, P, P]
         L.qo_bf16_to_f32.argtypes = [P, I64, P]
         L.qo_per_token_quant_mxfp8.argtypes = [P, I64, I64, P, P]
+        L.qo_accum_f8.argtypes = [P, P, I64, I64, I64, I64, P, I32, P, I64, P, P, I32]
+        L.qo_accum_f8.restype = C.c_int
         for f in (L.qo_group_offsets, L.qo_accum, L.qo_finalize, L.qo_per_token_quant, L.qo_bf16_to_f32,
                   L.qo_per_token_quant_mxfp8):
             f.restype = C.c_int
@@ -82,10 +84,12 @@ def group_offsets(group_list: np.ndarray, group_list_type: int, m: int) -> np.nd
 
 
 def _weights(x2: np.ndarray, weight: str, transpose_x2: bool = False):
-    """The C oracle's weight layout, (e, k, n) int8 or (e, k, n/8) int32.  A transposed
-    int8 x2 (page 1, full-quant scenario: (e, n, k)) is swapped back to it."""
+    """The C oracle's weight layout, (e, k, n) int8 / E4M3 bytes or (e, k, n/8) int32.
+    A transposed x2 (page 1, full-quant scenario: (e, n, k)) is swapped back to it."""
     if weight == "int8":
         return _c(np.swapaxes(x2, 1, 2) if transpose_x2 else x2, np.int8), 0
+    if weight == "fp8":
+        return _c(np.swapaxes(x2, 1, 2) if transpose_x2 else x2, np.uint8), 2
     if transpose_x2:
         raise ValueError("transposed x2 is int8 only")
     return _c(x2, np.int32), 1
@@ -94,7 +98,11 @@ def _weights(x2: np.ndarray, weight: str, transpose_x2: bool = False):
 def accum(x1, x2, group_list, group_list_type: int, weight: str = "int8",
           rows: Optional[np.ndarray] = None, threads: Optional[int] = None,
           transpose_x2: bool = False) -> np.ndarray:
-    """Exact int32 accumulators ``x1[i] @ W[g(i)]`` for source rows ``rows`` (default all)."""
+    """Exact int32 accumulators ``x1[i] @ W[g(i)]`` for source rows ``rows`` (default all).
+    FP8 (E4M3 bytes): use ``accum_f8``."""
+    if weight == "fp8":
+        return accum_f8(x1, x2, group_list, group_list_type, rows=rows, threads=threads,
+                        transpose_x2=transpose_x2)[0]
     x1 = _c(x1, np.int8)
     w, wt = _weights(x2, weight, transpose_x2)
     m, k = x1.shape
@@ -108,6 +116,25 @@ def accum(x1, x2, group_list, group_list_type: int, weight: str = "int8",
     if rc:
         raise OracleError(rc, "accum")
     return out
+
+
+def accum_f8(x1, x2, group_list, group_list_type: int, rows: Optional[np.ndarray] = None,
+             threads: Optional[int] = None, transpose_x2: bool = False):
+    """E4M3 operands (uint8 codes): exact double accumulators and the sums of
+    |products| for source rows ``rows`` (default all)."""
+    x1 = _c(x1, np.uint8)
+    w, _ = _weights(x2, "fp8", transpose_x2)
+    m, k = x1.shape
+    e, n = w.shape[0], w.shape[2]
+    r = _c(rows, np.int64)
+    nrows = m if r is None else r.shape[0]
+    acc = np.zeros((nrows, n), np.float64)
+    mag = np.zeros((nrows, n), np.float64)
+    rc = lib().qo_accum_f8(_ptr(x1), _ptr(w), m, k, n, e, _ptr(_c(group_list, np.int64)), group_list_type,
+                           _ptr(r), nrows, _ptr(acc), _ptr(mag), threads or default_threads())
+    if rc:
+        raise OracleError(rc, "accum_f8")
+    return acc, mag
 
 
 def finalize(x1, x2, group_list, group_list_type: int, *, weight: str = "int8",
@@ -126,11 +153,11 @@ def finalize(x1, x2, group_list, group_list_type: int, *, weight: str = "int8",
     """
     if scale is not None and scale.dtype == np.uint16:
         scale = bf16_to_f32(scale)
-    x1 = _c(x1, np.int8)
+    x1 = _c(x1, np.uint8 if weight == "fp8" else np.int8)
     w, wt = _weights(x2, weight, transpose_x2)
     m, k = x1.shape
     e = w.shape[0]
-    n = w.shape[2] * (8 if wt else 1)
+    n = w.shape[2] * (8 if wt == 1 else 1)
     if output_bs is None:
         output_bs = m
     ri = None

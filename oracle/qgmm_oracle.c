@@ -51,6 +51,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+float qo_e4m3_decode(uint8_t c);
+
 enum {
     QO_OK = 0,
     QO_ERR_NEGATIVE_COUNT = 1,
@@ -105,6 +107,28 @@ static int64_t group_of_row(const int64_t *off, int64_t e, int64_t i)
     return -1;
 }
 
+/* FLOAT8 E4M3 operands (weight_type 2, page 1: x1 and x2 both FLOAT8_E4M3FN in the
+ * Atlas 350 per-token / per-channel mode): acc[j] = sum_kk x1[i][kk] * x2[g][kk][j]
+ * over the values the codes stand for, in double.  Exact: every product of two
+ * E4M3 values is a multiple of 2^-18 below 2^18, so a sum of at most 65536 of them
+ * needs under 53 significant bits.  mag[j] = sum_kk |x1[i][kk] * x2[g][kk][j]|. */
+static void accum_row_f8(const int8_t *x1, const void *x2, int64_t k, int64_t n, int64_t g, int64_t i,
+                         double *acc, double *mag)
+{
+    const uint8_t *a = (const uint8_t *)x1 + i * k;
+    for (int64_t j = 0; j < n; ++j) acc[j] = mag[j] = 0.0;
+    for (int64_t kk = 0; kk < k; ++kk) {
+        double av = (double)qo_e4m3_decode(a[kk]);
+        if (av == 0.0) continue;
+        const uint8_t *wrow = (const uint8_t *)x2 + (g * k + kk) * n;
+        for (int64_t j = 0; j < n; ++j) {
+            double p = av * (double)qo_e4m3_decode(wrow[j]);
+            acc[j] += p;
+            mag[j] += fabs(p);
+        }
+    }
+}
+
 /* acc[j] = sum_kk x1[i][kk] * W(g, kk, j), exact; returns 0 or overflow code */
 static int accum_row(const int8_t *x1, const void *x2, int weight_type, int64_t k, int64_t n,
                      int64_t g, int64_t i, int64_t *acc64 /* [n] scratch */, int32_t *acc)
@@ -130,7 +154,7 @@ static int accum_row(const int8_t *x1, const void *x2, int weight_type, int64_t 
 
 /* ---- parallel-for over a list of items ---------------------------------- */
 typedef struct {
-    void (*fn)(void *ctx, int64_t item, int64_t *s64, int32_t *s32, int *rc);
+    void (*fn)(void *ctx, int64_t item, int64_t *s64, int32_t *s32, double *sd, int *rc);
     void *ctx;
     int64_t nitems, n;
     int nthreads, tid;
@@ -142,14 +166,16 @@ static void *job_main(void *p)
     job_t *j = (job_t *)p;
     int64_t *s64 = (int64_t *)malloc(sizeof(int64_t) * (size_t)j->n);
     int32_t *s32 = (int32_t *)malloc(sizeof(int32_t) * (size_t)j->n);
-    if (!s64 || !s32) { j->rc = QO_ERR_ARG; free(s64); free(s32); return NULL; }
-    for (int64_t it = j->tid; it < j->nitems; it += j->nthreads) j->fn(j->ctx, it, s64, s32, &j->rc);
+    double *sd = (double *)malloc(sizeof(double) * 2 * (size_t)j->n);
+    if (!s64 || !s32 || !sd) { j->rc = QO_ERR_ARG; free(s64); free(s32); free(sd); return NULL; }
+    for (int64_t it = j->tid; it < j->nitems; it += j->nthreads) j->fn(j->ctx, it, s64, s32, sd, &j->rc);
     free(s64);
     free(s32);
+    free(sd);
     return NULL;
 }
 
-static int run_parallel(void (*fn)(void *, int64_t, int64_t *, int32_t *, int *), void *ctx,
+static int run_parallel(void (*fn)(void *, int64_t, int64_t *, int32_t *, double *, int *), void *ctx,
                         int64_t nitems, int64_t n, int nthreads)
 {
     if (nthreads < 1) nthreads = 1;
@@ -174,10 +200,11 @@ typedef struct {
     const int64_t *off; const int64_t *rows; int32_t *acc_out;
 } accum_ctx;
 
-static void accum_item(void *p, int64_t it, int64_t *s64, int32_t *s32, int *rc)
+static void accum_item(void *p, int64_t it, int64_t *s64, int32_t *s32, double *sd, int *rc)
 {
     accum_ctx *c = (accum_ctx *)p;
     (void)s32;
+    (void)sd;
     int64_t i = c->rows ? c->rows[it] : it;
     int32_t *dst = c->acc_out + it * c->n;
     int64_t g = group_of_row(c->off, c->e, i);
@@ -199,6 +226,45 @@ int qo_accum(const int8_t *x1, const void *x2, int weight_type, int64_t m, int64
     if (rc == QO_OK) {
         accum_ctx c = {x1, x2, weight_type, k, n, e, off, rows, acc_out};
         rc = run_parallel(accum_item, &c, nrows, n, nthreads);
+    }
+    free(off);
+    return rc;
+}
+
+/* FP8 accumulators acc_out[r][j] (double, exact) and mag_out[r][j] (sum of
+ * |products|, may be NULL) for source rows rows[0..nrows); rows past the total
+ * come back as zeros. */
+typedef struct {
+    const int8_t *x1; const void *x2; int64_t k, n, e;
+    const int64_t *off; const int64_t *rows; double *acc_out, *mag_out;
+} accum_f8_ctx;
+
+static void accum_f8_item(void *p, int64_t it, int64_t *s64, int32_t *s32, double *sd, int *rc)
+{
+    accum_f8_ctx *c = (accum_f8_ctx *)p;
+    (void)s64; (void)s32; (void)rc;
+    int64_t i = c->rows ? c->rows[it] : it;
+    double *dst = c->acc_out + it * c->n;
+    double *mag = c->mag_out ? c->mag_out + it * c->n : sd + c->n;
+    int64_t g = group_of_row(c->off, c->e, i);
+    if (g < 0) {
+        for (int64_t j = 0; j < c->n; ++j) dst[j] = mag[j] = 0.0;
+        return;
+    }
+    accum_row_f8(c->x1, c->x2, c->k, c->n, g, i, dst, mag);
+}
+
+int qo_accum_f8(const int8_t *x1, const void *x2, int64_t m, int64_t k, int64_t n, int64_t e,
+                const int64_t *group_list, int group_list_type, const int64_t *rows, int64_t nrows,
+                double *acc_out, double *mag_out, int nthreads)
+{
+    if (!x1 || !x2 || !acc_out || k < 1 || n < 1) return QO_ERR_ARG;
+    int64_t *off = (int64_t *)malloc(sizeof(int64_t) * (size_t)(e + 1));
+    if (!off) return QO_ERR_ARG;
+    int rc = qo_group_offsets(group_list, e, group_list_type, m, off);
+    if (rc == QO_OK) {
+        accum_f8_ctx c = {x1, x2, k, n, e, off, rows, acc_out, mag_out};
+        rc = run_parallel(accum_f8_item, &c, nrows, n, nthreads);
     }
     free(off);
     return rc;
@@ -230,7 +296,7 @@ static inline int64_t dest_of(const fin_ctx *c, int64_t i)
     return (int64_t)((const int32_t *)c->row_index)[i];
 }
 
-static void fin_item(void *p, int64_t it, int64_t *s64, int32_t *acc, int *rc)
+static void fin_item(void *p, int64_t it, int64_t *s64, int32_t *acc, double *sd, int *rc)
 {
     fin_ctx *c = (fin_ctx *)p;
     const int64_t n = c->n;
@@ -253,22 +319,31 @@ static void fin_item(void *p, int64_t it, int64_t *s64, int32_t *acc, int *rc)
         if (d < 0 || d >= c->output_bs) { *rc = QO_ERR_BAD_ROW_INDEX; continue; }
         if (d != r) continue;
         int64_t g = group_of_row(c->off, c->e, i);
-        int ar = accum_row(c->x1, c->x2, c->weight_type, c->k, n, g, i, s64, acc);
-        if (ar != QO_OK) *rc = ar;
+        const int f8 = c->weight_type == 2;
+        double *accd = sd, *mag = sd + n;       /* FP8: exact sums and sums of |products| */
+        if (f8) {
+            accum_row_f8(c->x1, c->x2, c->k, n, g, i, accd, mag);
+        } else {
+            int ar = accum_row(c->x1, c->x2, c->weight_type, c->k, n, g, i, s64, acc);
+            if (ar != QO_OK) *rc = ar;
+        }
         const float pts = c->pts ? c->pts[i] : 1.0f;
         const float lg = c->logit ? c->logit[i] : 1.0f;
         for (int64_t j = 0; j < n; ++j) {
             const float sc = c->scale ? c->scale[g * n + j] : 1.0f;
             const float bs = c->bias ? c->bias[g * n + j] : 0.0f;
+            const double av = f8 ? accd[j] : (double)acc[j];
             if (o64 || a64) {
-                double y = (((double)acc[j] * (double)sc) * (double)pts + (double)bs) * (double)lg;
+                double y = ((av * (double)sc) * (double)pts + (double)bs) * (double)lg;
                 if (o64) o64[j] += y;
                 /* the rounding of (acc*scale*pts + bias)*logit in any f32 order is bounded by a
-                   few ulp of the summands' magnitudes, taken before the bias can cancel */
-                if (a64) a64[j] += (fabs((double)acc[j] * (double)sc * (double)pts) + fabs((double)bs)) * fabs((double)lg);
+                   few ulp of the summands' magnitudes, taken before the bias can cancel; for FP8
+                   operands the accumulation itself rounds, so its terms are sum |products| */
+                const double am = f8 ? mag[j] : fabs(av);
+                if (a64) a64[j] += (am * fabs((double)sc * (double)pts) + fabs((double)bs)) * fabs((double)lg);
             }
             if (o32) {
-                float y = (float)acc[j];        /* round to nearest even */
+                float y = (float)av;            /* round to nearest even (FP8: of the exact sum) */
                 y = y * sc;
                 y = y * pts;
                 y = y + bs;
@@ -295,7 +370,9 @@ int qo_finalize(const int8_t *x1, const void *x2, int weight_type, int64_t m, in
                 const int64_t *dest_rows, int64_t ndest,
                 double *out64, double *sabs64, float *out32, int nthreads)
 {
-    if (!x1 || !x2 || k < 1 || n < 1 || output_bs < 1 || (weight_type == 1 && n % 8)) return QO_ERR_ARG;
+    if (!x1 || !x2 || k < 1 || n < 1 || output_bs < 1 || (weight_type == 1 && n % 8) || weight_type < 0 ||
+        weight_type > 2)
+        return QO_ERR_ARG;
     if (shared && (shared_offset < 0 || shared_offset + shared_bs > output_bs)) return QO_ERR_ARG;
     int64_t *off = (int64_t *)malloc(sizeof(int64_t) * (size_t)(e + 1));
     if (!off) return QO_ERR_ARG;

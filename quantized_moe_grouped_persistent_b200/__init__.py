@@ -36,6 +36,7 @@ QGMM_STATIC_SCRATCH_BYTES = 16 << 20
 
 QGMM_W_INT8 = 0
 QGMM_W_INT4_PACKED_INT32 = 1
+QGMM_W_FP8_E4M3 = 2
 QGMM_IDX_INT64 = 0
 QGMM_IDX_INT32 = 1
 QGMM_GROUP_CUMSUM = 0

@@ -263,7 +263,8 @@ constexpr int NCHUNK = BN / 32;   // 32-column chunks per accumulator
 // Thread = accumulator row: write its 32 values of one chunk into the warp's
 // staging rows (f32 of the int32 value, or its raw bits for the debug output).
 // SHIFT undoes the int4 path's x16 operand scale (arithmetic shift, exact).
-template <int EPI, int SHIFT>
+// FACC: the accumulator already is f32 (E4M3 operands); its bits pass through.
+template <int EPI, int SHIFT, bool FACC = false>
 __device__ __forceinline__ void epi_stage_chunk(float *stage, int lane, const uint32_t (&r)[32])
 {
     float *srow = stage + lane * EPI_LD;
@@ -273,7 +274,7 @@ __device__ __forceinline__ void epi_stage_chunk(float *stage, int lane, const ui
 #pragma unroll
         for (int u = 0; u < 4; ++u) a[u] = static_cast<int>(r[4 * v + u]) >> SHIFT;
         float4 f;
-        if constexpr (EPI == EPI_RAW_ACC) {
+        if constexpr (EPI == EPI_RAW_ACC || FACC) {
             f = make_float4(__int_as_float(a[0]), __int_as_float(a[1]), __int_as_float(a[2]), __int_as_float(a[3]));
         } else {
             f = make_float4(__int2float_rn(a[0]), __int2float_rn(a[1]), __int2float_rn(a[2]), __int2float_rn(a[3]));
@@ -345,7 +346,7 @@ __device__ __forceinline__ EpiSmem epi_smem(float *epi_stage, float *row_pts, fl
 // accumulator, and TMEM chunk k+1 is loaded while chunk k is written out.
 // SHIFT: W4_ACC_SHIFT for int4 weights, else 0.  Returns false if the wait for
 // the accumulator ran out.
-template <int EPI, int NCH, int SHIFT>
+template <int EPI, int NCH, int SHIFT, bool FACC = false>
 __device__ __forceinline__ bool epilogue_tile(const GemmArgs &args, const TileCoord &c, int64_t row_base,
                                               int rows_here, int row_off, uint32_t tmem_acc, int q, int tmem_col,
                                               int glob_col, int lane, uint64_t *tfull_bar, uint32_t use,
@@ -402,13 +403,13 @@ __device__ __forceinline__ bool epilogue_tile(const GemmArgs &args, const TileCo
 #pragma unroll
         for (int pc = 0; pc < NCH; pc += 2) {
             ptx::tmem_ld_wait(ra);
-            epi_stage_chunk<EPI, SHIFT>(sm.stage, lane, ra);
+            epi_stage_chunk<EPI, SHIFT, FACC>(sm.stage, lane, ra);
             ptx::tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>((pc + 1) * 32), rb);
             __syncwarp();
             epi_write_chunk<EPI>(args, sm.stage, sm.rp, sm.rl, sm.rd, sub, col4, ldd, n0 + pc * 32, sc[pc], bs[pc]);
             __syncwarp();
             ptx::tmem_ld_wait(rb);
-            epi_stage_chunk<EPI, SHIFT>(sm.stage, lane, rb);
+            epi_stage_chunk<EPI, SHIFT, FACC>(sm.stage, lane, rb);
             if (pc + 2 < NCH) ptx::tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>((pc + 2) * 32), ra);
             __syncwarp();
             epi_write_chunk<EPI>(args, sm.stage, sm.rp, sm.rl, sm.rd, sub, col4, ldd, n0 + (pc + 1) * 32, sc[pc + 1],
@@ -433,7 +434,7 @@ __device__ __forceinline__ bool epilogue_tile(const GemmArgs &args, const TileCo
 constexpr int EPI_COLS = 128;
 constexpr int EPI_CHUNKS = EPI_COLS / 64;
 
-template <int EPI>
+template <int EPI, bool FACC>
 __device__ __forceinline__ void epi_direct_rows(const GemmArgs &args, const uint32_t (&v)[32], long long dA,
                                                 long long dB, float pA, float pB, float lA, float lB,
                                                 const float2 (&sc)[8], const float2 (&bs)[8], int64_t ldd, int64_t col0)
@@ -451,10 +452,10 @@ __device__ __forceinline__ void epi_direct_rows(const GemmArgs &args, const uint
                     make_int2(static_cast<int>(u0), static_cast<int>(u1));
             } else {
                 const float p = h ? pB : pA, l = h ? lB : lA;
-                const float y0 = __fmul_rn(
-                    __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(u0)), sc[j].x), p), bs[j].x), l);
-                const float y1 = __fmul_rn(
-                    __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(u1)), sc[j].y), p), bs[j].y), l);
+                const float a0 = FACC ? __uint_as_float(u0) : __int2float_rn(static_cast<int>(u0));
+                const float a1 = FACC ? __uint_as_float(u1) : __int2float_rn(static_cast<int>(u1));
+                const float y0 = __fmul_rn(__fadd_rn(__fmul_rn(__fmul_rn(a0, sc[j].x), p), bs[j].x), l);
+                const float y1 = __fmul_rn(__fadd_rn(__fmul_rn(__fmul_rn(a1, sc[j].y), p), bs[j].y), l);
                 if constexpr (EPI == EPI_ATOMIC) {
                     ptx::red_add_v2(args.out + d * ldd + col, y0, y1);
                 } else {
@@ -465,7 +466,7 @@ __device__ __forceinline__ void epi_direct_rows(const GemmArgs &args, const uint
     }
 }
 
-template <int EPI>
+template <int EPI, bool FACC>
 __device__ __forceinline__ bool epilogue_tile_direct(const GemmArgs &args, const TileCoord &c, int64_t row_base,
                                                      int rows_here, uint32_t tmem_acc, int q, int col_begin, int lane,
                                                      uint64_t *tfull_bar, uint32_t use, volatile int *abort_flag)
@@ -533,9 +534,9 @@ __device__ __forceinline__ bool epilogue_tile_direct(const GemmArgs &args, const
             ptx::tmem_ld_16x256b_x8(col + (static_cast<uint32_t>(q * 32) << 16), va);
             ptx::tmem_ld_16x256b_x8(col + (static_cast<uint32_t>(q * 32 + 16) << 16), vb);
             ptx::tmem_ld_wait2(va, vb);
-            epi_direct_rows<EPI>(args, va, dst[0], dst[1], pts[0], pts[1], lg[0], lg[1], sc[ch], bs[ch], ldd,
+            epi_direct_rows<EPI, FACC>(args, va, dst[0], dst[1], pts[0], pts[1], lg[0], lg[1], sc[ch], bs[ch], ldd,
                                  n0 + 64 * ch);
-            epi_direct_rows<EPI>(args, vb, dst[2], dst[3], pts[2], pts[3], lg[2], lg[3], sc[ch], bs[ch], ldd,
+            epi_direct_rows<EPI, FACC>(args, vb, dst[2], dst[3], pts[2], pts[3], lg[2], lg[3], sc[ch], bs[ch], ldd,
                                  n0 + 64 * ch);
         }
     }
@@ -545,7 +546,9 @@ __device__ __forceinline__ bool epilogue_tile_direct(const GemmArgs &args, const
 }
 
 // ---------------------------------------------------------------- K2
-template <int EPI, bool W4>
+// F8: E4M3 operands (tcgen05.mma kind::f8f6f4, f32 accumulators); same tiles and
+// shared-memory layout as int8, one byte per element and K = 32 per instruction.
+template <int EPI, bool W4, bool F8 = false>
 __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                         const GemmArgs args)
@@ -684,7 +687,7 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
         if (lane == 0) {
             // int4 tiles are always unpacked MN-major; int8 (e, n, k) weights land K-major
             const bool bk = !W4 && args.b_kmajor != 0;
-            const uint32_t idesc = ptx::idesc_i8(BM, BN, !bk);
+            const uint32_t idesc = F8 ? ptx::idesc_e4m3(BM, BN, !bk) : ptx::idesc_i8(BM, BN, !bk);
             const uint32_t b_kstep = bk ? UMMA_K : UMMA_K * 128, b_lbo = bk ? 16 : B_ATOM_BYTES;
             int stage = 0;
             uint32_t phase = 0;
@@ -715,7 +718,10 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
                         // B: MN-major, 128-column atoms B_ATOM_BYTES apart, 8-row K groups 1024 B
                         // apart; or K-major like A, 8-row n groups 1024 B apart
                         const uint64_t bdesc = ptx::smem_desc_sw128(b0 + kk * b_kstep, b_lbo, 1024);
-                        ptx::mma_i8(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        if constexpr (F8)
+                            ptx::mma_e4m3(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        else
+                            ptx::mma_i8(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     ptx::mma_commit(&empty[stage]);
                     if (++stage == S) {
@@ -741,7 +747,7 @@ __global__ void __launch_bounds__(GemmCfg<W4>::THREADS, 1)
             const TileCoord c = tile_coord(t, MT, SW, off, cum, e, tile_rows, args.sched);
             const int buf = lt & 1;
             const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
-            if (!epilogue_tile_direct<EPI>(args, c, c.row0, tile_rows, tmem_base + static_cast<uint32_t>(buf * BN), q,
+            if (!epilogue_tile_direct<EPI, F8>(args, c, c.row0, tile_rows, tmem_base + static_cast<uint32_t>(buf * BN), q,
                                            col_begin, lane, &tfull[buf], use, abort_flag)) {
                 fail();
                 break;
@@ -860,7 +866,7 @@ struct PairCfg {
     static_assert(SMEM_BYTES <= 232448, "shared memory above the sm_100 per-block limit");
 };
 
-template <int EPI, bool W4>
+template <int EPI, bool W4, bool F8 = false>
 __global__ void __launch_bounds__(PairCfg<W4>::THREADS, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                              const GemmArgs args)
@@ -999,8 +1005,10 @@ __global__ void __launch_bounds__(PairCfg<W4>::THREADS, 1)
         // ------------------------------------------------ MMA issuer (leader CTA only)
         if (lane == 0 && leader) {
             const bool bk = args.b_kmajor != 0;
-            const uint32_t IDESC_FULL = ptx::idesc_i8(2 * BM, BN, !bk);   // 256 rows: 128 per CTA
-            const uint32_t IDESC_TAIL = ptx::idesc_i8(BM, BN, !bk);       // 128 rows: 64 per CTA
+            const uint32_t IDESC_FULL = F8 ? ptx::idesc_e4m3(2 * BM, BN, !bk)   // 256 rows: 128 per CTA
+                                           : ptx::idesc_i8(2 * BM, BN, !bk);
+            const uint32_t IDESC_TAIL = F8 ? ptx::idesc_e4m3(BM, BN, !bk)       // 128 rows: 64 per CTA
+                                           : ptx::idesc_i8(BM, BN, !bk);
             const uint32_t b_kstep = bk ? UMMA_K : UMMA_K * 128, b_lbo = bk ? 16 : B_ATOM_BYTES;
             int stage = 0;
             uint32_t phase = 0;
@@ -1031,7 +1039,10 @@ __global__ void __launch_bounds__(PairCfg<W4>::THREADS, 1)
                     for (int kk = 0; kk < BK / UMMA_K; ++kk) {
                         const uint64_t adesc = ptx::smem_desc_sw128(a0 + kk * UMMA_K, 16, 1024);
                         const uint64_t bdesc = ptx::smem_desc_sw128(b0 + kk * b_kstep, b_lbo, 1024);
-                        ptx::mma_i8_pair(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                        if constexpr (F8)
+                            ptx::mma_e4m3_pair(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                        else
+                            ptx::mma_i8_pair(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
                     }
                     ptx::mma_commit_pair(ptx::map_to_rank(&empty[stage], 0));
                     ptx::mma_commit_pair(ptx::map_to_rank(&empty[stage], 1));
@@ -1072,11 +1083,11 @@ __global__ void __launch_bounds__(PairCfg<W4>::THREADS, 1)
             if (c.tail) {
                 // M=128 pair tile: this CTA's 64 rows; TMEM lanes 0-63 hold columns 0-127,
                 // lanes 64-127 hold columns 128-255, in the buffer's first 128 columns.
-                ok = epilogue_tile<EPI, 4, SHIFT>(args, c, base_tail, 64, 32 * (q & 1), acc, q, 0, (q >> 1) * 128,
-                                                  lane, &tfull[buf], use, abort_flag, sm);
+                ok = epilogue_tile<EPI, 4, SHIFT, F8>(args, c, base_tail, 64, 32 * (q & 1), acc, q, 0, (q >> 1) * 128,
+                                                      lane, &tfull[buf], use, abort_flag, sm);
             } else {
-                ok = epilogue_tile<EPI, NCHUNK, SHIFT>(args, c, base_full, 128, q * 32, acc, q, 0, 0, lane,
-                                                       &tfull[buf], use, abort_flag, sm);
+                ok = epilogue_tile<EPI, NCHUNK, SHIFT, F8>(args, c, base_full, 128, q * 32, acc, q, 0, 0, lane,
+                                                           &tfull[buf], use, abort_flag, sm);
             }
             if (!ok) {
                 fail();

@@ -322,6 +322,31 @@ __host__ __device__ constexpr uint32_t idesc_i8(int M, int N, bool b_mn_major)
            | (static_cast<uint32_t>(M >> 4) << 24);  // M / 16
 }
 
+// Instruction descriptor for kind::f8f6f4 with E4M3 A and B: f32 accumulator,
+// A K-major, B K-major or MN-major, shape M x N.  (A/B format code 0 is E4M3.)
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool b_mn_major)
+{
+    return (1u << 4)                                 // D format: F32
+           | (0u << 7)                               // A: E4M3
+           | (0u << 10)                              // B: E4M3
+           | (0u << 15)                              // A K-major
+           | ((b_mn_major ? 1u : 0u) << 16)          // B major
+           | (static_cast<uint32_t>(N >> 3) << 17)   // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24);  // M / 16
+}
+
+// D[tmem] (+)= A * B, E4M3 x E4M3 -> f32, one CTA (K = 32 per instruction, as kind::i8).
+__device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // ---------------------------------------------------------------- CTA pairs (cluster of 2, cta_group::2)
 __device__ __forceinline__ uint32_t cluster_ctarank()
 {
@@ -413,6 +438,18 @@ __device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, ui
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Pair form of mma_e4m3 (leader CTA only).
+__device__ __forceinline__ void mma_e4m3_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }

@@ -32,9 +32,9 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 struct DeviceInfo {
     int sms = 0;
     int major = 0;
-    bool attr_set[3][2] = {};
-    bool pair_attr_set[3][2] = {};
-    int pair_clusters[3][2] = {};   // co-resident CTA pairs of the pair kernel, per epilogue and weight kind
+    bool attr_set[3][3] = {};
+    bool pair_attr_set[3][3] = {};
+    int pair_clusters[3][3] = {};   // co-resident CTA pairs of the pair kernel, per epilogue and weight kind
 };
 
 std::mutex g_mu;
@@ -80,7 +80,9 @@ qgmm_status device_info(DeviceInfo **out)
 qgmm_status check_problem(const qgmm_problem *p)
 {
     if (!p) return QGMM_ERR_NULL_PTR;
-    if (p->weight_type != QGMM_W_INT8 && p->weight_type != QGMM_W_INT4_PACKED_INT32) return QGMM_ERR_DTYPE;
+    if (p->weight_type != QGMM_W_INT8 && p->weight_type != QGMM_W_INT4_PACKED_INT32 &&
+        p->weight_type != QGMM_W_FP8_E4M3)
+        return QGMM_ERR_DTYPE;
     if (p->group_list_type != QGMM_GROUP_CUMSUM && p->group_list_type != QGMM_GROUP_COUNTS) return QGMM_ERR_DTYPE;
     if (p->row_index_type != QGMM_IDX_INT64 && p->row_index_type != QGMM_IDX_INT32) return QGMM_ERR_DTYPE;
     if (p->scale_type != QGMM_SCALE_F32 && p->scale_type != QGMM_SCALE_BF16) return QGMM_ERR_DTYPE;
@@ -94,7 +96,7 @@ qgmm_status check_problem(const qgmm_problem *p)
     if (p->deterministic != 0 && p->deterministic != 1) return QGMM_ERR_SHAPE;
     if (p->expected_m_per_expert < 0) return QGMM_ERR_SHAPE;
     if (p->transpose_x2 != 0 && p->transpose_x2 != 1) return QGMM_ERR_SHAPE;
-    if (p->transpose_x2 && p->weight_type != QGMM_W_INT8) return QGMM_ERR_UNSUPPORTED;
+    if (p->transpose_x2 && p->weight_type == QGMM_W_INT4_PACKED_INT32) return QGMM_ERR_UNSUPPORTED;
     if (p->ld_x2 < 0 || p->ld_sb < 0 || p->ld_out < 0 || p->ld_shared < 0) return QGMM_ERR_SHAPE;
     if (p->ld_x2 && (p->ld_x2 < p->n || p->ld_x2 % 32)) return QGMM_ERR_SHAPE;
     if (p->ld_sb && (p->ld_sb < p->n || p->ld_sb % 8)) return QGMM_ERR_SHAPE;
@@ -191,7 +193,7 @@ Plan make_plan(const qgmm_problem *p, int sms, int epi)
     // form (each CTA unpacks its own 128-column half) is exact but measured slower
     // (W4A8 at 256 and 512 rows per expert: 1.22 / 2.07 ms against 0.89 / 1.64 ms).
     pl.pair = pl.tile_rows == 128 && env_int("QGMM_PAIR", 1) != 0 &&
-              (p->weight_type == QGMM_W_INT8 || env_int("QGMM_PAIR_W4", 0) != 0);
+              (p->weight_type != QGMM_W_INT4_PACKED_INT32 || env_int("QGMM_PAIR_W4", 0) != 0);
     const int rows_per_tile = pl.pair ? 256 : pl.tile_rows;
     const int64_t max_mt = (p->m + rows_per_tile - 1) / rows_per_tile + p->e;
     const int64_t max_tiles = max_mt * NT;
@@ -237,7 +239,8 @@ qgmm_status make_maps(const qgmm_problem *p, const int8_t *x1, const void *x2, i
             return QGMM_ERR_CUDA;
     }
     const cuuint64_t ld = cuuint64_t(ld_x2(p));
-    if (p->weight_type == QGMM_W_INT8 && p->transpose_x2) {
+    const bool bytes = p->weight_type != QGMM_W_INT4_PACKED_INT32;   // int8 or E4M3: one byte per element
+    if (bytes && p->transpose_x2) {
         // (e, n, k): K-major B, a box of 128 K bytes x 128 n-rows -- the x1 tile's layout
         const cuuint64_t gdim[3] = {cuuint64_t(p->k), cuuint64_t(p->n), cuuint64_t(p->e)};
         const cuuint64_t gstride[2] = {cuuint64_t(p->k), cuuint64_t(p->k) * ld};
@@ -247,7 +250,7 @@ qgmm_status make_maps(const qgmm_problem *p, const int8_t *x1, const void *x2, i
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return QGMM_ERR_CUDA;
-    } else if (p->weight_type == QGMM_W_INT8) {
+    } else if (bytes) {
         const cuuint64_t gdim[3] = {cuuint64_t(p->n), cuuint64_t(p->k), cuuint64_t(p->e)};
         const cuuint64_t gstride[2] = {ld, ld * cuuint64_t(p->k)};
         const cuuint32_t box[3] = {128, cuuint32_t(BK), 1};
@@ -270,18 +273,27 @@ qgmm_status make_maps(const qgmm_problem *p, const int8_t *x1, const void *x2, i
     return QGMM_OK;
 }
 
-template <int EPI, bool W4>
+// Weight kinds of the kernel instantiations: int8, packed int4, E4M3.
+constexpr int WK_INT8 = 0, WK_INT4 = 1, WK_F8 = 2;
+
+int weight_kind(const qgmm_problem *p)
+{
+    return p->weight_type == QGMM_W_INT4_PACKED_INT32 ? WK_INT4 : p->weight_type == QGMM_W_FP8_E4M3 ? WK_F8 : WK_INT8;
+}
+
+template <int EPI, bool W4, bool F8 = false>
 qgmm_status launch_gemm_t(DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma, const CUtensorMap &mb,
                           const GemmArgs &a, cudaStream_t st)
 {
-    auto kern = grouped_gemm_kernel<EPI, W4>;
+    auto kern = grouped_gemm_kernel<EPI, W4, F8>;
     const size_t smem = GemmCfg<W4>::SMEM_BYTES;
+    const int wk = W4 ? WK_INT4 : F8 ? WK_F8 : WK_INT8;
     {
         std::lock_guard<std::mutex> lk(g_mu);
-        if (!dev->attr_set[EPI][W4 ? 1 : 0]) {
+        if (!dev->attr_set[EPI][wk]) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
                 return QGMM_ERR_CUDA;
-            dev->attr_set[EPI][W4 ? 1 : 0] = true;
+            dev->attr_set[EPI][wk] = true;
         }
     }
     // Programmatic dependent launch: the GEMM's prologue and mainloop may
@@ -300,11 +312,12 @@ qgmm_status launch_gemm_t(DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma
     return cudaGetLastError() == cudaSuccess ? QGMM_OK : QGMM_ERR_CUDA;
 }
 
-template <int EPI, bool W4>
+template <int EPI, bool W4, bool F8 = false>
 qgmm_status launch_pair_t(DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma, const CUtensorMap &mb,
                           const GemmArgs &a, cudaStream_t st)
 {
-    auto kern = grouped_gemm_pair_kernel<EPI, W4>;
+    auto kern = grouped_gemm_pair_kernel<EPI, W4, F8>;
+    const int wk = W4 ? WK_INT4 : F8 ? WK_F8 : WK_INT8;
     const size_t smem = PairCfg<W4>::SMEM_BYTES;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
@@ -321,19 +334,19 @@ qgmm_status launch_pair_t(DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma
     cfg.numAttrs = 1;   // the occupancy query below uses the cluster shape only
     {
         std::lock_guard<std::mutex> lk(g_mu);
-        if (!dev->pair_attr_set[EPI][W4 ? 1 : 0]) {
+        if (!dev->pair_attr_set[EPI][wk]) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
                 return QGMM_ERR_CUDA;
             cfg.gridDim = dim3(static_cast<unsigned>(dev->sms & ~1), 1, 1);
             int clusters = 0;
             if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1)
                 return QGMM_ERR_CUDA;
-            dev->pair_clusters[EPI][W4 ? 1 : 0] = clusters;
-            dev->pair_attr_set[EPI][W4 ? 1 : 0] = true;
+            dev->pair_clusters[EPI][wk] = clusters;
+            dev->pair_attr_set[EPI][wk] = true;
         }
     }
     int grid = pl.grid;
-    if (grid > 2 * dev->pair_clusters[EPI][W4 ? 1 : 0]) grid = 2 * dev->pair_clusters[EPI][W4 ? 1 : 0];
+    if (grid > 2 * dev->pair_clusters[EPI][wk]) grid = 2 * dev->pair_clusters[EPI][wk];
     cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
     cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, kern, ma, mb, a) != cudaSuccess) return QGMM_ERR_CUDA;
@@ -345,14 +358,57 @@ int gemm_launches(const Plan &pl) { return pl.pair && pl.tail_mode == 1 ? 2 : 1;
 
 // mb: weight map of the main launch; mb_tail: weight map of the single-CTA
 // tail launch (they differ only for int4 weights on CTA pairs).
+// One launch of the pair kernel / the single-CTA kernel for a runtime epilogue and weight kind.
+template <int EPI>
+qgmm_status launch_pair_wk(int wk, DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma, const CUtensorMap &mb,
+                           const GemmArgs &a, cudaStream_t st)
+{
+    switch (wk) {
+    case WK_INT4: return launch_pair_t<EPI, true>(dev, pl, ma, mb, a, st);
+    case WK_F8: return launch_pair_t<EPI, false, true>(dev, pl, ma, mb, a, st);
+    default: return launch_pair_t<EPI, false>(dev, pl, ma, mb, a, st);
+    }
+}
+
+template <int EPI>
+qgmm_status launch_single_wk(int wk, DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma, const CUtensorMap &mb,
+                             const GemmArgs &a, cudaStream_t st)
+{
+    switch (wk) {
+    case WK_INT4: return launch_gemm_t<EPI, true>(dev, pl, ma, mb, a, st);
+    case WK_F8: return launch_gemm_t<EPI, false, true>(dev, pl, ma, mb, a, st);
+    default: return launch_gemm_t<EPI, false>(dev, pl, ma, mb, a, st);
+    }
+}
+
+qgmm_status launch_pair_any(int epi, int wk, DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma,
+                            const CUtensorMap &mb, const GemmArgs &a, cudaStream_t st)
+{
+    switch (epi) {
+    case EPI_ATOMIC: return launch_pair_wk<EPI_ATOMIC>(wk, dev, pl, ma, mb, a, st);
+    case EPI_STORE_Y: return launch_pair_wk<EPI_STORE_Y>(wk, dev, pl, ma, mb, a, st);
+    default: return launch_pair_wk<EPI_RAW_ACC>(wk, dev, pl, ma, mb, a, st);
+    }
+}
+
+qgmm_status launch_single_any(int epi, int wk, DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma,
+                              const CUtensorMap &mb, const GemmArgs &a, cudaStream_t st)
+{
+    switch (epi) {
+    case EPI_ATOMIC: return launch_single_wk<EPI_ATOMIC>(wk, dev, pl, ma, mb, a, st);
+    case EPI_STORE_Y: return launch_single_wk<EPI_STORE_Y>(wk, dev, pl, ma, mb, a, st);
+    default: return launch_single_wk<EPI_RAW_ACC>(wk, dev, pl, ma, mb, a, st);
+    }
+}
+
 qgmm_status launch_gemm(int epi, DeviceInfo *dev, const qgmm_problem *p, const Plan &pl, const CUtensorMap &ma,
                         const CUtensorMap &mb, const CUtensorMap &mb_tail, const GemmArgs &a, cudaStream_t st)
 {
-    const bool w4 = p->weight_type == QGMM_W_INT4_PACKED_INT32;
+    const int wk = weight_kind(p);
     if (std::getenv("QGMM_LOG"))
         std::fprintf(stderr,
-                     "qgmm: gemm epi=%d w4=%d pair=%d m=%lld k=%lld n=%lld e=%lld tile_rows=%d slab=%d grid=%d\n",
-                     epi, int(w4), int(pl.pair), (long long)p->m, (long long)p->k, (long long)p->n, (long long)p->e,
+                     "qgmm: gemm epi=%d weights=%d pair=%d m=%lld k=%lld n=%lld e=%lld tile_rows=%d slab=%d grid=%d\n",
+                     epi, wk, int(pl.pair), (long long)p->m, (long long)p->k, (long long)p->n, (long long)p->e,
                      pl.tile_rows, pl.slab_ntiles, pl.grid);
     if (pl.pair) {
         // Pairs of 128-row half tiles on CTA pairs.  A group's odd last half tile
@@ -366,38 +422,16 @@ qgmm_status launch_gemm(int epi, DeviceInfo *dev, const qgmm_problem *p, const P
         const bool tails = tail_mode == 1;
         GemmArgs ap = a;
         ap.sched = tail_mode == 2 ? SCHED_PAIRS_TAIL128 : tails ? SCHED_PAIRS : SCHED_PAIRS_ALL;
-        qgmm_status s = QGMM_OK;
-        switch (epi) {
-        case EPI_ATOMIC: s = w4 ? launch_pair_t<EPI_ATOMIC, true>(dev, pl, ma, mb, ap, st)
-                                : launch_pair_t<EPI_ATOMIC, false>(dev, pl, ma, mb, ap, st); break;
-        case EPI_STORE_Y: s = w4 ? launch_pair_t<EPI_STORE_Y, true>(dev, pl, ma, mb, ap, st)
-                                 : launch_pair_t<EPI_STORE_Y, false>(dev, pl, ma, mb, ap, st); break;
-        default: s = w4 ? launch_pair_t<EPI_RAW_ACC, true>(dev, pl, ma, mb, ap, st)
-                        : launch_pair_t<EPI_RAW_ACC, false>(dev, pl, ma, mb, ap, st); break;
-        }
+        const qgmm_status s = launch_pair_any(epi, wk, dev, pl, ma, mb, ap, st);
         if (s != QGMM_OK || !tails) return s;
         GemmArgs at = a;
         at.sched = SCHED_TAILS;
         Plan pt = pl;
         const int64_t tail_tiles = p->e * (p->n / BN);
         pt.grid = static_cast<int>(tail_tiles < dev->sms ? tail_tiles : dev->sms);
-        switch (epi) {
-        case EPI_ATOMIC: return w4 ? launch_gemm_t<EPI_ATOMIC, true>(dev, pt, ma, mb_tail, at, st)
-                                   : launch_gemm_t<EPI_ATOMIC, false>(dev, pt, ma, mb_tail, at, st);
-        case EPI_STORE_Y: return w4 ? launch_gemm_t<EPI_STORE_Y, true>(dev, pt, ma, mb_tail, at, st)
-                                    : launch_gemm_t<EPI_STORE_Y, false>(dev, pt, ma, mb_tail, at, st);
-        default: return w4 ? launch_gemm_t<EPI_RAW_ACC, true>(dev, pt, ma, mb_tail, at, st)
-                           : launch_gemm_t<EPI_RAW_ACC, false>(dev, pt, ma, mb_tail, at, st);
-        }
+        return launch_single_any(epi, wk, dev, pt, ma, mb_tail, at, st);
     }
-    switch (epi) {
-    case EPI_ATOMIC: return w4 ? launch_gemm_t<EPI_ATOMIC, true>(dev, pl, ma, mb, a, st)
-                               : launch_gemm_t<EPI_ATOMIC, false>(dev, pl, ma, mb, a, st);
-    case EPI_STORE_Y: return w4 ? launch_gemm_t<EPI_STORE_Y, true>(dev, pl, ma, mb, a, st)
-                                : launch_gemm_t<EPI_STORE_Y, false>(dev, pl, ma, mb, a, st);
-    default: return w4 ? launch_gemm_t<EPI_RAW_ACC, true>(dev, pl, ma, mb, a, st)
-                       : launch_gemm_t<EPI_RAW_ACC, false>(dev, pl, ma, mb, a, st);
-    }
+    return launch_single_any(epi, wk, dev, pl, ma, mb, a, st);
 }
 
 GemmArgs base_args(const qgmm_problem *p, const int64_t *group_list, const Plan &pl, uint32_t *status)

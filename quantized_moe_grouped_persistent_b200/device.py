@@ -11,7 +11,8 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (QGMM_IDX_INT32, QGMM_IDX_INT64, QGMM_SCALE_BF16, QGMM_SCALE_F32, QGMM_W_INT4_PACKED_INT32, QGMM_W_INT8,
+from . import (QGMM_IDX_INT32, QGMM_IDX_INT64, QGMM_SCALE_BF16, QGMM_SCALE_F32, QGMM_W_FP8_E4M3,
+               QGMM_W_INT4_PACKED_INT32, QGMM_W_INT8,
                debug_accum, device_status, finalize, finalize_workspace, make_problem, per_token_quant)
 
 
@@ -31,7 +32,8 @@ class DeviceProblem:
         self.device = torch.device(device)
         self.m, self.k, self.n, self.e = p.m, p.k, p.n, p.e
         self.output_bs = p.output_bs
-        self.weight_type = QGMM_W_INT8 if p.weight == "int8" else QGMM_W_INT4_PACKED_INT32
+        self.weight_type = {"int8": QGMM_W_INT8, "int4": QGMM_W_INT4_PACKED_INT32,
+                            "fp8": QGMM_W_FP8_E4M3}[p.weight]
         self.group_list_type = p.group_list_type
         self.expected_m_per_expert = expected_m_per_expert
         dev = self.device

@@ -38,7 +38,7 @@ class Spec:
     routing: str          # 'top_normal' | 'zipf' | 'uniform' | 'dirichlet'
     routing_param: float
     group_list_type: int  # 0 = cumulative ends, 1 = per-group counts
-    weight: str           # 'int8' | 'int4'
+    weight: str           # 'int8' | 'int4' | 'fp8' (x1 and x2 FLOAT8 E4M3FN)
     bias: bool
     shared: bool
     shared_offset: int
@@ -59,6 +59,11 @@ CONFIGS = {
     "w4a8_prologue": Spec(5, 4096, 8, 128, 2048, 7168, "uniform", 0.0, 0, "int4", True, False, 0, True,
                           "tokens=4096 topK=8 m=32768 e=128 k=2048 n=7168; int4 weights packed 8 per int32, "
                           "bf16 activations quantised per token, bias"),
+    # page 1's Atlas 350 per-token / per-channel mode (x1 and x2 FLOAT8 E4M3FN) on the
+    # large prefill's shapes and routing
+    "fp8_prefill": Spec(6, 16384, 8, 256, 2048, 7168, "dirichlet", 0.3, 0, "fp8", False, True, 0, False,
+                        "tokens=16384 topK=8 m=131072 e=256 k=2048 n=7168; x1 and x2 FLOAT8 E4M3FN, "
+                        "Dirichlet(0.3) popularity, bf16 sharedInput at offset 0"),
 }
 
 
@@ -77,7 +82,7 @@ class Problem:
     weight: str
     x1: Optional[np.ndarray]          # int8 [m, k]   (None when the prologue makes it)
     x_bf16: Optional[np.ndarray]      # uint16 bf16 bits [m, k] (prologue workloads only)
-    x2: np.ndarray                    # int8 [e, k, n] or int32 [e, k, n/8]
+    x2: np.ndarray                    # int8 / E4M3 bytes [e, k, n] or int32 [e, k, n/8]
     scale: np.ndarray                 # f32 [e, n]
     pertoken_scale: Optional[np.ndarray]  # f32 [m]  (None when the prologue makes it)
     group_list: np.ndarray            # int64 [e]
@@ -147,6 +152,18 @@ def bf16_bits_normal(rng: np.random.Generator, shape, std: float = 1.0) -> np.nd
     return torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
 
 
+def e4m3_codes_normal(rng: np.random.Generator, shape, std: float) -> np.ndarray:
+    """FLOAT8 E4M3FN codes (uint8) of normal(0, std) draws, converted by torch's
+    float8_e4m3fn cast (round to nearest even) in chunks of the leading axis."""
+    import torch
+    out = np.empty(shape, np.uint8)
+    lead = out.reshape(shape[0], -1)
+    for i in range(shape[0]):
+        v = rng.standard_normal(lead.shape[1], dtype=np.float32) * np.float32(std)
+        lead[i] = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    return out
+
+
 def make_problem(name: str, *, tokens: Optional[int] = None, e: Optional[int] = None,
                  k: Optional[int] = None, n: Optional[int] = None, seed: Optional[int] = None,
                  group_list_type: Optional[int] = None, weights_only_experts: Optional[np.ndarray] = None,
@@ -170,12 +187,18 @@ def make_problem(name: str, *, tokens: Optional[int] = None, e: Optional[int] = 
         x1 = None
         x_bf16 = bf16_bits_normal(rng, (m, k))
         pts = None
+    elif spec.weight == "fp8":
+        x1 = e4m3_codes_normal(rng, (m, k), 4.0)
+        x_bf16 = None
+        pts = rng.uniform(1e-3, 1e-2, size=m).astype(np.float32)
     else:
         x1 = rng.integers(-127, 128, size=(m, k), dtype=np.int8)
         x_bf16 = None
         pts = rng.uniform(1e-3, 1e-2, size=m).astype(np.float32)
     if spec.weight == "int8":
         x2 = rng.integers(-127, 128, size=(e, k, n), dtype=np.int8)
+    elif spec.weight == "fp8":
+        x2 = e4m3_codes_normal(rng, (e, k, n), 0.5)
     else:
         x2 = rng.integers(0, 2 ** 32, size=(e, k, n // 8), dtype=np.uint32).view(np.int32)
     scale = rng.uniform(1e-3, 1e-2, size=(e, n)).astype(np.float32)

@@ -115,7 +115,7 @@ def test_workspace_sizes(qgmm):
     (dict(e=0), "SHAPE"), (dict(e=1025), "SHAPE"), (dict(output_bs=0), "SHAPE"),
     (dict(shared_bs=33), "SHAPE"), (dict(shared_bs=8, shared_offset=25), "SHAPE"),
     (dict(shared_offset=-1), "SHAPE"), (dict(expected_m_per_expert=-1), "SHAPE"),
-    (dict(weight_type=2), "DTYPE"), (dict(group_list_type=2), "DTYPE"), (dict(row_index_type=5), "DTYPE"),
+    (dict(weight_type=3), "DTYPE"), (dict(weight_type=-1), "DTYPE"), (dict(group_list_type=2), "DTYPE"), (dict(row_index_type=5), "DTYPE"),
     (dict(scale_type=2), "DTYPE"), (dict(scale_type=-1), "DTYPE"),
     (dict(transpose_x2=1, weight_type=1), "UNSUPPORTED"),
 ])

@@ -556,3 +556,48 @@ def test_mxfp8_cast_bounds_and_non_finite(oracle):
     q, sf = oracle.per_token_quant_mxfp8(y)
     assert sf[0, 0] == 120 and q[0, 0] == 0x7F and q[0, 1] == 0x70 and q[0, 2] == 0xF8 and q[0, 3] == 0x7F
     assert sf[0, 1] == 247 and q[0, 32] == 0x7E and q[0, 33] == 0
+
+
+# --- FP8 E4M3 operands (Atlas 350 per-token / per-channel mode) ----------------
+def test_worked_example_in_fp8(oracle):
+    """The worked example of "matmul支持pertoken量化模式", 计算示例, with x and w given
+    as FLOAT8 E4M3 codes (1, 2, 3, 4, 5, 6 are exact E4M3 values: 0x38, 0x40, 0x44,
+    0x48, 0x4A, 0x4C): the same output [[9, 24, 45], [38, 104, 198]]."""
+    g = _golden("per_token_worked_example.json")
+    code = {1: 0x38, 2: 0x40, 3: 0x44, 4: 0x48, 5: 0x4A, 6: 0x4C}
+    x = np.vectorize(code.get)(np.array(g["x"])).astype(np.uint8)
+    w = np.vectorize(code.get)(np.array(g["weight"])).astype(np.uint8)[None]
+    for gtype, gl in ((0, [2]), (1, [2])):
+        o64, _, o32 = oracle.finalize(x, w, np.array(gl, np.int64), gtype, weight="fp8",
+                                      scale=np.array([g["deqScale"]], np.float32),
+                                      pertoken_scale=np.array(g["perTokenScale"], np.float32),
+                                      row_index=np.array([0, 1], np.int64), output_bs=2)
+        np.testing.assert_array_equal(o64, g["output"])
+        np.testing.assert_array_equal(o32, np.array(g["output"], np.float32))
+
+
+def test_fp8_accum_matches_library_matmul_and_is_exact(oracle):
+    """Accumulators of E4M3 operands equal numpy's float64 matmul of the values that
+    torch's float8_e4m3fn decoding gives (library routines), group by group; and a
+    sum whose exact value needs more than f32's 24 bits (448*448 + 2^-9*2^-9) is
+    exact; the magnitude is the sum of |products|."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(41)
+    counts = np.array([5, 0, 9, 3], np.int64)
+    m, k, n, e = 17, 64, 24, 4
+    x1 = rng.integers(0, 256, (m, k), dtype=np.uint8)
+    x2 = rng.integers(0, 256, (e, k, n), dtype=np.uint8)
+    x1[(x1 & 0x7F) == 0x7F] = 0x38                             # no NaN codes
+    x2[(x2 & 0x7F) == 0x7F] = 0xB8
+    dec = lambda a: torch.from_numpy(a).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    acc, mag = oracle.accum_f8(x1, x2, counts, 1)
+    off = np.concatenate([[0], np.cumsum(counts)])
+    for g in range(e):
+        r = slice(off[g], off[g + 1])
+        np.testing.assert_array_equal(acc[r], dec(x1[r]) @ dec(x2[g]))
+        np.testing.assert_array_equal(mag[r], np.abs(dec(x1[r])) @ np.abs(dec(x2[g])))
+    assert (acc[off[-1]:] == 0).all()
+    a = np.array([[0x7E, 0x01]], np.uint8)                      # 448, 2^-9
+    w = np.array([[[0x7E], [0x01]]], np.uint8)
+    acc, _ = oracle.accum_f8(a, w, np.array([1], np.int64), 1)
+    assert acc[0, 0] == 448.0 * 448.0 + 2.0 ** -18 and np.float32(acc[0, 0]) == 200704.0
