@@ -545,7 +545,7 @@ def main():
             rates = {"pct_of_dense_int8_peak": {"nominal_4500": 100.0 * value / world / NOMINAL_INT8_TOPS,
                                                 "measured_burst": 100.0 * value / world / int8_peak,
                                                 "measured_sustained": 100.0 * value / world / int8_peak_sustained}}
-            roofline = {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TOPS",
+            roofline = {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": unit,
                         "frac": achieved / int8_peak, "traffic": committed_traffic(args.workload),
                         "kernel": gemm_kernel, "kernel_ms": gemm_max,
                         "frac_of_sustained": achieved / int8_peak_sustained,
@@ -562,7 +562,7 @@ def main():
                         "gemm_mean": gemm_max, "gemm_median": per_step["gemm_ms_median"],
                         "gemm_best": per_step["gemm_ms_best"], "of_rank": rank},
             "higher_is_better": True, "scaling": "strong",
-            "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "vs_baseline": None, "dtype": "e4m3" if p.weight == "fp8" else "int8", "data": "synthetic",
             "config": {"workload": spec_desc, "tokens": p.tokens, "topk": p.topk, "m": p.m, "e": p.e, "k": p.k,
                        "n": p_full.n, "output_bs": p.output_bs, "mode": mode,
                        "l2": "inputs larger than L2 (x2 %.2f GB on rank 0), no flush" % (p.x2.nbytes / 1e9),
