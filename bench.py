@@ -59,6 +59,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
     ap.add_argument("--tokens", type=int, default=None, help="shrink the workload (profiling proxies)")
     ap.add_argument("--experts", type=int, default=None, help="shrink the workload (profiling proxies)")
+    ap.add_argument("--transpose-x2", action="store_true",
+                    help="store the int8 / E4M3 weights (e, n, k) instead of (e, k, n); same result")
     return ap.parse_args()
 
 
@@ -431,6 +433,11 @@ def main():
     dev_index = torch.cuda.current_device()
 
     p_full = make_problem(args.workload, tokens=args.tokens, e=args.experts)
+    if args.transpose_x2:
+        import numpy as np
+        p_full.x2 = np.ascontiguousarray(np.swapaxes(p_full.x2, 1, 2))
+        p_full.transpose_x2 = True
+        spec_desc += "; weights stored (e, n, k)"
     if args.tokens or args.experts:
         spec_desc += f" (reduced: tokens={p_full.tokens}, e={p_full.e})"
     p, (c0, c1) = rank_problem(p_full, world, rank)

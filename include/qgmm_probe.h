@@ -29,6 +29,15 @@ extern "C" {
 int qgmm_probe_mma_i8(int32_t clusters, int32_t iters, unsigned long long *clock_out, uint32_t *status,
                       void *cuda_stream);
 
+/*
+ * The same probe for other tile forms: N in [16, 256], a multiple of 16 (one
+ * launch then performs clusters * iters * 256 * N * 32 MACs), and the operand
+ * majors swapped when a_mn_major != 0 (A MN-major, B K-major; otherwise A
+ * K-major, B MN-major).  qgmm_probe_mma_i8 is N = 256, a_mn_major = 0.
+ */
+int qgmm_probe_mma_i8_shape(int32_t clusters, int32_t iters, int32_t n, int32_t a_mn_major,
+                            unsigned long long *clock_out, uint32_t *status, void *cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -20,8 +20,8 @@ namespace probe {
 
 constexpr int OPERAND_BYTES = 2 * 16384;   // one 128-row A half and one 128-column B half
 
-__global__ void __launch_bounds__(64, 1) mma_i8_pair_probe(int32_t iters, unsigned long long *clock_out,
-                                                           uint32_t *status)
+__global__ void __launch_bounds__(64, 1) mma_i8_pair_probe(int32_t iters, int32_t n, int32_t a_mn_major,
+                                                           unsigned long long *clock_out, uint32_t *status)
 {
     __shared__ __align__(1024) uint8_t operands[OPERAND_BYTES];
     __shared__ uint64_t drain;
@@ -46,14 +46,17 @@ __global__ void __launch_bounds__(64, 1) mma_i8_pair_probe(int32_t iters, unsign
     ptx::tc_fence_after();
     const uint32_t tmem = holder;
     if (warp == 0 && lane == 0 && leader) {
-        const uint32_t idesc = ptx::idesc_i8(256, 256, true);
+        // A K-major and B MN-major (the grouped GEMM's int8 pair tile), or A MN-major
+        // and B K-major (the same tile transposed)
+        const uint32_t idesc = a_mn_major ? ptx::idesc_i8(256, n, false, true) : ptx::idesc_i8(256, n, true);
         const uint32_t a0 = ptx::smem_addr(operands), b0 = a0 + 16384;
         const unsigned long long c0 = clock64();
         const uint64_t g0 = ptx::globaltimer();
         for (int32_t it = 0; it < iters; ++it) {
             const uint32_t kk = static_cast<uint32_t>(it & 3);
-            const uint64_t adesc = ptx::smem_desc_sw128(a0 + kk * 32, 16, 1024);
-            const uint64_t bdesc = ptx::smem_desc_sw128(b0 + kk * 32 * 128, 16384, 1024);
+            const uint64_t kmaj = ptx::smem_desc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t mnmaj = ptx::smem_desc_sw128(b0 + kk * 32 * 128, 16384, 1024);
+            const uint64_t adesc = a_mn_major ? mnmaj : kmaj, bdesc = a_mn_major ? kmaj : mnmaj;
             ptx::mma_i8_pair(tmem, adesc, bdesc, idesc, it != 0 ? 1u : 0u);
         }
         ptx::mma_commit_pair(ptx::map_to_rank(&drain, 0));
@@ -77,10 +80,10 @@ __global__ void __launch_bounds__(64, 1) mma_i8_pair_probe(int32_t iters, unsign
 }  // namespace probe
 }  // namespace qgmm
 
-QGMM_PROBE_API int qgmm_probe_mma_i8(int32_t clusters, int32_t iters, unsigned long long *clock_out,
-                                     uint32_t *status, void *cuda_stream)
+QGMM_PROBE_API int qgmm_probe_mma_i8_shape(int32_t clusters, int32_t iters, int32_t n, int32_t a_mn_major,
+                                           unsigned long long *clock_out, uint32_t *status, void *cuda_stream)
 {
-    if (clusters < 1 || iters < 1 || !status) return 2;
+    if (clusters < 1 || iters < 1 || !status || n < 16 || n > 256 || n % 16) return 2;
     int dev = 0, major = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
@@ -98,6 +101,14 @@ QGMM_PROBE_API int qgmm_probe_mma_i8(int32_t clusters, int32_t iters, unsigned l
     cfg.stream = static_cast<cudaStream_t>(cuda_stream);
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, qgmm::probe::mma_i8_pair_probe, iters, clock_out, status) != cudaSuccess) return 6;
+    if (cudaLaunchKernelEx(&cfg, qgmm::probe::mma_i8_pair_probe, iters, n, a_mn_major ? 1 : 0, clock_out, status) !=
+        cudaSuccess)
+        return 6;
     return cudaGetLastError() == cudaSuccess ? 0 : 6;
+}
+
+QGMM_PROBE_API int qgmm_probe_mma_i8(int32_t clusters, int32_t iters, unsigned long long *clock_out,
+                                     uint32_t *status, void *cuda_stream)
+{
+    return qgmm_probe_mma_i8_shape(clusters, iters, 256, 0, clock_out, status, cuda_stream);
 }

@@ -310,26 +310,26 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
 }
 
 // Instruction descriptor for kind::i8: signed A and B, int32 accumulator,
-// A K-major, B K-major or MN-major, shape M x N.
-__host__ __device__ constexpr uint32_t idesc_i8(int M, int N, bool b_mn_major)
+// A and B each K-major or MN-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_i8(int M, int N, bool b_mn_major, bool a_mn_major = false)
 {
     return (2u << 4)                                 // D format: S32
            | (1u << 7)                               // A: signed 8-bit
            | (1u << 10)                              // B: signed 8-bit
-           | (0u << 15)                              // A K-major
+           | ((a_mn_major ? 1u : 0u) << 15)          // A major
            | ((b_mn_major ? 1u : 0u) << 16)          // B major
            | (static_cast<uint32_t>(N >> 3) << 17)   // N / 8
            | (static_cast<uint32_t>(M >> 4) << 24);  // M / 16
 }
 
 // Instruction descriptor for kind::f8f6f4 with E4M3 A and B: f32 accumulator,
-// A K-major, B K-major or MN-major, shape M x N.  (A/B format code 0 is E4M3.)
-__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool b_mn_major)
+// A and B each K-major or MN-major, shape M x N.  (A/B format code 0 is E4M3.)
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool b_mn_major, bool a_mn_major = false)
 {
     return (1u << 4)                                 // D format: F32
            | (0u << 7)                               // A: E4M3
            | (0u << 10)                              // B: E4M3
-           | (0u << 15)                              // A K-major
+           | ((a_mn_major ? 1u : 0u) << 15)          // A major
            | ((b_mn_major ? 1u : 0u) << 16)          // B major
            | (static_cast<uint32_t>(N >> 3) << 17)   // N / 8
            | (static_cast<uint32_t>(M >> 4) << 24);  // M / 16

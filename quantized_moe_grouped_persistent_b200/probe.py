@@ -9,7 +9,7 @@ import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 PROBE_LIB_PATH = os.path.join(HERE, "libqgmm_probe.so")
-MACS_PER_MMA = 256 * 256 * 32          # one cta_group::2 kind::i8 MMA, M = 256, N = 256, K = 32
+MACS_PER_MMA = 256 * 256 * 32          # one cta_group::2 kind::i8 MMA, M = 256, N = 256, K = 32 (scaled by N/256)
 
 _lib = None
 
@@ -23,14 +23,18 @@ def lib():
         L = C.CDLL(PROBE_LIB_PATH)
         L.qgmm_probe_mma_i8.argtypes = [C.c_int32, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p]
         L.qgmm_probe_mma_i8.restype = C.c_int
+        L.qgmm_probe_mma_i8_shape.argtypes = [C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p,
+                                              C.c_void_p]
+        L.qgmm_probe_mma_i8_shape.restype = C.c_int
         _lib = L
     return _lib
 
 
-def mma_i8_rate(iters: int = 16384, launches: int = 20, warmup: int = 3, clusters: int = 0) -> dict:
+def mma_i8_rate(iters: int = 16384, launches: int = 20, warmup: int = 3, clusters: int = 0, n: int = 256,
+                a_mn_major: bool = False) -> dict:
     """Median int8 rate over `launches` timed launches of the probe on every SM pair
     (or `clusters` pairs): int ops per second, MACs per clock per SM from the SM
-    clock CTA 0 saw, and that clock."""
+    clock CTA 0 saw, and that clock.  `n` and `a_mn_major` select the tile form."""
     import torch
     if clusters <= 0:
         clusters = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count // 2
@@ -39,7 +43,8 @@ def mma_i8_rate(iters: int = 16384, launches: int = 20, warmup: int = 3, cluster
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
 
     def launch():
-        rc = lib().qgmm_probe_mma_i8(clusters, iters, clk.data_ptr(), status.data_ptr(), stream.cuda_stream)
+        rc = lib().qgmm_probe_mma_i8_shape(clusters, iters, n, int(a_mn_major), clk.data_ptr(), status.data_ptr(),
+                                           stream.cuda_stream)
         if rc:
             raise RuntimeError(f"qgmm_probe_mma_i8 returned {rc}")
 
@@ -55,7 +60,7 @@ def mma_i8_rate(iters: int = 16384, launches: int = 20, warmup: int = 3, cluster
         raise RuntimeError("the probe's bounded wait ran out")
     ms = sorted(ev[i].elapsed_time(ev[i + 1]) for i in range(launches))
     med = ms[len(ms) // 2]
-    macs = clusters * iters * MACS_PER_MMA
+    macs = clusters * iters * MACS_PER_MMA * n // 256
     cycles, ns = (int(v) for v in clk.cpu().tolist())
     return {"tops": 2.0 * macs / (med * 1e-3) / 1e12, "tops_best": 2.0 * macs / (ms[0] * 1e-3) / 1e12,
             "ms_median": med, "mac_per_clk_per_sm": macs / (2 * clusters) / max(cycles, 1),

@@ -43,7 +43,7 @@ def test_probe_library_exports_its_declared_symbol(qgmm):
     exports exactly what its header declares.  Argument checks need no device."""
     text = open(os.path.join(ROOT, "include", "qgmm_probe.h")).read()
     declared = sorted(set(re.findall(r"^int\s+(qgmm_\w+)\s*\(", text, re.M)))
-    assert declared == ["qgmm_probe_mma_i8"]
+    assert declared == ["qgmm_probe_mma_i8", "qgmm_probe_mma_i8_shape"]
     from quantized_moe_grouped_persistent_b200 import probe
     out = subprocess.run(["nm", "-D", "--defined-only", probe.PROBE_LIB_PATH], capture_output=True, text=True,
                          check=True).stdout
