@@ -51,6 +51,15 @@ def lib():
         L.qo_per_token_quant_mxfp8.argtypes = [P, I64, I64, P, P]
         L.qo_accum_f8.argtypes = [P, P, I64, I64, I64, I64, P, I32, P, I64, P, P, I32]
         L.qo_accum_f8.restype = C.c_int
+        L.qo_accum_mx.argtypes = [P, P, P, P, I64, I64, I64, I64, P, I32, P, I64, P, P, I32]
+        L.qo_accum_mx.restype = C.c_int
+        L.qo_finalize_mx.argtypes = [P, P, P, P, I64, I64, I64, I64, P, I32, P, P, P, I32, P, I64, I64, I64,
+                                     P, I64, P, P, P, I32]
+        L.qo_finalize_mx.restype = C.c_int
+        L.qo_e2m1_decode.argtypes = [C.c_uint8]
+        L.qo_e2m1_decode.restype = C.c_double
+        L.qo_e8m0_decode.argtypes = [C.c_uint8]
+        L.qo_e8m0_decode.restype = C.c_double
         for f in (L.qo_group_offsets, L.qo_accum, L.qo_finalize, L.qo_per_token_quant, L.qo_bf16_to_f32,
                   L.qo_per_token_quant_mxfp8):
             f.restype = C.c_int
@@ -240,3 +249,60 @@ def per_token_quant_mxfp8(x_bf16: np.ndarray):
     if rc:
         raise OracleError(rc, "per_token_quant_mxfp8")
     return q, sf
+
+
+def e2m1_decode(nibble: int) -> float:
+    """The value of an FP4 E2M1 code (low 4 bits)."""
+    return float(lib().qo_e2m1_decode(int(nibble) & 0xF))
+
+
+def e8m0_decode(code: int) -> float:
+    """The value of an E8M0 scale code: 2^(code - 127), NaN for 0xFF."""
+    return float(lib().qo_e8m0_decode(int(code)))
+
+
+def accum_mx(x1, sfa, x2, sfb, group_list, group_list_type: int, rows=None, threads=None):
+    """MxA8W4 accumulators: x1 E4M3 uint8 [m, k], sfa E8M0 [m, k/32], x2 E2M1 pairs
+    uint8 [e, n, k/2] (lower k in the low nibble), sfb E8M0 [e, n, k/32].  Returns
+    (acc, mag) in double for source rows ``rows`` (default all)."""
+    x1, sfa, x2, sfb = (_c(a, np.uint8) for a in (x1, sfa, x2, sfb))
+    m, k = x1.shape
+    e, n = x2.shape[0], x2.shape[1]
+    r = _c(rows, np.int64)
+    nrows = m if r is None else r.shape[0]
+    acc = np.zeros((nrows, n), np.float64)
+    mag = np.zeros((nrows, n), np.float64)
+    rc = lib().qo_accum_mx(_ptr(x1), _ptr(sfa), _ptr(x2), _ptr(sfb), m, k, n, e, _ptr(_c(group_list, np.int64)),
+                           group_list_type, _ptr(r), nrows, _ptr(acc), _ptr(mag), threads or default_threads())
+    if rc:
+        raise OracleError(rc, "accum_mx")
+    return acc, mag
+
+
+def finalize_mx(x1, sfa, x2, sfb, group_list, group_list_type: int, *, logit=None, bias=None, row_index=None,
+                shared=None, shared_offset: int = 0, output_bs: Optional[int] = None, dest_rows=None,
+                want64: bool = True, want32: bool = True, threads: Optional[int] = None):
+    """MxA8W4 output rows (see ``accum_mx``): (acc + bias) * logit combined by row index.
+    Returns (out64, sabs64, out32) as ``finalize`` does."""
+    x1, sfa, x2, sfb = (_c(a, np.uint8) for a in (x1, sfa, x2, sfb))
+    m, k = x1.shape
+    e, n = x2.shape[0], x2.shape[1]
+    if output_bs is None:
+        output_bs = m
+    ri, rit = None, 0
+    if row_index is not None:
+        ri, rit = (_c(row_index, np.int32), 1) if row_index.dtype == np.int32 else (_c(row_index, np.int64), 0)
+    sh = _c(shared, np.uint16)
+    shared_bs = 0 if sh is None else sh.shape[0]
+    d = _c(dest_rows, np.int64)
+    nd = output_bs if d is None else d.shape[0]
+    out64 = np.zeros((nd, n), np.float64) if want64 else None
+    sabs = np.zeros((nd, n), np.float64) if want64 else None
+    out32 = np.zeros((nd, n), np.float32) if want32 else None
+    rc = lib().qo_finalize_mx(_ptr(x1), _ptr(sfa), _ptr(x2), _ptr(sfb), m, k, n, e, _ptr(_c(group_list, np.int64)),
+                              group_list_type, _ptr(_c(logit, np.float32)), _ptr(_c(bias, np.float32)), _ptr(ri),
+                              rit, _ptr(sh), shared_bs, shared_offset, output_bs, _ptr(d), nd, _ptr(out64),
+                              _ptr(sabs), _ptr(out32), threads or default_threads())
+    if rc:
+        raise OracleError(rc, "finalize_mx")
+    return out64, sabs, out32

@@ -52,6 +52,8 @@
 #include <string.h>
 
 float qo_e4m3_decode(uint8_t c);
+double qo_e2m1_decode(uint8_t nibble);
+double qo_e8m0_decode(uint8_t c);
 
 enum {
     QO_OK = 0,
@@ -129,6 +131,40 @@ static void accum_row_f8(const int8_t *x1, const void *x2, int64_t k, int64_t n,
     }
 }
 
+/* MxA8W4 (weight_type 3, page 1's Atlas 350 MxA8W4 mode): x1 is FLOAT8 E4M3 [m, k]
+ * with one E8M0 scale per 32 k-elements, sfa [m, k/32] (pertokenScale, shape
+ * (m, ceil(k/64), 2)); the weights are FP4 E2M1, transposed (e, n, k) as page 1
+ * requires for this mode, two per byte with the lower k in the low nibble (a
+ * reading), (e, n, k/2) bytes, with one E8M0 scale per 32 k-elements, sfb
+ * [e, n, k/32] (scale, shape (e, n, ceil(k/64), 2)).  A block's products are
+ * summed, then multiplied by both of the block's scales:
+ *   acc[j] = sum_b 2^(sfa[i][b] - 127) * 2^(sfb[g][j][b] - 127) * sum_{kk in b} x1[i][kk] * W(g, j, kk)
+ * in double; mag[j] is the same sum of |scaled products|. */
+static void accum_row_mx(const uint8_t *x1, const uint8_t *sfa, const uint8_t *w, const uint8_t *sfb, int64_t k,
+                         int64_t n, int64_t g, int64_t i, double *acc, double *mag, double *xrow)
+{
+    const int64_t nb = k / 32;
+    for (int64_t kk = 0; kk < k; ++kk) xrow[kk] = (double)qo_e4m3_decode(x1[i * k + kk]);
+    for (int64_t j = 0; j < n; ++j) {
+        const uint8_t *wr = w + (g * n + j) * (k / 2);
+        double a = 0.0, am = 0.0;
+        for (int64_t b = 0; b < nb; ++b) {
+            double sum = 0.0, sabs = 0.0;
+            for (int64_t kk = b * 32; kk < b * 32 + 32; ++kk) {
+                const uint8_t byte = wr[kk / 2];
+                const double p = xrow[kk] * qo_e2m1_decode((kk & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF));
+                sum += p;
+                sabs += fabs(p);
+            }
+            const double sc = qo_e8m0_decode(sfa[i * nb + b]) * qo_e8m0_decode(sfb[(g * n + j) * nb + b]);
+            a += sc * sum;
+            am += sc * sabs;
+        }
+        acc[j] = a;
+        mag[j] = am;
+    }
+}
+
 /* acc[j] = sum_kk x1[i][kk] * W(g, kk, j), exact; returns 0 or overflow code */
 static int accum_row(const int8_t *x1, const void *x2, int weight_type, int64_t k, int64_t n,
                      int64_t g, int64_t i, int64_t *acc64 /* [n] scratch */, int32_t *acc)
@@ -166,7 +202,7 @@ static void *job_main(void *p)
     job_t *j = (job_t *)p;
     int64_t *s64 = (int64_t *)malloc(sizeof(int64_t) * (size_t)j->n);
     int32_t *s32 = (int32_t *)malloc(sizeof(int32_t) * (size_t)j->n);
-    double *sd = (double *)malloc(sizeof(double) * 2 * (size_t)j->n);
+    double *sd = (double *)malloc(sizeof(double) * (2 * (size_t)j->n + 65536));   /* + one decoded x1 row */
     if (!s64 || !s32 || !sd) { j->rc = QO_ERR_ARG; free(s64); free(s32); free(sd); return NULL; }
     for (int64_t it = j->tid; it < j->nitems; it += j->nthreads) j->fn(j->ctx, it, s64, s32, sd, &j->rc);
     free(s64);
@@ -279,6 +315,7 @@ typedef struct {
     const uint16_t *shared; int64_t shared_bs, shared_offset, output_bs;
     const int64_t *dest_rows;
     double *out64; double *sabs64; float *out32;
+    const uint8_t *sfa, *sfb;   /* weight_type 3 only */
 } fin_ctx;
 
 static inline float bf16_to_f32(uint16_t b)
@@ -319,9 +356,12 @@ static void fin_item(void *p, int64_t it, int64_t *s64, int32_t *acc, double *sd
         if (d < 0 || d >= c->output_bs) { *rc = QO_ERR_BAD_ROW_INDEX; continue; }
         if (d != r) continue;
         int64_t g = group_of_row(c->off, c->e, i);
-        const int f8 = c->weight_type == 2;
-        double *accd = sd, *mag = sd + n;       /* FP8: exact sums and sums of |products| */
-        if (f8) {
+        const int f8 = c->weight_type == 2 || c->weight_type == 3;
+        double *accd = sd, *mag = sd + n;       /* FP8 / MX: the sums and sums of |products| */
+        if (c->weight_type == 3) {
+            accum_row_mx((const uint8_t *)c->x1, c->sfa, (const uint8_t *)c->x2, c->sfb, c->k, n, g, i, accd, mag,
+                         sd + 2 * n);
+        } else if (f8) {
             accum_row_f8(c->x1, c->x2, c->k, n, g, i, accd, mag);
         } else {
             int ar = accum_row(c->x1, c->x2, c->weight_type, c->k, n, g, i, s64, acc);
@@ -380,8 +420,75 @@ int qo_finalize(const int8_t *x1, const void *x2, int weight_type, int64_t m, in
     if (rc == QO_OK) {
         fin_ctx c = {x1, x2, weight_type, m, k, n, e, off, off[e], scale, pts, logit, bias,
                      row_index, row_index_type, shared, shared_bs, shared_offset, output_bs,
-                     dest_rows, out64, sabs64, out32};
+                     dest_rows, out64, sabs64, out32, NULL, NULL};
         rc = run_parallel(fin_item, &c, ndest, n, nthreads);
+    }
+    free(off);
+    return rc;
+}
+
+/*
+ * MxA8W4 (accum_row_mx): x1 E4M3 [m, k] with sfa E8M0 [m, k/32]; weights E2M1
+ * (e, n, k/2) bytes with sfb E8M0 [e, n, k/32]; k % 32 == 0, k <= 65536.  The
+ * output is (acc + bias) * logit combined as in qo_finalize (the block scales
+ * take the place of scale and pertokenScale); the arguments after sfb are those
+ * of qo_finalize.
+ */
+int qo_finalize_mx(const uint8_t *x1, const uint8_t *sfa, const uint8_t *x2, const uint8_t *sfb, int64_t m,
+                   int64_t k, int64_t n, int64_t e, const int64_t *group_list, int group_list_type,
+                   const float *logit, const float *bias, const void *row_index, int row_index_type,
+                   const uint16_t *shared, int64_t shared_bs, int64_t shared_offset, int64_t output_bs,
+                   const int64_t *dest_rows, int64_t ndest, double *out64, double *sabs64, float *out32,
+                   int nthreads)
+{
+    if (!x1 || !sfa || !x2 || !sfb || k < 32 || k % 32 || k > 65536 || n < 1 || output_bs < 1) return QO_ERR_ARG;
+    if (shared && (shared_offset < 0 || shared_offset + shared_bs > output_bs)) return QO_ERR_ARG;
+    int64_t *off = (int64_t *)malloc(sizeof(int64_t) * (size_t)(e + 1));
+    if (!off) return QO_ERR_ARG;
+    int rc = qo_group_offsets(group_list, e, group_list_type, m, off);
+    if (rc == QO_OK) {
+        fin_ctx c = {(const int8_t *)x1, x2, 3, m, k, n, e, off, off[e], NULL, NULL, logit, bias,
+                     row_index, row_index_type, shared, shared_bs, shared_offset, output_bs,
+                     dest_rows, out64, sabs64, out32, sfa, sfb};
+        rc = run_parallel(fin_item, &c, ndest, n, nthreads);
+    }
+    free(off);
+    return rc;
+}
+
+/* MxA8W4 accumulators (accum_row_mx) for source rows rows[0..nrows) (NULL: all);
+ * rows past the total come back as zeros. */
+typedef struct {
+    const uint8_t *x1, *sfa, *x2, *sfb; int64_t k, n, e;
+    const int64_t *off; const int64_t *rows; double *acc_out, *mag_out;
+} accum_mx_ctx;
+
+static void accum_mx_item(void *p, int64_t it, int64_t *s64, int32_t *s32, double *sd, int *rc)
+{
+    accum_mx_ctx *c = (accum_mx_ctx *)p;
+    (void)s64; (void)s32; (void)rc;
+    int64_t i = c->rows ? c->rows[it] : it;
+    double *dst = c->acc_out + it * c->n;
+    double *mag = c->mag_out ? c->mag_out + it * c->n : sd + c->n;
+    int64_t g = group_of_row(c->off, c->e, i);
+    if (g < 0) {
+        for (int64_t j = 0; j < c->n; ++j) dst[j] = mag[j] = 0.0;
+        return;
+    }
+    accum_row_mx(c->x1, c->sfa, c->x2, c->sfb, c->k, c->n, g, i, dst, mag, sd + 2 * c->n);
+}
+
+int qo_accum_mx(const uint8_t *x1, const uint8_t *sfa, const uint8_t *x2, const uint8_t *sfb, int64_t m,
+                int64_t k, int64_t n, int64_t e, const int64_t *group_list, int group_list_type,
+                const int64_t *rows, int64_t nrows, double *acc_out, double *mag_out, int nthreads)
+{
+    if (!x1 || !sfa || !x2 || !sfb || !acc_out || k < 32 || k % 32 || k > 65536 || n < 1) return QO_ERR_ARG;
+    int64_t *off = (int64_t *)malloc(sizeof(int64_t) * (size_t)(e + 1));
+    if (!off) return QO_ERR_ARG;
+    int rc = qo_group_offsets(group_list, e, group_list_type, m, off);
+    if (rc == QO_OK) {
+        accum_mx_ctx c = {x1, sfa, x2, sfb, k, n, e, off, rows, acc_out, mag_out};
+        rc = run_parallel(accum_mx_item, &c, nrows, n, nthreads);
     }
     free(off);
     return rc;
@@ -499,4 +606,19 @@ int qo_per_token_quant_mxfp8(const uint16_t *x_bf16, int64_t rows, int64_t k, ui
         }
     }
     return QO_OK;
+}
+
+/* FP4 E2M1 from its definition: sign (bit 3), 2 exponent bits (bias 1), 1 fraction
+ * bit; exponent 0 holds the subnormal m * 0.5.  Values 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+double qo_e2m1_decode(uint8_t nibble)
+{
+    const int e = (nibble >> 1) & 3, m = nibble & 1;
+    const double v = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return (nibble & 8) ? -v : v;
+}
+
+/* E8M0 scale from its definition: 2^(c - 127); 0xFF is NaN. */
+double qo_e8m0_decode(uint8_t c)
+{
+    return c == 0xFF ? NAN : ldexp(1.0, (int)c - 127);
 }

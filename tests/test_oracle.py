@@ -601,3 +601,75 @@ def test_fp8_accum_matches_library_matmul_and_is_exact(oracle):
     w = np.array([[[0x7E], [0x01]]], np.uint8)
     acc, _ = oracle.accum_f8(a, w, np.array([1], np.int64), 1)
     assert acc[0, 0] == 448.0 * 448.0 + 2.0 ** -18 and np.float32(acc[0, 0]) == 200704.0
+
+
+# --- MxA8W4: E4M3 activations, E2M1 weights, E8M0 scales per 32 k -------------
+def test_e2m1_and_e8m0_code_points(oracle):
+    """FP4 E2M1 (sign, 2 exponent bits with bias 1, 1 fraction bit, subnormal 0.5 at
+    exponent 0): the 16 code points by hand.  E8M0 (2^(c-127), 0xFF NaN): every code
+    against torch's float8_e8m0fnu decoding (a library routine)."""
+    vals = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    for c in range(16):
+        v = oracle.e2m1_decode(c)
+        assert v == (-vals[c - 8] if c >= 8 else vals[c]) and (np.signbit(v) == (c >= 8)), c
+    torch = pytest.importorskip("torch")
+    codes = np.arange(255, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e8m0fnu).to(torch.float64).numpy()
+    np.testing.assert_array_equal([oracle.e8m0_decode(int(c)) for c in codes], ref)
+    assert np.isnan(oracle.e8m0_decode(0xFF))
+
+
+def test_mx_hand_worked_blocks(oracle):
+    """One row, one output column, k = 64 (two blocks of 32), by hand:
+      block 0: x = 1.0 (0x38) everywhere, w = 1.5 (nibble 3) everywhere: sum 48;
+               scales 2^0 (127) and 2^1 (128): 96
+      block 1: x[32] = 2.0 (0x40), x[33] = 1.0, the rest 0; w[32] = -6 (nibble 0xF, the
+               byte's low nibble: even k), w[33] = 0.5 (nibble 1, high nibble): sum
+               -12 + 0.5 = -11.5; scales 2^-1 (126) and 2^0: -5.75
+      acc = 90.25; bias 1, logit 0.5: (90.25 + 1) * 0.5 = 45.625.
+    The other nibble order would give block 1 = 2*0.5 + 1*(-6) = -5 -> out 47.25."""
+    x1 = np.zeros((1, 64), np.uint8)
+    x1[0, :32] = 0x38
+    x1[0, 32], x1[0, 33] = 0x40, 0x38
+    w = np.zeros((1, 1, 32), np.uint8)
+    w[0, 0, :16] = 0x33
+    w[0, 0, 16] = 0x1F                                  # k = 32: low nibble 0xF, k = 33: high nibble 1
+    sfa = np.array([[127, 126]], np.uint8)
+    sfb = np.array([[[128, 127]]], np.uint8)
+    acc, mag = oracle.accum_mx(x1, sfa, w, sfb, np.array([1], np.int64), 1)
+    assert acc[0, 0] == 90.25 and mag[0, 0] == 96 + 0.5 * 12.5
+    o64, sabs, o32 = oracle.finalize_mx(x1, sfa, w, sfb, np.array([1], np.int64), 1,
+                                        logit=np.array([0.5], np.float32), bias=np.array([[1.0]], np.float32),
+                                        output_bs=1)
+    assert o64[0, 0] == 45.625 and o32[0, 0] == np.float32(45.625)
+
+
+def test_mx_accum_matches_blockwise_library_matmul(oracle):
+    """Accumulators against numpy float64 matmuls, block by block, of torch-decoded E4M3
+    activations and E2M1 weights (decoded through a table of the 16 code points),
+    scaled by torch-decoded E8M0 scales, with empty and ragged groups."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(77)
+    counts = np.array([3, 0, 6, 2], np.int64)
+    m, k, n, e = 13, 96, 10, 4
+    x1 = rng.integers(0, 256, (m, k), dtype=np.uint8)
+    x1[(x1 & 0x7F) == 0x7F] = 0x30
+    w = rng.integers(0, 256, (e, n, k // 2), dtype=np.uint8)
+    sfa = rng.integers(118, 136, (m, k // 32), dtype=np.uint8)
+    sfb = rng.integers(118, 136, (e, n, k // 32), dtype=np.uint8)
+    table = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0])
+    wv = np.empty((e, n, k))
+    wv[:, :, 0::2] = table[w & 0xF]
+    wv[:, :, 1::2] = table[w >> 4]
+    xv = torch.from_numpy(x1).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    e8 = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.float8_e8m0fnu).to(torch.float64).numpy()
+    acc, _ = oracle.accum_mx(x1, sfa, w, sfb, counts, 1)
+    off = np.concatenate([[0], np.cumsum(counts)])
+    for g in range(e):
+        r = slice(off[g], off[g + 1])
+        ref = np.zeros((counts[g], n))
+        for b in range(k // 32):
+            kb = slice(32 * b, 32 * b + 32)
+            ref += (xv[r, kb] @ wv[g][:, kb].T) * e8(sfa[r, b])[:, None] * e8(sfb[g, :, b])[None, :]
+        np.testing.assert_allclose(acc[r], ref, rtol=1e-13, atol=0)
+    assert (acc[off[-1]:] == 0).all()
