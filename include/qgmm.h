@@ -63,8 +63,9 @@ typedef enum {
 } qgmm_status;
 
 /* x2 (and x1) element type: int8 x2 (e,k,n) | int4 packed in int32 (e,k,n/8) |
- * FLOAT8 E4M3FN x1 and x2 (e,k,n), page 1's Atlas 350 per-token / per-channel mode */
-enum { QGMM_W_INT8 = 0, QGMM_W_INT4_PACKED_INT32 = 1, QGMM_W_FP8_E4M3 = 2 };
+ * FLOAT8 E4M3FN x1 and x2 (e,k,n), page 1's Atlas 350 per-token / per-channel mode |
+ * MxA8W4: E4M3 x1, FP4 E2M1 x2 (e,n,k/2 bytes), E8M0 block scales (page 1, Atlas 350) */
+enum { QGMM_W_INT8 = 0, QGMM_W_INT4_PACKED_INT32 = 1, QGMM_W_FP8_E4M3 = 2, QGMM_W_MXFP4 = 3 };
 enum { QGMM_IDX_INT64 = 0, QGMM_IDX_INT32 = 1 };          /* row_index element type             */
 enum { QGMM_GROUP_CUMSUM = 0, QGMM_GROUP_COUNTS = 1 };    /* group_list meaning                 */
 enum { QGMM_SCALE_F32 = 0, QGMM_SCALE_BF16 = 1 };         /* scale element type                 */
@@ -89,6 +90,19 @@ enum { QGMM_SCALE_F32 = 0, QGMM_SCALE_BF16 = 1 };         /* scale element type 
  *                   per-token pertokenScale); acc is then the tensor core's f32 sum
  *                   of the E4M3 products (not exact: rounded once per K = 32 step
  *                   at most), and the dequant below starts from that f32 value.
+ *                   With QGMM_W_MXFP4 (page 1's Atlas 350 MxA8W4 mode, where x2 is
+ *                   transposed and pertokenScale and scale hold one scale per 32
+ *                   k-elements): x1 is E4M3 [m, k]; x2 holds FP4 E2M1 values
+ *                   (e, n, k), two per byte with the lower k in the low nibble,
+ *                   (e, n, k/2) bytes, and transpose_x2 must be 1; pertoken_scale
+ *                   points to E8M0 bytes sfa [m, k/32] (as produced by
+ *                   qgmm_per_token_quant_mxfp8) and scale to E8M0 bytes sfb
+ *                   [e, n, k/32], both required; then
+ *                     acc[i][j] = sum_b 2^(sfa[i][b]-127) 2^(sfb[g][j][b]-127)
+ *                                       * sum_{kk in block b} x1[i][kk] W(g, j, kk)
+ *                   summed by the tensor core in f32 (tcgen05.mma
+ *                   kind::mxf8f6f4.block_scale), and y = (acc + bias) * logit.
+ *                   ld_sb is then the n-stride of sfb and bias; ld_x2 that of x2.
  *   group_list_type QGMM_GROUP_CUMSUM (0) | QGMM_GROUP_COUNTS (1)
  *   row_index_type  QGMM_IDX_INT64 | QGMM_IDX_INT32
  *   shared_bs, shared_offset   sharedInput rows and where they land;
@@ -152,7 +166,8 @@ typedef struct {
  *                                      max(1, floor(max(2^24, m*n/16) / output_bs)))
  *   + (output_bs + 1)*4        bucket boundaries
  *   + m*4                      source rows grouped by destination
- * Errors: NULL_PTR, SHAPE, DTYPE, UNSUPPORTED (transpose_x2 with int4 weights).
+ * Errors: NULL_PTR, SHAPE, DTYPE, UNSUPPORTED (transpose_x2 with int4 weights, or
+ * QGMM_W_MXFP4 without transpose_x2).
  */
 qgmm_status qgmm_finalize_workspace(const qgmm_problem *p, size_t *ws_bytes);
 
@@ -315,11 +330,24 @@ qgmm_status qgmm_per_token_quant_mxfp8(const uint16_t *x_bf16, int64_t rows, int
  * past the total are not written.  acc_out: int32 [m, n], 16-byte aligned.
  * `p` supplies m, k, n, e, weight_type, group_list_type and the tiling hint;
  * the workspace is the atomic-mode one (>= 256 bytes).
- * Errors: as qgmm_finalize.
+ * Errors: as qgmm_finalize, and DTYPE for QGMM_W_MXFP4 (use qgmm_debug_accum_mx).
  */
 qgmm_status qgmm_debug_accum(const qgmm_problem *p, const int8_t *x1, const void *x2,
                              const int64_t *group_list, int32_t *acc_out, void *workspace,
                              size_t ws_bytes, void *cuda_stream);
+
+/*
+ * The parity hook for QGMM_W_MXFP4 (qgmm_debug_accum has no scale arguments;
+ * no counterpart on the pages): the block-scaled f32 accumulators acc_out[i][j]
+ * (see QGMM_W_MXFP4 above) for every row i below the groups' total, written by the
+ * same kernel qgmm_finalize runs for this type, with no epilogue arithmetic and no
+ * combine.  x1 E4M3 [m, k], sfa E8M0 [m, k/32], x2 E2M1 pairs (e, n, k/2), sfb E8M0
+ * [e, n, k/32], acc_out f32 [m, n]; all 16-byte aligned; workspace >= 256 bytes.
+ * Errors: as qgmm_debug_accum, and DTYPE for any other weight type.
+ */
+qgmm_status qgmm_debug_accum_mx(const qgmm_problem *p, const uint8_t *x1, const uint8_t *sfa, const void *x2,
+                                const uint8_t *sfb, const int64_t *group_list, float *acc_out, void *workspace,
+                                size_t ws_bytes, void *cuda_stream);
 
 /*
  * Page 1, return values of both stages: each call returns a status code (an

@@ -37,6 +37,7 @@ QGMM_STATIC_SCRATCH_BYTES = 16 << 20
 QGMM_W_INT8 = 0
 QGMM_W_INT4_PACKED_INT32 = 1
 QGMM_W_FP8_E4M3 = 2
+QGMM_W_MXFP4 = 3
 QGMM_IDX_INT64 = 0
 QGMM_IDX_INT32 = 1
 QGMM_GROUP_CUMSUM = 0
@@ -51,7 +52,8 @@ QGMM_DEV_ROW_INDEX_RANGE = 1 << 3
 QGMM_DEV_TIMEOUT = 1 << 4
 
 EXPORTS = ("qgmm_finalize_workspace", "qgmm_finalize_launches", "qgmm_plan", "qgmm_finalize", "qgmm_finalize_profiled",
-           "qgmm_per_token_quant", "qgmm_per_token_quant_mxfp8", "qgmm_debug_accum", "qgmm_device_status",
+           "qgmm_per_token_quant", "qgmm_per_token_quant_mxfp8", "qgmm_debug_accum", "qgmm_debug_accum_mx",
+           "qgmm_device_status",
            "qgmm_finalize_static_scratch", "qgmm_status_string")
 
 
@@ -101,6 +103,7 @@ def lib():
         L.qgmm_per_token_quant.argtypes = [P, I64, I64, P, P, P]
         L.qgmm_per_token_quant_mxfp8.argtypes = [P, I64, I64, P, P, P]
         L.qgmm_debug_accum.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, U, P]
+        L.qgmm_debug_accum_mx.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, P, P, U, P]
         L.qgmm_device_status.argtypes = [P, C.POINTER(C.c_uint32), P]
         L.qgmm_finalize_static_scratch.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, P, P, P, P, P, P]
         L.qgmm_status_string.argtypes = [C.c_int]
@@ -218,6 +221,16 @@ def debug_accum(problem: QgmmProblem, x1, x2, group_list, acc_out, workspace, ws
     rc = lib().qgmm_debug_accum(C.byref(problem), _ptr(x1), _ptr(x2), _ptr(group_list), _ptr(acc_out),
                                 _ptr(workspace), ws_bytes, _stream(stream))
     _check(rc, "qgmm_debug_accum")
+
+
+def debug_accum_mx(problem: QgmmProblem, x1, sfa, x2, sfb, group_list, acc_out, workspace,
+                   ws_bytes: Optional[int] = None, stream=None) -> None:
+    """MxA8W4 block-scaled f32 accumulators into ``acc_out`` (f32 [m, n])."""
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().qgmm_debug_accum_mx(C.byref(problem), _ptr(x1), _ptr(sfa), _ptr(x2), _ptr(sfb), _ptr(group_list),
+                                   _ptr(acc_out), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "qgmm_debug_accum_mx")
 
 
 def device_status(workspace, stream=None) -> int:

@@ -100,6 +100,8 @@ struct GemmArgs {
     float *out;            // EPI_ATOMIC: out [output_bs, ldd]; EPI_STORE_Y: y [m, ldd]
     int32_t *acc_out;      // EPI_RAW_ACC: [m, ldd]
     int64_t ldd;           // row stride of the destination (out, y or acc_out)
+    const uint8_t *sfa;    // MX kernel: E8M0 scales of x1 [m, k/32]
+    const uint8_t *sfb;    // MX kernel: E8M0 scales of the weights [e, ld_sb, k/32]
     uint32_t *status;
 };
 
@@ -350,7 +352,7 @@ template <int EPI, int NCH, int SHIFT, bool FACC = false>
 __device__ __forceinline__ bool epilogue_tile(const GemmArgs &args, const TileCoord &c, int64_t row_base,
                                               int rows_here, int row_off, uint32_t tmem_acc, int q, int tmem_col,
                                               int glob_col, int lane, uint64_t *tfull_bar, uint32_t use,
-                                              volatile int *abort_flag, const EpiSmem &sm)
+                                              volatile int *abort_flag, const EpiSmem &sm, int tile_n = BN)
 {
     const int64_t ldd = args.ldd;
     const int col_begin = glob_col;       // tile column of this warp's first TMEM column
@@ -382,7 +384,7 @@ __device__ __forceinline__ bool epilogue_tile(const GemmArgs &args, const TileCo
         bs[k] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     if (EPI != EPI_RAW_ACC && any) {
-        const int64_t base = static_cast<int64_t>(c.g) * args.ld_sb + static_cast<int64_t>(c.nt) * BN + col_begin + col4;
+        const int64_t base = static_cast<int64_t>(c.g) * args.ld_sb + static_cast<int64_t>(c.nt) * tile_n + col_begin + col4;
         if (args.scale) {
 #pragma unroll
             for (int k = 0; k < NCH; ++k) sc[k] = load_scale4(args, base + k * 32);
@@ -396,7 +398,7 @@ __device__ __forceinline__ bool epilogue_tile(const GemmArgs &args, const TileCo
     if (!ptx::mbar_wait(tfull_bar, use, abort_flag)) return false;
     ptx::tc_fence_after();
     if (any) {
-        const int64_t n0 = static_cast<int64_t>(c.nt) * BN + col_begin;
+        const int64_t n0 = static_cast<int64_t>(c.nt) * tile_n + col_begin;
         const uint32_t tbase = tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(tmem_col);
         uint32_t ra[32], rb[32];
         ptx::tmem_ld_32x32b_x32(tbase, ra);
@@ -1144,6 +1146,322 @@ __global__ void __launch_bounds__(PairCfg<W4>::THREADS, 1)
     if (warp == 1) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- K2, MxA8W4 form
+// Page 1's Atlas 350 MxA8W4 mode: x1 FLOAT8 E4M3 [m, k] with an E8M0 scale per 32
+// k-elements (sfa [m, k/32]); weights FP4 E2M1, transposed (e, n, k) and packed two
+// per byte (lower k in the low nibble), with an E8M0 scale per 32 k-elements (sfb
+// [e, n, k/32]).  Single CTA, M = 128 rows x N = 128 columns per tile, K = 128 per
+// stage.  The producer TMA-loads the x1 tile (128-byte swizzle) and the packed
+// weight tile (128 n-rows x 64 bytes), and its 32 lanes load the stage's scale
+// words (4 blocks of each row and column) into shared memory in the 32 x 16-byte
+// layout that tcgen05.cp .32x128b.warpx4 takes: byte (r % 32) * 16 + (r / 32) * 4 + b.
+// Four unpack warps turn each E2M1 nibble into the E4M3 byte of the same value
+// (exact: every E2M1 value is an E4M3 value) in a K-major 128-byte-swizzled tile.
+// The MMA thread copies the scale words into tensor memory and issues
+// tcgen05.mma.kind::mxf8f6f4.block_scale (E4M3 x E4M3, one scale byte per 32 K per
+// row of A and column of B, selected per instruction), accumulating f32 in TMEM.
+// The epilogue is the staged one with unit scale and pertokenScale: the block
+// scales already sit inside the accumulator, so y = (acc + bias) * logit.
+constexpr int MX_BN = 128;                     // output columns per MX tile
+constexpr int MX_SF_BYTES = 512;               // one stage's scale words of 128 rows (or columns)
+constexpr uint32_t MX_TMEM_SF = 2 * MX_BN;     // TMEM column of the scale-factor buffers
+
+struct MxCfg {
+    static constexpr int STAGES = 4;
+    static constexpr int EPI_WARPS = 4;
+    static constexpr int UNPACK_WARPS = 4;
+    static constexpr int THREADS = (2 + EPI_WARPS + UNPACK_WARPS) * 32;
+    static constexpr int A_BYTES = BM * BK;            // x1 tile
+    static constexpr int B_BYTES = MX_BN * BK;         // unpacked weight tile (E4M3, K-major)
+    static constexpr int P_BYTES = MX_BN * BK / 2;     // packed E2M1 weight tile
+    static constexpr int NUM_BARS = 3 * STAGES + 2 + 2 + 1;
+    static constexpr int CTRL_BYTES = (NUM_BARS * 8 + 16 + 15) / 16 * 16;
+    static constexpr int TABLE_BYTES = (2 * (MAX_E + 1) * 4 + 15) / 16 * 16;
+    static constexpr int EPI_STAGE_BYTES = EPI_WARPS * 32 * EPI_LD * 4;
+    static constexpr int ROWINFO_BYTES = EPI_WARPS * 32 * 16;
+    static constexpr size_t OFF_B = size_t(STAGES) * A_BYTES;
+    static constexpr size_t OFF_P = OFF_B + size_t(STAGES) * B_BYTES;
+    static constexpr size_t OFF_SFA = OFF_P + size_t(STAGES) * P_BYTES;
+    static constexpr size_t OFF_SFB = OFF_SFA + size_t(STAGES) * MX_SF_BYTES;
+    static constexpr size_t OFF_CTRL = OFF_SFB + size_t(STAGES) * MX_SF_BYTES;
+    static constexpr size_t OFF_TABLE = OFF_CTRL + CTRL_BYTES;
+    static constexpr size_t OFF_EPI = OFF_TABLE + TABLE_BYTES;
+    static constexpr size_t OFF_ROWS = OFF_EPI + EPI_STAGE_BYTES;
+    static constexpr size_t SMEM_BYTES = 1024 + OFF_ROWS + ROWINFO_BYTES;
+    static_assert(SMEM_BYTES <= 232448, "shared memory above the sm_100 per-block limit");
+};
+
+// Eight E2M1 nibbles (lowest first) -> eight E4M3 bytes: the magnitude through an
+// 8-entry byte table (prmt), the sign from the nibble's top bit (prmt sign mode on
+// bytes whose top bit is that sign).
+__device__ __forceinline__ void e2m1x8_to_e4m3(uint32_t w, uint32_t &lo, uint32_t &hi)
+{
+    constexpr uint32_t LUT_LO = 0x3C383000u;   // 0, 0.5, 1, 1.5
+    constexpr uint32_t LUT_HI = 0x4C484440u;   // 2, 3, 4, 6
+    const uint32_t w4 = w << 4;
+    lo = __byte_perm(LUT_LO, LUT_HI, w & 0x7777u) | (__byte_perm(w4, w, 0xD9C8u) & 0x80808080u);
+    hi = __byte_perm(LUT_LO, LUT_HI, (w >> 16) & 0x7777u) | (__byte_perm(w4, w, 0xFBEAu) & 0x80808080u);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(MxCfg::THREADS, 1)
+    grouped_gemm_mx_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                           const GemmArgs args)
+{
+    using Cfg = MxCfg;
+    constexpr int S = Cfg::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *smem_a = smem;
+    uint8_t *smem_b = smem + Cfg::OFF_B;
+    uint8_t *smem_p = smem + Cfg::OFF_P;
+    uint8_t *smem_sfa = smem + Cfg::OFF_SFA;
+    uint8_t *smem_sfb = smem + Cfg::OFF_SFB;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_CTRL);
+    uint64_t *pfull = bars;           // x1 tile and packed weight tile landed
+    uint64_t *full = bars + S;        // weights unpacked and scale words written
+    uint64_t *empty = bars + 2 * S;   // MMAs finished reading the stage
+    uint64_t *tfull = bars + 3 * S;   // accumulator buffer ready for the epilogue
+    uint64_t *tempty = tfull + 2;     // epilogue drained the accumulator buffer
+    uint64_t *drain = tempty + 2;     // all issued MMAs completed
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + Cfg::NUM_BARS);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    int32_t *off = reinterpret_cast<int32_t *>(smem + Cfg::OFF_TABLE);
+    int32_t *cum = off + (MAX_E + 1);
+    float *epi_stage = reinterpret_cast<float *>(smem + Cfg::OFF_EPI);
+    float *row_pts = reinterpret_cast<float *>(smem + Cfg::OFF_ROWS);
+    float *row_lg = row_pts + Cfg::EPI_WARPS * 32;
+    long long *row_dst = reinterpret_cast<long long *>(row_lg + Cfg::EPI_WARPS * 32);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            ptx::mbar_init(&pfull[s], 1);
+            ptx::mbar_init(&full[s], Cfg::UNPACK_WARPS + 1);   // the unpack warps and the scale writer
+            ptx::mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&tfull[b], 1);
+            ptx::mbar_init(&tempty[b], Cfg::EPI_WARPS);
+        }
+        ptx::mbar_init(drain, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    volatile uint32_t *group_flags = reinterpret_cast<volatile uint32_t *>(tmem_holder + 2);
+    if (warp == 0) {
+        const uint32_t flags = decode_groups_warp(args.group_list, args.e, args.group_list_type, args.m, BM,
+                                                  SCHED_TILES, off, cum);
+        if (lane == 0) {
+            *group_flags = flags;
+            ptx::prefetch_tmap(&map_a);
+            ptx::prefetch_tmap(&map_b);
+        }
+    } else if (warp == 1) {
+        ptx::tmem_alloc(tmem_holder, 512);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    const int e = args.e;
+    const int MT = cum[e];
+    const int NT = args.n / MX_BN;
+    const int SW = args.slab_ntiles;
+    const int T = MT * NT;
+    const int KB = args.k / BK;
+    const int64_t nb = args.k / 32;   // scale bytes per row / column
+
+    // The status word is cleared by the kernel this one may overlap under programmatic
+    // dependent launch: wait for that kernel before setting a bit in it.
+    auto fail = [&]() {
+        ptx::pdl_wait_primary();
+        atomicOr(args.status, QGMM_DEV_TIMEOUT);
+        *abort_flag = 1;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------ producer: TMA (lane 0) and scale words (all lanes)
+        uint32_t issued[S];
+#pragma unroll
+        for (int s = 0; s < S; ++s) issued[s] = 0;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = args.stall_producer == 0;
+        for (int t = blockIdx.x; t < T && ok; t += gridDim.x) {
+            const TileCoord c = tile_coord(t, MT, SW, off, cum, e, BM, SCHED_TILES);
+            const int n0 = c.nt * MX_BN;
+            for (int kb = 0; kb < KB; ++kb) {
+                bool got = true;
+                if (lane == 0) got = ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag);
+                got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+                if (!got) {
+                    if (lane == 0) fail();
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    ptx::mbar_arrive_expect_tx(&pfull[stage], Cfg::A_BYTES + Cfg::P_BYTES);
+                    ptx::tma_load_2d(smem_a + stage * Cfg::A_BYTES, &map_a, &pfull[stage], kb * BK, c.row0);
+                    ptx::tma_load_3d(smem_p + stage * Cfg::P_BYTES, &map_b, &pfull[stage], kb * (BK / 2), n0, c.g);
+                }
+                // scale words of the stage's 4 blocks: rows / columns lane, lane + 32, lane + 64, lane + 96
+                uint32_t wa[4], wb[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int64_t r = static_cast<int64_t>(c.row0) + lane + 32 * j;
+                    wa[j] = r < args.m ? __ldg(reinterpret_cast<const unsigned int *>(args.sfa + r * nb + 4 * kb)) : 0u;
+                    const int64_t col = static_cast<int64_t>(c.g) * args.ld_sb + n0 + lane + 32 * j;
+                    wb[j] = __ldg(reinterpret_cast<const unsigned int *>(args.sfb + col * nb + 4 * kb));
+                }
+                *reinterpret_cast<uint4 *>(smem_sfa + stage * MX_SF_BYTES + lane * 16) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+                *reinterpret_cast<uint4 *>(smem_sfb + stage * MX_SF_BYTES + lane * 16) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+                ptx::fence_async_shared();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&full[stage]);
+                ++issued[stage];
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            // let the copies already in flight land before the CTA leaves
+            for (int s = 0; s < S; ++s) {
+                if (issued[s] == 0) continue;
+                volatile int never = 0;
+                ptx::mbar_wait(&pfull[s], (issued[s] - 1u) & 1u, &never);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int lt = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < T && ok; t += gridDim.x, ++lt) {
+                const int buf = lt & 1;
+                const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
+                if (!ptx::mbar_wait(&tempty[buf], use ^ 1u, abort_flag)) {
+                    fail();
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * MX_BN);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!ptx::mbar_wait(&full[stage], phase, abort_flag)) {
+                        fail();
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    // this stage's scale words into TMEM (two buffers, by stage parity)
+                    const uint32_t sfa_t = tmem_base + MX_TMEM_SF + 8u * static_cast<uint32_t>(stage & 1);
+                    const uint32_t sfb_t = sfa_t + 4u;
+                    ptx::tmem_cp_32x128b_warpx4(sfa_t, ptx::smem_desc_noswizzle(
+                                                           ptx::smem_addr(smem_sfa + stage * MX_SF_BYTES), 16, 128));
+                    ptx::tmem_cp_32x128b_warpx4(sfb_t, ptx::smem_desc_noswizzle(
+                                                           ptx::smem_addr(smem_sfb + stage * MX_SF_BYTES), 16, 128));
+                    const uint32_t a0 = ptx::smem_addr(smem_a + stage * Cfg::A_BYTES);
+                    const uint32_t b0 = ptx::smem_addr(smem_b + stage * Cfg::B_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+                        const uint64_t adesc = ptx::smem_desc_sw128(a0 + kk * UMMA_K, 16, 1024);
+                        const uint64_t bdesc = ptx::smem_desc_sw128(b0 + kk * UMMA_K, 16, 1024);
+                        ptx::mma_mx_e4m3(d_tmem, adesc, bdesc, ptx::idesc_mx_e4m3(BM, MX_BN, kk, kk), sfa_t, sfb_t,
+                                         (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    ptx::mma_commit(&empty[stage]);
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (ok) ptx::mma_commit(&tfull[buf]);
+            }
+            ptx::mma_commit(drain);
+            volatile int never = 0;
+            ptx::mbar_wait(drain, 0, &never);
+        }
+        __syncwarp();
+    } else if (warp < 2 + Cfg::EPI_WARPS) {
+        // ------------------------------------------------ epilogue: 4 warps, staged through smem
+        ptx::pdl_wait_primary();
+        if (warp == 2 && lane == 0 && blockIdx.x == 0 && *group_flags) atomicOr(args.status, *group_flags);
+        const int q = warp & 3;
+        const EpiSmem sm = epi_smem(epi_stage, row_pts, row_lg, row_dst, q);
+        int lt = 0;
+        for (int t = blockIdx.x; t < T; t += gridDim.x, ++lt) {
+            const TileCoord c = tile_coord(t, MT, SW, off, cum, e, BM, SCHED_TILES);
+            const int buf = lt & 1;
+            const uint32_t use = static_cast<uint32_t>(lt >> 1) & 1u;
+            if (!epilogue_tile<EPI, MX_BN / 32, 0, true>(args, c, c.row0, BM, q * 32,
+                                                         tmem_base + static_cast<uint32_t>(buf * MX_BN), q, 0, 0,
+                                                         lane, &tfull[buf], use, abort_flag, sm, MX_BN)) {
+                fail();
+                break;
+            }
+            if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
+        }
+    } else {
+        // ------------------------------------------------ E2M1 -> E4M3 unpack into the K-major B tile
+        // Per pass a warp takes 8 weight rows x 4 packed 16-byte chunks (lanes 4r..4r+3:
+        // row r, chunks 0-3), reading 512 contiguous bytes; each chunk (32 k) becomes two
+        // 16-byte E4M3 chunks at the row's swizzled positions.
+        const int ut = threadIdx.x - (2 + Cfg::EPI_WARPS) * 32;   // 0..127
+        const int qc = ut & 3;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < T && ok; t += gridDim.x) {
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!ptx::mbar_wait(&pfull[stage], phase, abort_flag)) {
+                    fail();
+                    ok = false;
+                    break;
+                }
+                const uint8_t *pk = smem_p + stage * Cfg::P_BYTES;
+                uint8_t *bb = smem_b + stage * Cfg::B_BYTES;
+#pragma unroll
+                for (int it = 0; it < 4; ++it) {
+                    const int r = (ut >> 2) + 32 * it;    // weight row (output column) in the tile
+                    const uint4 w = *reinterpret_cast<const uint4 *>(pk + r * (BK / 2) + qc * 16);
+                    uint4 o0, o1;
+                    e2m1x8_to_e4m3(w.x, o0.x, o0.y);
+                    e2m1x8_to_e4m3(w.y, o0.z, o0.w);
+                    e2m1x8_to_e4m3(w.z, o1.x, o1.y);
+                    e2m1x8_to_e4m3(w.w, o1.z, o1.w);
+                    uint8_t *rowp = bb + r * 128;
+                    const int c0 = 2 * qc;                // 16-byte chunk (16 k) inside the 128-byte row
+                    *reinterpret_cast<uint4 *>(rowp + ((c0 ^ (r & 7)) << 4)) = o0;
+                    *reinterpret_cast<uint4 *>(rowp + (((c0 + 1) ^ (r & 7)) << 4)) = o1;
+                }
+                ptx::fence_async_shared();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&full[stage]);
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, 512);
     }
 }
 

@@ -347,6 +347,54 @@ __device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint6
         : "memory");
 }
 
+// ---------------------------------------------------------------- block-scaled MMA (MX formats)
+// Instruction descriptor for kind::mxf8f6f4 with E4M3 A and B, K-major A and B,
+// shape M x N, E8M0 scale factors; a_sf / b_sf pick the byte (the 32-element K
+// block) of each 32-bit scale-factor word that this instruction applies.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N, int a_sf, int b_sf)
+{
+    return (static_cast<uint32_t>(b_sf & 3) << 4)   // B scale-factor byte
+           | (0u << 7)                               // A: E4M3
+           | (0u << 10)                              // B: E4M3
+           | (0u << 15) | (0u << 16)                 // A and B K-major
+           | (static_cast<uint32_t>(N >> 3) << 17)   // N / 8
+           | (1u << 23)                              // scale factors: UE8M0
+           | (static_cast<uint32_t>(M >> 4) << 24)   // M / 16
+           | (static_cast<uint32_t>(a_sf & 3) << 29);   // A scale-factor byte
+}
+
+// D[tmem] (+)= (A * scale_A) * (B * scale_B), E4M3 x E4M3 -> f32, one CTA, one E8M0
+// scale per 32 K-elements of each A row and each B column, read from tensor memory.
+__device__ __forceinline__ void mma_mx_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.scale_vec::1X [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::
+            "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
+// Copy 32 rows x 128 bits from shared memory (descriptor) into tensor memory, the
+// same 32 rows into each of the four 32-lane quarters (4 columns).
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory descriptor without swizzle: 8-row core matrices of 16-byte rows,
+// `sbo_bytes` apart; for the 32 x 16-byte scale-factor blocks of tmem_cp_32x128b_warpx4.
+__device__ __forceinline__ uint64_t smem_desc_noswizzle(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes)
+{
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100
+    return d;                             // layout type 0: no swizzle
+}
+
 // ---------------------------------------------------------------- CTA pairs (cluster of 2, cta_group::2)
 __device__ __forceinline__ uint32_t cluster_ctarank()
 {

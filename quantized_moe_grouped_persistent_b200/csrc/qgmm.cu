@@ -33,6 +33,7 @@ struct DeviceInfo {
     int sms = 0;
     int major = 0;
     bool attr_set[3][3] = {};
+    bool mx_attr_set[3] = {};
     bool pair_attr_set[3][3] = {};
     int pair_clusters[3][3] = {};   // co-resident CTA pairs of the pair kernel, per epilogue and weight kind
 };
@@ -81,7 +82,7 @@ qgmm_status check_problem(const qgmm_problem *p)
 {
     if (!p) return QGMM_ERR_NULL_PTR;
     if (p->weight_type != QGMM_W_INT8 && p->weight_type != QGMM_W_INT4_PACKED_INT32 &&
-        p->weight_type != QGMM_W_FP8_E4M3)
+        p->weight_type != QGMM_W_FP8_E4M3 && p->weight_type != QGMM_W_MXFP4)
         return QGMM_ERR_DTYPE;
     if (p->group_list_type != QGMM_GROUP_CUMSUM && p->group_list_type != QGMM_GROUP_COUNTS) return QGMM_ERR_DTYPE;
     if (p->row_index_type != QGMM_IDX_INT64 && p->row_index_type != QGMM_IDX_INT32) return QGMM_ERR_DTYPE;
@@ -97,6 +98,7 @@ qgmm_status check_problem(const qgmm_problem *p)
     if (p->expected_m_per_expert < 0) return QGMM_ERR_SHAPE;
     if (p->transpose_x2 != 0 && p->transpose_x2 != 1) return QGMM_ERR_SHAPE;
     if (p->transpose_x2 && p->weight_type == QGMM_W_INT4_PACKED_INT32) return QGMM_ERR_UNSUPPORTED;
+    if (p->weight_type == QGMM_W_MXFP4 && !p->transpose_x2) return QGMM_ERR_UNSUPPORTED;   // (e, n, k) only
     if (p->ld_x2 < 0 || p->ld_sb < 0 || p->ld_out < 0 || p->ld_shared < 0) return QGMM_ERR_SHAPE;
     if (p->ld_x2 && (p->ld_x2 < p->n || p->ld_x2 % 32)) return QGMM_ERR_SHAPE;
     if (p->ld_sb && (p->ld_sb < p->n || p->ld_sb % 8)) return QGMM_ERR_SHAPE;
@@ -192,7 +194,8 @@ Plan make_plan(const qgmm_problem *p, int sms, int epi)
     // single CTAs.  int4 weights run on single CTAs unless QGMM_PAIR_W4=1: the pair
     // form (each CTA unpacks its own 128-column half) is exact but measured slower
     // (W4A8 at 256 and 512 rows per expert: 1.22 / 2.07 ms against 0.89 / 1.64 ms).
-    pl.pair = pl.tile_rows == 128 && env_int("QGMM_PAIR", 1) != 0 &&
+    if (p->weight_type == QGMM_W_MXFP4) pl.tile_rows = 128;   // the MX kernel's tile: 128 x 128
+    pl.pair = pl.tile_rows == 128 && env_int("QGMM_PAIR", 1) != 0 && p->weight_type != QGMM_W_MXFP4 &&
               (p->weight_type != QGMM_W_INT4_PACKED_INT32 || env_int("QGMM_PAIR_W4", 0) != 0);
     const int rows_per_tile = pl.pair ? 256 : pl.tile_rows;
     const int64_t max_mt = (p->m + rows_per_tile - 1) / rows_per_tile + p->e;
@@ -240,7 +243,18 @@ qgmm_status make_maps(const qgmm_problem *p, const int8_t *x1, const void *x2, i
     }
     const cuuint64_t ld = cuuint64_t(ld_x2(p));
     const bool bytes = p->weight_type != QGMM_W_INT4_PACKED_INT32;   // int8 or E4M3: one byte per element
-    if (bytes && p->transpose_x2) {
+    if (p->weight_type == QGMM_W_MXFP4) {
+        // E2M1 pairs (e, n, k/2): a box of 64 bytes (128 k) x 128 n-rows, unswizzled
+        const cuuint64_t kb = cuuint64_t(p->k / 2);
+        const cuuint64_t gdim[3] = {kb, cuuint64_t(p->n), cuuint64_t(p->e)};
+        const cuuint64_t gstride[2] = {kb, kb * ld};
+        const cuuint32_t box[3] = {cuuint32_t(BK / 2), cuuint32_t(MX_BN), 1};
+        const cuuint32_t es[3] = {1, 1, 1};
+        if (enc(mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(x2), gdim, gstride, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return QGMM_ERR_CUDA;
+    } else if (bytes && p->transpose_x2) {
         // (e, n, k): K-major B, a box of 128 K bytes x 128 n-rows -- the x1 tile's layout
         const cuuint64_t gdim[3] = {cuuint64_t(p->k), cuuint64_t(p->n), cuuint64_t(p->e)};
         const cuuint64_t gstride[2] = {cuuint64_t(p->k), cuuint64_t(p->k) * ld};
@@ -271,6 +285,36 @@ qgmm_status make_maps(const qgmm_problem *p, const int8_t *x1, const void *x2, i
             return QGMM_ERR_CUDA;
     }
     return QGMM_OK;
+}
+
+template <int EPI>
+qgmm_status launch_mx_t(DeviceInfo *dev, const Plan &pl, const CUtensorMap &ma, const CUtensorMap &mb,
+                        const GemmArgs &a, cudaStream_t st)
+{
+    auto kern = grouped_gemm_mx_kernel<EPI>;
+    const size_t smem = MxCfg::SMEM_BYTES;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!dev->mx_attr_set[EPI]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+                return QGMM_ERR_CUDA;
+            dev->mx_attr_set[EPI] = true;
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.grid), 1, 1);
+    cfg.blockDim = dim3(MxCfg::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    GemmArgs am = a;
+    am.slab_ntiles = 2 * pl.slab_ntiles;   // the plan counts 256-column tiles, the MX kernel 128-column ones
+    if (cudaLaunchKernelEx(&cfg, kern, ma, mb, am) != cudaSuccess) return QGMM_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? QGMM_OK : QGMM_ERR_CUDA;
 }
 
 // Weight kinds of the kernel instantiations: int8, packed int4, E4M3.
@@ -410,6 +454,16 @@ qgmm_status launch_gemm(int epi, DeviceInfo *dev, const qgmm_problem *p, const P
                      "qgmm: gemm epi=%d weights=%d pair=%d m=%lld k=%lld n=%lld e=%lld tile_rows=%d slab=%d grid=%d\n",
                      epi, wk, int(pl.pair), (long long)p->m, (long long)p->k, (long long)p->n, (long long)p->e,
                      pl.tile_rows, pl.slab_ntiles, pl.grid);
+    if (p->weight_type == QGMM_W_MXFP4) {
+        Plan pm = pl;
+        const int64_t tiles = ((p->m + BM - 1) / BM + p->e) * (p->n / MX_BN);
+        pm.grid = static_cast<int>(tiles < dev->sms ? tiles : dev->sms);
+        switch (epi) {
+        case EPI_ATOMIC: return launch_mx_t<EPI_ATOMIC>(dev, pm, ma, mb, a, st);
+        case EPI_STORE_Y: return launch_mx_t<EPI_STORE_Y>(dev, pm, ma, mb, a, st);
+        default: return launch_mx_t<EPI_RAW_ACC>(dev, pm, ma, mb, a, st);
+        }
+    }
     if (pl.pair) {
         // Pairs of 128-row half tiles on CTA pairs.  A group's odd last half tile
         // (its final <= 128 rows) goes, by pl.tail_mode (make_plan's choice, or
@@ -494,8 +548,11 @@ qgmm_status finalize_impl(const qgmm_problem *p, const int8_t *x1, const void *x
     if (s != QGMM_OK) return s;
     if (!x1 || !x2 || !group_list || !out || !workspace) return QGMM_ERR_NULL_PTR;
     if (p->shared_bs > 0 && !shared_input) return QGMM_ERR_NULL_PTR;
+    const bool mx = p->weight_type == QGMM_W_MXFP4;
+    if (mx && (!scale || !pertoken_scale)) return QGMM_ERR_NULL_PTR;   // the block scales are required
     if (!aligned16(x1) || !aligned16(x2) || !aligned16(out) || (p->shared_bs > 0 && !aligned16(shared_input)) ||
-        (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || !aligned16(scale) || !aligned16(bias))
+        (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || !aligned16(scale) || !aligned16(bias) ||
+        (mx && !aligned16(pertoken_scale)))
         return QGMM_ERR_ALIGNMENT;
     if (ws_bytes < workspace_bytes(p)) return QGMM_ERR_WORKSPACE_TOO_SMALL;
     DeviceInfo *dev = nullptr;
@@ -513,9 +570,16 @@ qgmm_status finalize_impl(const qgmm_problem *p, const int8_t *x1, const void *x
         return s;
 
     GemmArgs a = base_args(p, group_list, pl, status);
-    a.scale = scale;
-    a.scale_bf16 = p->scale_type == QGMM_SCALE_BF16;
-    a.pts = pertoken_scale;
+    if (mx) {
+        // MxA8W4: scale and pertoken_scale hold the E8M0 block scales of the weights
+        // and of x1; the epilogue's own scale and pertokenScale are then 1
+        a.sfb = static_cast<const uint8_t *>(scale);
+        a.sfa = reinterpret_cast<const uint8_t *>(pertoken_scale);
+    } else {
+        a.scale = scale;
+        a.scale_bf16 = p->scale_type == QGMM_SCALE_BF16;
+        a.pts = pertoken_scale;
+    }
     a.logit = logit;
     a.bias = bias;
     a.row_index = row_index;
@@ -623,6 +687,7 @@ QGMM_API qgmm_status qgmm_debug_accum(const qgmm_problem *p, const int8_t *x1, c
 {
     qgmm_status s = check_problem(p);
     if (s != QGMM_OK) return s;
+    if (p->weight_type == QGMM_W_MXFP4) return QGMM_ERR_DTYPE;   // needs the block scales: qgmm_debug_accum_mx
     if (!x1 || !x2 || !group_list || !acc_out || !workspace) return QGMM_ERR_NULL_PTR;
     if (!aligned16(x1) || !aligned16(x2) || !aligned16(acc_out) ||
         (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
@@ -644,6 +709,35 @@ QGMM_API qgmm_status qgmm_debug_accum(const qgmm_problem *p, const int8_t *x1, c
     GemmArgs a = base_args(p, group_list, pl, status);
     a.acc_out = acc_out;
     return launch_gemm(EPI_RAW_ACC, dev, p, pl, ma, mb, mb_tail, a, st);
+}
+
+QGMM_API qgmm_status qgmm_debug_accum_mx(const qgmm_problem *p, const uint8_t *x1, const uint8_t *sfa,
+                                         const void *x2, const uint8_t *sfb, const int64_t *group_list,
+                                         float *acc_out, void *workspace, size_t ws_bytes, void *cuda_stream)
+{
+    qgmm_status s = check_problem(p);
+    if (s != QGMM_OK) return s;
+    if (p->weight_type != QGMM_W_MXFP4) return QGMM_ERR_DTYPE;
+    if (!x1 || !sfa || !x2 || !sfb || !group_list || !acc_out || !workspace) return QGMM_ERR_NULL_PTR;
+    if (!aligned16(x1) || !aligned16(x2) || !aligned16(acc_out) || !aligned16(sfa) || !aligned16(sfb) ||
+        (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+        return QGMM_ERR_ALIGNMENT;
+    if (ws_bytes < kAlign) return QGMM_ERR_WORKSPACE_TOO_SMALL;
+    DeviceInfo *dev = nullptr;
+    if ((s = device_info(&dev)) != QGMM_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    uint32_t *status = static_cast<uint32_t *>(workspace);
+    const Plan pl = make_plan(p, dev->sms, EPI_RAW_ACC);
+    CUtensorMap ma, mb;
+    if ((s = make_maps(p, reinterpret_cast<const int8_t *>(x1), x2, pl.tile_rows, 32, &ma, &mb)) != QGMM_OK)
+        return s;
+    clear_status_kernel<<<1, 1, 0, st>>>(status);
+    if (cudaGetLastError() != cudaSuccess) return QGMM_ERR_CUDA;
+    GemmArgs a = base_args(p, group_list, pl, status);
+    a.acc_out = reinterpret_cast<int32_t *>(acc_out);
+    a.sfa = sfa;
+    a.sfb = sfb;
+    return launch_gemm(EPI_RAW_ACC, dev, p, pl, ma, mb, mb, a, st);
 }
 
 QGMM_API qgmm_status qgmm_per_token_quant(const uint16_t *x_bf16, int64_t rows, int64_t k, int8_t *x1_out,

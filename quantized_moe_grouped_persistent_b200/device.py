@@ -12,7 +12,7 @@ import numpy as np
 import torch
 
 from . import (QGMM_IDX_INT32, QGMM_IDX_INT64, QGMM_SCALE_BF16, QGMM_SCALE_F32, QGMM_W_FP8_E4M3,
-               QGMM_W_INT4_PACKED_INT32, QGMM_W_INT8,
+               QGMM_W_INT4_PACKED_INT32, QGMM_W_INT8, QGMM_W_MXFP4, debug_accum_mx, per_token_quant_mxfp8,
                debug_accum, device_status, finalize, finalize_workspace, make_problem, per_token_quant)
 
 
@@ -33,12 +33,17 @@ class DeviceProblem:
         self.m, self.k, self.n, self.e = p.m, p.k, p.n, p.e
         self.output_bs = p.output_bs
         self.weight_type = {"int8": QGMM_W_INT8, "int4": QGMM_W_INT4_PACKED_INT32,
-                            "fp8": QGMM_W_FP8_E4M3}[p.weight]
+                            "fp8": QGMM_W_FP8_E4M3, "mxfp4": QGMM_W_MXFP4}[p.weight]
+        self.mx = p.weight == "mxfp4"
         self.group_list_type = p.group_list_type
         self.expected_m_per_expert = expected_m_per_expert
         dev = self.device
         self.prologue = p.x1 is None
-        if self.prologue:
+        if self.prologue and self.mx:     # the per-32-group FP8 cast: E4M3 codes and E8M0 scales
+            self.x_bf16 = to_device(p.x_bf16, dev)
+            self.x1 = torch.empty((p.m, p.k), dtype=torch.uint8, device=dev)
+            self.pts = torch.empty((p.m, p.k // 32), dtype=torch.uint8, device=dev)
+        elif self.prologue:
             self.x_bf16 = to_device(p.x_bf16, dev)
             self.x1 = torch.empty((p.m, p.k), dtype=torch.int8, device=dev)
             self.pts = torch.empty(p.m, dtype=torch.float32, device=dev)
@@ -88,7 +93,9 @@ class DeviceProblem:
         return self._ws[key]
 
     def quantize(self, stream=None):
-        if self.prologue:
+        if self.prologue and self.mx:
+            per_token_quant_mxfp8(self.x_bf16, self.x1, self.pts, stream=stream)
+        elif self.prologue:
             per_token_quant(self.x_bf16, self.x1, self.pts, stream=stream)
 
     def run(self, deterministic: bool = False, stream=None, out: Optional[torch.Tensor] = None,
@@ -101,6 +108,11 @@ class DeviceProblem:
         return out
 
     def accum(self, stream=None) -> torch.Tensor:
+        if self.mx:   # block-scaled f32 accumulators
+            acc = torch.zeros((self.m, self.n), dtype=torch.float32, device=self.device)
+            debug_accum_mx(self.problem(False), self.x1, self.pts, self.x2, self.scale, self.group_list, acc,
+                           self.workspace(False), stream=stream)
+            return acc
         acc = torch.zeros((self.m, self.n), dtype=torch.int32, device=self.device)
         debug_accum(self.problem(False), self.x1, self.x2, self.group_list, acc, self.workspace(False),
                     stream=stream)

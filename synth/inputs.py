@@ -38,7 +38,7 @@ class Spec:
     routing: str          # 'top_normal' | 'zipf' | 'uniform' | 'dirichlet'
     routing_param: float
     group_list_type: int  # 0 = cumulative ends, 1 = per-group counts
-    weight: str           # 'int8' | 'int4' | 'fp8' (x1 and x2 FLOAT8 E4M3FN)
+    weight: str           # 'int8' | 'int4' | 'fp8' (x1 and x2 FLOAT8 E4M3FN) | 'mxfp4' (MxA8W4)
     bias: bool
     shared: bool
     shared_offset: int
@@ -64,6 +64,11 @@ CONFIGS = {
     "fp8_prefill": Spec(6, 16384, 8, 256, 2048, 7168, "dirichlet", 0.3, 0, "fp8", False, True, 0, False,
                         "tokens=16384 topK=8 m=131072 e=256 k=2048 n=7168; x1 and x2 FLOAT8 E4M3FN, "
                         "Dirichlet(0.3) popularity, bf16 sharedInput at offset 0"),
+    # page 1's Atlas 350 MxA8W4 mode on the W4A8 workload's shapes: bf16 activations
+    # through the per-32-group FP8 cast, FP4 E2M1 weights (e, n, k) with E8M0 block scales
+    "w4a8_mx": Spec(7, 4096, 8, 128, 2048, 7168, "uniform", 0.0, 0, "mxfp4", True, False, 0, True,
+                    "tokens=4096 topK=8 m=32768 e=128 k=2048 n=7168; MxA8W4: bf16 activations cast to E4M3 "
+                    "with E8M0 scales per 32, FP4 E2M1 weights (e, n, k) with E8M0 scales per 32, bias"),
 }
 
 
@@ -199,16 +204,24 @@ def make_problem(name: str, *, tokens: Optional[int] = None, e: Optional[int] = 
         x2 = rng.integers(-127, 128, size=(e, k, n), dtype=np.int8)
     elif spec.weight == "fp8":
         x2 = e4m3_codes_normal(rng, (e, k, n), 0.5)
+    elif spec.weight == "mxfp4":
+        x2 = rng.integers(0, 256, size=(e, n, k // 2), dtype=np.uint8)     # every nibble uniform over the 16 codes
     else:
         x2 = rng.integers(0, 2 ** 32, size=(e, k, n // 8), dtype=np.uint32).view(np.int32)
-    scale = rng.uniform(1e-3, 1e-2, size=(e, n)).astype(np.float32)
+    if spec.weight == "mxfp4":      # E8M0 weight scales per 32 k: 2^-9 .. 2^0
+        scale = rng.integers(118, 128, size=(e, n, k // 32), dtype=np.uint8)
+    else:
+        scale = rng.uniform(1e-3, 1e-2, size=(e, n)).astype(np.float32)
     bias = rng.normal(0.0, 0.01, size=(e, n)).astype(np.float32) if spec.bias else None
     shared = bf16_bits_normal(rng, (tokens, n)) if spec.shared else None
-    return Problem(name=name, tokens=tokens, topk=topk, m=m, e=e, k=k, n=n, output_bs=tokens,
-                   group_list_type=gtype, weight=spec.weight, x1=x1, x_bf16=x_bf16, x2=x2,
-                   scale=scale, pertoken_scale=pts, group_list=group_list, counts=counts,
-                   logit=logit, row_index=row_index, bias=bias, shared=shared,
-                   shared_offset=spec.shared_offset)
+    pr = Problem(name=name, tokens=tokens, topk=topk, m=m, e=e, k=k, n=n, output_bs=tokens,
+                 group_list_type=gtype, weight=spec.weight, x1=x1, x_bf16=x_bf16, x2=x2,
+                 scale=scale, pertoken_scale=pts, group_list=group_list, counts=counts,
+                 logit=logit, row_index=row_index, bias=bias, shared=shared,
+                 shared_offset=spec.shared_offset)
+    if spec.weight == "mxfp4":
+        pr.transpose_x2 = True      # the MX weights are (e, n, k), as page 1 requires in that mode
+    return pr
 
 
 def sample_rows(rng_seed: int, limit: int, count: int) -> np.ndarray:

@@ -23,7 +23,8 @@ def _declared_functions():
 def test_header_declares_the_abi():
     assert _declared_functions() == sorted([
         "qgmm_finalize_workspace", "qgmm_finalize", "qgmm_finalize_profiled", "qgmm_per_token_quant",
-        "qgmm_per_token_quant_mxfp8", "qgmm_debug_accum", "qgmm_device_status", "qgmm_finalize_static_scratch",
+        "qgmm_per_token_quant_mxfp8", "qgmm_debug_accum", "qgmm_debug_accum_mx", "qgmm_device_status",
+        "qgmm_finalize_static_scratch",
         "qgmm_status_string",
         "qgmm_finalize_launches", "qgmm_plan"])
 
@@ -115,9 +116,9 @@ def test_workspace_sizes(qgmm):
     (dict(e=0), "SHAPE"), (dict(e=1025), "SHAPE"), (dict(output_bs=0), "SHAPE"),
     (dict(shared_bs=33), "SHAPE"), (dict(shared_bs=8, shared_offset=25), "SHAPE"),
     (dict(shared_offset=-1), "SHAPE"), (dict(expected_m_per_expert=-1), "SHAPE"),
-    (dict(weight_type=3), "DTYPE"), (dict(weight_type=-1), "DTYPE"), (dict(group_list_type=2), "DTYPE"), (dict(row_index_type=5), "DTYPE"),
+    (dict(weight_type=4), "DTYPE"), (dict(weight_type=-1), "DTYPE"), (dict(group_list_type=2), "DTYPE"), (dict(row_index_type=5), "DTYPE"),
     (dict(scale_type=2), "DTYPE"), (dict(scale_type=-1), "DTYPE"),
-    (dict(transpose_x2=1, weight_type=1), "UNSUPPORTED"),
+    (dict(transpose_x2=1, weight_type=1), "UNSUPPORTED"), (dict(weight_type=3), "UNSUPPORTED"),
 ])
 def test_stage_one_rejects(qgmm, kw, code):
     rc, _ = _ws(qgmm, _prob(qgmm, **kw))
