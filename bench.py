@@ -107,11 +107,17 @@ def algorithmic_bytes(p):
     scale/bias rows), x1 (or the bf16 activations), the per-row vectors, the output
     written once, and the sharedInput read once."""
     used = int((p.counts > 0).sum())
-    w_bytes = p.k * p.n // 2 if p.weight == "int4" else p.k * p.n
-    per_expert = w_bytes + 4 * p.n + (4 * p.n if p.bias is not None else 0)
+    w_bytes = p.k * p.n // 2 if p.weight in ("int4", "mxfp4") else p.k * p.n
+    scale_bytes = p.n * p.k // 32 if p.weight == "mxfp4" else 4 * p.n     # E8M0 per 32 k, or f32 per column
+    per_expert = w_bytes + scale_bytes + (4 * p.n if p.bias is not None else 0)
     b = used * per_expert
     m = total_rows(p)
-    b += m * p.k if p.x1 is not None else m * p.k * 2 + m * p.k + 4 * m   # prologue reads bf16, writes int8 + scale
+    if p.x1 is not None:
+        b += m * p.k
+    elif p.weight == "mxfp4":   # the FP8 cast reads bf16, writes E4M3 + a scale byte per 32; the GEMM reads both
+        b += m * p.k * 2 + 2 * (m * p.k + m * p.k // 32)
+    else:                       # the int8 prologue reads bf16, writes int8 + a scale; the GEMM reads both
+        b += m * p.k * 2 + m * p.k + 4 * m
     b += m * (4 + 4 + p.row_index.dtype.itemsize)
     b += p.output_bs * p.n * 4
     if p.shared is not None:
@@ -327,7 +333,7 @@ def line_unit(workload, p):
     of the ops is credited the same fraction of the workload's algorithmic bytes)."""
     if workload == "decode":
         return "GB/s", 1e3 * algorithmic_bytes(p) / int_ops(p)
-    if p.weight == "fp8":
+    if p.weight in ("fp8", "mxfp4"):
         return "TFLOPS", 1.0
     return "TOPS", 1.0
 
@@ -516,18 +522,19 @@ def main():
         torch.cuda.empty_cache()
     if world == 1 and not args.no_extras and args.workload == "large_prefill":
         # the other prefill-shaped workloads, atomic combine, with their own int8 roofline
-        for name in ("mid_prefill", "w4a8_prologue"):
+        for name in ("mid_prefill", "w4a8_prologue", "w4a8_mx"):
             ps = make_problem(name)
             ds = DeviceProblem(ps)
             ds.run()
             torch.cuda.synchronize()
             sms_, sgemm = time_steps(ds, max(10, args.steps), 3, False)
             sops = int_ops(ps)
+            sunit, _ = line_unit(name, ps)
             extras[name] = {
                 "workload": f"{name}: " + CONFIGS[name].description + "; atomic combine",
-                "value": sops / (sms_ * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": sms_, "gemm_ms": sgemm,
+                "value": sops / (sms_ * 1e-3) / 1e12, "unit": sunit, "ms_per_step": sms_, "gemm_ms": sgemm,
                 "roofline": {"bound": "tensor", "achieved": sops / (sgemm * 1e-3) / 1e12, "peak": int8_peak,
-                             "unit": "TOPS", "frac": sops / (sgemm * 1e-3) / 1e12 / int8_peak,
+                             "unit": sunit, "frac": sops / (sgemm * 1e-3) / 1e12 / int8_peak,
                              "traffic": committed_traffic(name), "kernel_ms": sgemm},
             }
             del ds

@@ -348,14 +348,15 @@ __device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint6
 }
 
 // ---------------------------------------------------------------- block-scaled MMA (MX formats)
-// Instruction descriptor for kind::mxf8f6f4 with E4M3 A and B, K-major A and B,
-// shape M x N, E8M0 scale factors; a_sf / b_sf pick the byte (the 32-element K
-// block) of each 32-bit scale-factor word that this instruction applies.
-__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N, int a_sf, int b_sf)
+// Instruction descriptor for kind::mxf8f6f4 with E4M3 A and an E4M3 or E2M1 B
+// (b_e2m1), K-major A and B, shape M x N, E8M0 scale factors; a_sf / b_sf pick the
+// byte (the 32-element K block) of each 32-bit scale-factor word that this
+// instruction applies.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N, int a_sf, int b_sf, bool b_e2m1 = false)
 {
     return (static_cast<uint32_t>(b_sf & 3) << 4)   // B scale-factor byte
            | (0u << 7)                               // A: E4M3
-           | (0u << 10)                              // B: E4M3
+           | ((b_e2m1 ? 5u : 0u) << 10)              // B: E4M3 (0) or E2M1 (5)
            | (0u << 15) | (0u << 16)                 // A and B K-major
            | (static_cast<uint32_t>(N >> 3) << 17)   // N / 8
            | (1u << 23)                              // scale factors: UE8M0
