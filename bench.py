@@ -43,6 +43,8 @@ TRAFFIC_SUMMARY = {
     "large_prefill": "profiles/grouped_gemm_large_prefill.md",
     "decode": "profiles/grouped_gemm_decode.md",
     "w4a8_prologue": "profiles/grouped_gemm_w4a8.md",
+    "w4a8_mx": "profiles/grouped_gemm_w4a8_mx.md",
+    "mid_prefill": "profiles/grouped_gemm_mid_prefill.md",
 }
 
 
