@@ -12,6 +12,7 @@ Entry points mirror the C ABI:
     per_token_quant(x_bf16, x1_out, scale_out)
     debug_accum(problem, x1, x2, group_list, acc_out, workspace)
     device_status(workspace) -> QGMM_DEV_* flags
+    ep_plan(world, e, send_counts, recv_counts) -> offsets of the expert-parallel dispatch
 """
 from __future__ import annotations
 
@@ -54,7 +55,7 @@ QGMM_DEV_TIMEOUT = 1 << 4
 EXPORTS = ("qgmm_finalize_workspace", "qgmm_finalize_launches", "qgmm_plan", "qgmm_finalize", "qgmm_finalize_profiled",
            "qgmm_per_token_quant", "qgmm_per_token_quant_mxfp8", "qgmm_debug_accum", "qgmm_debug_accum_mx",
            "qgmm_device_status",
-           "qgmm_finalize_static_scratch", "qgmm_status_string")
+           "qgmm_finalize_static_scratch", "qgmm_ep_plan", "qgmm_status_string")
 
 
 class QgmmProblem(C.Structure):
@@ -106,6 +107,7 @@ def lib():
         L.qgmm_debug_accum_mx.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, P, P, U, P]
         L.qgmm_device_status.argtypes = [P, C.POINTER(C.c_uint32), P]
         L.qgmm_finalize_static_scratch.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, P, P, P, P, P, P]
+        L.qgmm_ep_plan.argtypes = [C.c_int32, C.c_int32, P, P, P, P, P, P]
         L.qgmm_status_string.argtypes = [C.c_int]
         L.qgmm_status_string.restype = C.c_char_p
         for name in EXPORTS[:-1]:
@@ -254,3 +256,26 @@ def finalize_static_scratch(problem: QgmmProblem, x1, x2, scale, pertoken_scale,
                                             _ptr(pertoken_scale), _ptr(group_list), _ptr(logit), _ptr(row_index),
                                             _ptr(bias), _ptr(shared_input), _ptr(out), _stream(stream))
     _check(rc, "qgmm_finalize_static_scratch")
+
+
+def ep_plan(world: int, e: int, send_counts, recv_counts) -> dict:
+    """Offsets of one card's expert-parallel dispatch (``qgmm_ep_plan``, a host call).
+
+    ``send_counts`` / ``recv_counts`` are ``world * e`` row counts, chunk (card, expert)
+    at ``card * e + expert``.  Returns ``send_offsets`` and ``recv_offsets`` (int64
+    numpy arrays of the same shape; receive offsets are rows of the permuted,
+    expert-major buffer), ``group_counts`` (rows per local expert) and ``bsk`` / ``a``.
+    """
+    import numpy as np
+    sc = np.ascontiguousarray(np.asarray(send_counts, dtype=np.int64).reshape(-1))
+    rc_ = np.ascontiguousarray(np.asarray(recv_counts, dtype=np.int64).reshape(-1))
+    if sc.size != world * e or rc_.size != world * e:
+        raise QgmmError(QGMM_ERR_SHAPE, "qgmm_ep_plan")
+    so = np.zeros(world * e, np.int64)
+    ro = np.zeros(world * e, np.int64)
+    gc = np.zeros(max(e, 1), np.int64)
+    tot = np.zeros(2, np.int64)
+    ptr = lambda a: a.ctypes.data_as(C.c_void_p)
+    _check(lib().qgmm_ep_plan(int(world), int(e), ptr(sc), ptr(rc_), ptr(so), ptr(ro), ptr(gc), ptr(tot)),
+           "qgmm_ep_plan")
+    return {"send_offsets": so, "recv_offsets": ro, "group_counts": gc[:e], "bsk": int(tot[0]), "a": int(tot[1])}

@@ -1,5 +1,5 @@
 """Compile the sm_100a CUDA libraries in-tree: quantized_moe_grouped_persistent_b200/libqgmm.so
-(the op) and libqgmm_probe.so (the int8 tensor-rate probe the benchmark reads its roofline against)."""
+(the op, with the expert-parallel dispatch plan) and libqgmm_probe.so (the int8 tensor-rate probe the benchmark reads its roofline against)."""
 from __future__ import annotations
 
 import glob
@@ -10,9 +10,9 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libqgmm.so")
-MAIN = os.path.join(HERE, "csrc", "qgmm.cu")
+MAIN = [os.path.join(HERE, "csrc", "qgmm.cu"), os.path.join(HERE, "csrc", "ep_plan.cu")]
 PROBE_LIB = os.path.join(HERE, "libqgmm_probe.so")
-PROBE = os.path.join(HERE, "csrc", "probe_mma.cu")
+PROBE = [os.path.join(HERE, "csrc", "probe_mma.cu")]
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
     "-Xcompiler", "-fPIC,-fvisibility=hidden", "-shared",
@@ -23,14 +23,14 @@ def sources():
     return sorted(glob.glob(os.path.join(HERE, "csrc", "*"))) + sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
-def _compile(src: str, lib: str, force: bool, verbose: bool) -> str:
+def _compile(srcs: list, lib: str, force: bool, verbose: bool) -> str:
     if not force and os.path.exists(lib):
         newest = max(os.path.getmtime(s) for s in sources())
         if os.path.getmtime(lib) >= newest:
             return lib
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = lib + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), src, "-o", tmp]
+    cmd = [nvcc, *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), *srcs, "-o", tmp]
     subprocess.run(cmd, check=True)
     os.replace(tmp, lib)
     return lib

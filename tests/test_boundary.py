@@ -1,5 +1,5 @@
 """The C ABI boundary, on the host: the library loads, exports every function
-``include/qgmm.h`` declares, its struct layout matches the binding, and every
+``include/qgmm.h`` and ``include/qgmm_ep.h`` declare, its struct layout matches the binding, and every
 host-side check returns its documented code before anything is launched.
 
 No test here reaches a kernel launch: each call fails a host check first.
@@ -13,10 +13,11 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "qgmm.h")
+EP_HEADER = os.path.join(ROOT, "include", "qgmm_ep.h")
 
 
-def _declared_functions():
-    text = open(HEADER).read()
+def _declared_functions(headers=(HEADER, EP_HEADER)):
+    text = "".join(open(h).read() for h in headers)
     return sorted(set(re.findall(r"^(?:qgmm_status|const char \*)\s*(qgmm_\w+)\s*\(", text, re.M)))
 
 
@@ -26,7 +27,8 @@ def test_header_declares_the_abi():
         "qgmm_per_token_quant_mxfp8", "qgmm_debug_accum", "qgmm_debug_accum_mx", "qgmm_device_status",
         "qgmm_finalize_static_scratch",
         "qgmm_status_string",
-        "qgmm_finalize_launches", "qgmm_plan"])
+        "qgmm_finalize_launches", "qgmm_plan", "qgmm_ep_plan"])
+    assert _declared_functions((EP_HEADER,)) == ["qgmm_ep_plan"]
 
 
 def test_library_exports_every_declared_symbol(qgmm):
