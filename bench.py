@@ -395,7 +395,8 @@ def reference_arm(args, p, spec_desc):
         total_ops += 2.0 * float(counts[rows].sum()) * p.k * p.n
     unit, factor = line_unit(args.workload, p)
     value = factor * total_ops / total_t / 1e12
-    sample = f"{nrows} of {p.output_bs} output rows per step (every contributing source row in full), {args.steps} steps"
+    sample = (f"{nrows} of {p.output_bs} output rows per step (every contributing source row in full), "
+              f"{args.steps} steps")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
@@ -408,6 +409,123 @@ def reference_arm(args, p, spec_desc):
 
 
 # ----------------------------------------------------------------------------- main
+def time_ep(mode, world, rank, dist, steps, warmup, int8_peak):
+    """The expert-parallel step of page "aclnnAlltoAllvQuantGroupedMatMul" on this
+    rank's card: AlltoAllv (NCCL send/recv between ranks; device copies for a card's
+    own chunks) with the permute folded in, the grouped matmul over the card's
+    experts and the shared expert's matmul on a side stream.  Inputs resident on the
+    device; per-card work fixed (weak scaling).  Returns a dict for the JSON line."""
+    import numpy as np
+    import torch
+    from quantized_moe_grouped_persistent_b200 import finalize_launches
+    from quantized_moe_grouped_persistent_b200.ep import EpGroupedMatmul
+    from synth.ep import EP_BENCH, make_ep_problem
+    cfg = dict(EP_BENCH)
+    e = min(cfg.pop("e"), 256 // world)            # page 2: e * epWorldSize <= 256
+    p = make_ep_problem(world=world, e=e, mode=mode, ranks=[rank], **cfg)
+    c = p.cards[rank]
+    m = EpGroupedMatmul(mode, world, rank, e, c.w, c.w_scale, c.mm_w, c.mm_w_scale)
+    dev = m.device
+    x = torch.from_numpy(c.x).to(dev)
+    mm_x = torch.from_numpy(c.mm_x).to(dev)
+    if mode == "mx":
+        xs = torch.from_numpy(np.ascontiguousarray(c.x_scale)).to(dev)
+        mms = torch.from_numpy(np.ascontiguousarray(c.mm_x_scale)).to(dev)
+    else:
+        xs, mms = c.x_scale, c.mm_x_scale
+    stream = torch.cuda.current_stream()
+
+    def step(events=None, check=False):
+        return m.forward(x, xs, c.send_counts, c.recv_counts, mm_x, mms, check_counts=check, events=events)
+
+    res = step(check=True)                          # first call: counts checked across ranks, workspaces
+    torch.cuda.synchronize()
+    a = int(res["permute_out"].shape[0])
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for b, en in ev:
+        b.record(stream)
+        en.record(stream)
+    for _ in range(warmup):
+        step(ev[0])
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    marks[0].record(stream)
+    for s_ in range(steps):
+        step(ev[s_])
+        marks[s_ + 1].record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ms = marks[0].elapsed_time(marks[-1]) / steps
+    gemm_ms = sum(b.elapsed_time(en) for b, en in ev) / steps
+    gmm_flops = 2.0 * a * p.h1 * p.n1
+    mm_flops = 2.0 * p.tokens * p.h2 * p.n2
+    flops = gmm_flops + mm_flops
+    ms_max, gemm_max = max_over_ranks([ms, gemm_ms], dist, device="cuda")
+    total = flops
+    if dist is not None:
+        t = torch.tensor([flops], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t)
+        total = float(t.item())
+    launches = (finalize_launches(m._problem(a, p.h1, p.n1, e))
+                + finalize_launches(m._problem(p.tokens, p.h2, p.n2, 1)))
+    achieved = gmm_flops / (gemm_ms * 1e-3) / 1e12
+    quant = "E4M3 x E2M1 with E8M0 scales per 32" if mode == "mx" else "E4M3, per-tensor scales"
+    return {
+        "workload": (f"ep_{mode}: page 2's AlltoAllv + grouped matmul + shared-expert matmul, {world} card(s), "
+                     f"e={e} experts per card, BS={p.tokens} tokens per card, topK={p.topk}, H1={p.h1}, N1={p.n1}, "
+                     f"H2={p.h2}, N2={p.n2}; {quant}"),
+        "value": total / (ms_max * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms_max,
+        "gemm_ms": gemm_max, "rows_received_rank0": a, "flops_rank0": flops,
+        "roofline": {"bound": "tensor", "kernel": "grouped GEMM over the card's experts", "achieved": achieved,
+                     "peak": int8_peak, "unit": "TFLOPS", "frac": achieved / int8_peak, "traffic": None,
+                     "kernel_ms": gemm_ms},
+        "gpu_launches_per_step": launches,
+    }
+
+
+def ep_main(args, world, rank, local_rank):
+    """``--workload ep_mx`` / ``ep_pertensor``: the expert-parallel step as the line."""
+    mode = args.workload[len("ep_"):]
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps({"impl": "reference", "unavailable": "the expert-parallel workload has no timed CPU "
+                              "leg; its oracle runs in the tests only"}), flush=True)
+        return
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist = tdist
+    else:
+        torch.cuda.set_device(0)
+    peaks = load_peaks()
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    r = time_ep(mode, world, rank, dist, args.steps, args.warmup, 2.0 * peaks["bf16"])
+    clocks = sampler.stop()
+    if rank == 0:
+        line = {"metric": "expert-parallel AlltoAllv + quantised grouped matmul + shared-expert matmul TFLOPS",
+                "value": r["value"], "unit": "TFLOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "e4m3", "data": "synthetic",
+                "config": {"workload": r["workload"], "l2": "inputs larger than L2, no flush",
+                           "parallelism": f"expert parallel over {world} GPU(s)"},
+                "roofline": r["roofline"], "gpu_launches": r["gpu_launches_per_step"] * args.steps,
+                "clocks": clocks, "e2e": None}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse_args()
     from synth import CONFIGS, make_problem
@@ -415,6 +533,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.workload in ("ep_mx", "ep_pertensor"):
+        return ep_main(args, world, rank, local_rank)
     spec = CONFIGS[args.workload]
     mode = "deterministic" if args.deterministic else "atomic"
     spec_desc = f"{args.workload}: {spec.description}; {mode} combine"
@@ -541,6 +661,8 @@ def main():
             }
             del ds
             torch.cuda.empty_cache()
+        extras["ep_mx"] = time_ep("mx", 1, 0, None, max(10, args.steps), 3, int8_peak)
+        torch.cuda.empty_cache()
 
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:

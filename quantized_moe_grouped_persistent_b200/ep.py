@@ -31,7 +31,7 @@ import numpy as np
 import torch
 
 from . import (QGMM_GROUP_COUNTS, QGMM_W_FP8_E4M3, QGMM_W_MXFP4, QgmmError, QGMM_ERR_SHAPE, ep_plan, finalize,
-               finalize_workspace, make_problem)
+               finalize_profiled, finalize_workspace, make_problem)
 
 MODES = ("pertensor", "mx")
 
@@ -42,6 +42,14 @@ def _dev(a, device):
     if isinstance(a, torch.Tensor):
         return a.to(device)
     return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def _counts_to(device, counts) -> torch.Tensor:
+    """Host counts -> a device int64 tensor, through pinned memory without a host wait."""
+    host = torch.tensor(np.asarray(counts, np.int64).reshape(-1), dtype=torch.int64)
+    if device.type != "cuda":
+        return host
+    return host.pin_memory().to(device, non_blocking=True)
 
 
 def _scalar(v) -> float:
@@ -155,10 +163,14 @@ class EpGroupedMatmul:
             self._ws[key] = ws
         return ws
 
-    def _matmul(self, key, x, x_scale, group_list, w, w_scale, k, n, e, out, stream):
+    def _matmul(self, key, x, x_scale, group_list, w, w_scale, k, n, e, out, stream, events=None):
         prob = self._problem(int(x.shape[0]), k, n, e)
-        finalize(prob, x, w, w_scale, x_scale, group_list, None, None, None, None, out, self._workspace(prob, key),
-                 stream=stream)
+        ws = self._workspace(prob, key)
+        if events is None:
+            finalize(prob, x, w, w_scale, x_scale, group_list, None, None, None, None, out, ws, stream=stream)
+        else:         # the caller's two CUDA events, recorded around the grouped GEMM's launch
+            finalize_profiled(prob, x, w, w_scale, x_scale, group_list, None, None, None, None, out, ws, events[0],
+                              events[1], stream=stream)
 
     # -- the three parts of one call ---------------------------------------------------
     def shared(self, mm_x, mm_x_scale):
@@ -173,7 +185,7 @@ class EpGroupedMatmul:
             mm_scale = torch.full((bs,), _scalar(mm_x_scale), dtype=torch.float32, device=dev)
         else:
             mm_scale = _dev(mm_x_scale, dev)
-        mm_gl = torch.tensor([bs], dtype=torch.int64, device=dev)
+        mm_gl = _counts_to(dev, [bs])
         mm_y = torch.empty((bs, self.n2), dtype=torch.float32, device=dev)
         if self._side is None:
             self._side = torch.cuda.Stream(dev)
@@ -213,27 +225,28 @@ class EpGroupedMatmul:
         self.exchange.run([(x, permute_out), (send_scale, permute_scale)], plan, send_counts, recv_counts)
         return permute_out, (permute_scale.reshape(-1) if self.mode == "pertensor" else permute_scale), plan
 
-    def grouped(self, permute_out, permute_scale, group_counts):
-        """The grouped matmul over this card's experts: f32 [A, n1] (None when A = 0)."""
+    def grouped(self, permute_out, permute_scale, group_counts, events=None):
+        """The grouped matmul over this card's experts: f32 [A, n1] (None when A = 0).
+        ``events``: two CUDA events to record around the grouped GEMM kernel."""
         dev = self.device
         a = int(permute_out.shape[0])
         if a == 0:
             return None
-        gl = torch.from_numpy(np.asarray(group_counts, np.int64).copy()).to(dev)
+        gl = _counts_to(dev, group_counts)
         gmm_y = torch.empty((a, self.n1), dtype=torch.float32, device=dev)
         self._matmul("gmm", permute_out, permute_scale, gl, self.w, self.w_scale, self.h1, self.n1, self.e, gmm_y,
-                     torch.cuda.current_stream(dev))
+                     torch.cuda.current_stream(dev), events)
         return gmm_y
 
     def forward(self, x, x_scale, send_counts, recv_counts, mm_x=None, mm_x_scale=None,
-                check_counts: bool = True) -> dict:
+                check_counts: bool = True, events=None) -> dict:
         """One call: the shared expert's matmul starts on the side stream, then the
         exchange, then the grouped matmul; the current stream then waits for both.
         Returns ``gmm_y`` f32 [A, n1] (None if A = 0), ``mm_y`` f32 [BS, n2] (None
         without a shared expert), ``permute_out``, ``permute_scale``, ``group_counts``."""
         mm_y = self.shared(mm_x, mm_x_scale) if mm_x is not None and self.mm_w is not None else None
         permute_out, permute_scale, plan = self.dispatch(x, x_scale, send_counts, recv_counts, check_counts)
-        gmm_y = self.grouped(permute_out, permute_scale, plan["group_counts"])
+        gmm_y = self.grouped(permute_out, permute_scale, plan["group_counts"], events)
         if mm_y is not None:
             self.join()
         return {"gmm_y": gmm_y, "mm_y": mm_y, "permute_out": permute_out, "permute_scale": permute_scale,

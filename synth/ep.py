@@ -24,7 +24,7 @@ Recipe (random draws and data layout only, none of the operation's arithmetic):
 from __future__ import annotations
 
 from dataclasses import dataclass, field
-from typing import List, Optional
+from typing import List, Optional, Sequence
 
 import numpy as np
 
@@ -37,12 +37,12 @@ EP_SEED_OFFSET = 100
 class EpCard:
     """One card's inputs.  Arrays are host numpy arrays in the op's layouts."""
     rank: int
-    x: np.ndarray                       # E4M3 codes [BSK, h1], send order
+    x: Optional[np.ndarray]             # E4M3 codes [BSK, h1], send order
     x_scale: Optional[np.ndarray]       # pertensor: f32 [1]; mx: E8M0 [BSK, h1/32]
     send_counts: np.ndarray             # int64 [world * e]
     recv_counts: np.ndarray             # int64 [world * e]
-    w: np.ndarray                       # pertensor: E4M3 [e, h1, n1]; mx: E2M1 pairs [e, n1, h1/2]
-    w_scale: np.ndarray                 # pertensor: f32 [1]; mx: E8M0 [e, n1, h1/32]
+    w: Optional[np.ndarray]             # pertensor: E4M3 [e, h1, n1]; mx: E2M1 pairs [e, n1, h1/2]
+    w_scale: Optional[np.ndarray]       # pertensor: f32 [1]; mx: E8M0 [e, n1, h1/32]
     mm_x: Optional[np.ndarray]          # E4M3 [BS, h2]
     mm_x_scale: Optional[np.ndarray]    # pertensor: f32 [1]; mx: E8M0 [BS, h2/32]
     mm_w: Optional[np.ndarray]          # pertensor: E4M3 [h2, n2]; mx: E2M1 pairs [n2, h2/2]
@@ -66,50 +66,59 @@ class EpProblem:
 
 def make_ep_problem(world: int, e: int, tokens: int, topk: int, h1: int, n1: int, h2: int = 0, n2: int = 0,
                     mode: str = "mx", routing: str = "uniform", routing_param: float = 0.0,
-                    seed: Optional[int] = None) -> EpProblem:
+                    seed: Optional[int] = None, ranks: Optional[Sequence[int]] = None) -> EpProblem:
+    """Every card's counts; the activations and weights of the cards in ``ranks``
+    (default all; a card left out has them as None).  One generator draws every
+    card's routing, then card c's data comes from a generator of its own, so a card's
+    data is the same whichever cards are drawn."""
     if mode not in ("pertensor", "mx"):
         raise ValueError(mode)
-    rng = np.random.default_rng(SEED_BASE + EP_SEED_OFFSET if seed is None else seed)
+    base = SEED_BASE + EP_SEED_OFFSET if seed is None else seed
+    rng = np.random.default_rng(base)
     E = world * e
     topk = min(topk, E)
-    sends = []
+    layouts = []
     for c in range(world):
         experts, _ = make_routing(rng, tokens, topk, E, routing, routing_param)
         tok = np.repeat(np.arange(tokens, dtype=np.int64), topk)
         dest = experts.reshape(-1)                     # global expert = card * e + local expert
         order = np.lexsort((tok, dest))                # by destination card and expert, then token
         counts = np.bincount(dest, minlength=E).astype(np.int64)
-        act = e4m3_codes_normal(rng, (tokens, h1), 2.0)
-        rows = tok[order]
-        x = act[rows]
-        if mode == "mx":
-            tok_sf = rng.integers(120, 128, size=(tokens, h1 // 32), dtype=np.uint8)
-            x_scale = tok_sf[rows]
-        else:
-            x_scale = np.array([rng.uniform(1e-3, 1e-2)], np.float32)
-        sends.append((x, x_scale, counts, rows))
+        layouts.append((counts, tok[order]))
+    wanted = set(range(world) if ranks is None else ranks)
     cards = []
     for r in range(world):
-        recv = np.array([sends[s][2][r * e + j] for s in range(world) for j in range(e)], np.int64)
-        if mode == "mx":
-            w = rng.integers(0, 256, size=(e, n1, h1 // 2), dtype=np.uint8)
-            w_scale = rng.integers(118, 128, size=(e, n1, h1 // 32), dtype=np.uint8)
-        else:
-            w = e4m3_codes_normal(rng, (e, h1, n1), 0.5)
-            w_scale = np.array([rng.uniform(1e-3, 1e-2)], np.float32)
-        mm_x = mm_x_scale = mm_w = mm_w_scale = None
-        if h2 > 0 and n2 > 0:
-            mm_x = e4m3_codes_normal(rng, (tokens, h2), 2.0)
+        counts, rows = layouts[r]
+        recv = np.array([layouts[s][0][r * e + j] for s in range(world) for j in range(e)], np.int64)
+        card = EpCard(rank=r, x=None, x_scale=None, send_counts=counts, recv_counts=recv, w=None, w_scale=None,
+                      mm_x=None, mm_x_scale=None, mm_w=None, mm_w_scale=None, tokens_of_rows=rows)
+        if r in wanted:
+            g = np.random.default_rng([base, r + 1])
+            act = e4m3_codes_normal(g, (tokens, h1), 2.0)
+            card.x = act[rows]
             if mode == "mx":
-                mm_x_scale = rng.integers(120, 128, size=(tokens, h2 // 32), dtype=np.uint8)
-                mm_w = rng.integers(0, 256, size=(n2, h2 // 2), dtype=np.uint8)
-                mm_w_scale = rng.integers(118, 128, size=(n2, h2 // 32), dtype=np.uint8)
+                card.x_scale = g.integers(120, 128, size=(tokens, h1 // 32), dtype=np.uint8)[rows]
+                card.w = g.integers(0, 256, size=(e, n1, h1 // 2), dtype=np.uint8)
+                card.w_scale = g.integers(118, 128, size=(e, n1, h1 // 32), dtype=np.uint8)
             else:
-                mm_x_scale = np.array([rng.uniform(1e-3, 1e-2)], np.float32)
-                mm_w = e4m3_codes_normal(rng, (h2, n2), 0.5)
-                mm_w_scale = np.array([rng.uniform(1e-3, 1e-2)], np.float32)
-        x, x_scale, counts, rows = sends[r]
-        cards.append(EpCard(rank=r, x=x, x_scale=x_scale, send_counts=counts, recv_counts=recv, w=w,
-                            w_scale=w_scale, mm_x=mm_x, mm_x_scale=mm_x_scale, mm_w=mm_w, mm_w_scale=mm_w_scale,
-                            tokens_of_rows=rows))
+                card.x_scale = np.array([g.uniform(1e-3, 1e-2)], np.float32)
+                card.w = e4m3_codes_normal(g, (e, h1, n1), 0.5)
+                card.w_scale = np.array([g.uniform(1e-3, 1e-2)], np.float32)
+            if h2 > 0 and n2 > 0:
+                card.mm_x = e4m3_codes_normal(g, (tokens, h2), 2.0)
+                if mode == "mx":
+                    card.mm_x_scale = g.integers(120, 128, size=(tokens, h2 // 32), dtype=np.uint8)
+                    card.mm_w = g.integers(0, 256, size=(n2, h2 // 2), dtype=np.uint8)
+                    card.mm_w_scale = g.integers(118, 128, size=(n2, h2 // 32), dtype=np.uint8)
+                else:
+                    card.mm_x_scale = np.array([g.uniform(1e-3, 1e-2)], np.float32)
+                    card.mm_w = e4m3_codes_normal(g, (h2, n2), 0.5)
+                    card.mm_w_scale = np.array([g.uniform(1e-3, 1e-2)], np.float32)
+        cards.append(card)
     return EpProblem(mode=mode, world=world, e=e, tokens=tokens, topk=topk, h1=h1, n1=n1, h2=h2, n2=n2, cards=cards)
+
+
+# The benchmark's expert-parallel workload, per card: page 2's limits (e <= 32 per card,
+# topK in [2, 8], H2 <= 12288) with the single-card workloads' hidden size as H1 and
+# H2 and a 4096-wide first projection (two 2048-wide halves) as N1 and N2.
+EP_BENCH = dict(e=32, tokens=4096, topk=8, h1=7168, n1=4096, h2=7168, n2=4096)
