@@ -58,7 +58,7 @@ typedef enum {
     QGMM_ERR_UNSUPPORTED = 5,         /* the device is not sm_100 or a feature is not built   */
     QGMM_ERR_CUDA = 6,                /* a CUDA runtime / driver call failed                  */
     QGMM_ERR_DEVICE_INPUT = 7,        /* qgmm_device_status found QGMM_DEV_* bits set         */
-    QGMM_ERR_ALIGNMENT = 8,           /* a pointer is not 16-byte aligned                     */
+    QGMM_ERR_ALIGNMENT = 8,           /* a pointer is not suitably (16- or 32-byte) aligned   */
     QGMM_ERR_SCRATCH_LIMIT = 9        /* qgmm_finalize_static_scratch: scratch above its cap  */
 } qgmm_status;
 
@@ -222,7 +222,8 @@ qgmm_status qgmm_plan(const qgmm_problem *p, int32_t sms, qgmm_plan_info *info);
  * (Rows of x2, scale and bias, out, and shared_input are ld_x2, ld_sb, ld_out
  * and ld_shared apart; the shapes above are for the default strides.)
  *   workspace       device memory of ws_bytes bytes, 256-byte aligned
- * x1, x2, out, shared_input, scale and bias must be 16-byte aligned.  Rows at
+ * x1, x2, out, shared_input, scale and bias must be 16-byte aligned (x2 32-byte
+ * aligned with QGMM_W_MXFP4, the base its packed 4-bit tile copy needs).  Rows at
  * or past the groups' total are ignored.
  * Errors: NULL_PTR, SHAPE, DTYPE, ALIGNMENT, WORKSPACE_TOO_SMALL, UNSUPPORTED, CUDA.
  */
@@ -342,7 +343,8 @@ qgmm_status qgmm_debug_accum(const qgmm_problem *p, const int8_t *x1, const void
  * (see QGMM_W_MXFP4 above) for every row i below the groups' total, written by the
  * same kernel qgmm_finalize runs for this type, with no epilogue arithmetic and no
  * combine.  x1 E4M3 [m, k], sfa E8M0 [m, k/32], x2 E2M1 pairs (e, n, k/2), sfb E8M0
- * [e, n, k/32], acc_out f32 [m, n]; all 16-byte aligned; workspace >= 256 bytes.
+ * [e, n, k/32], acc_out f32 [m, n]; all 16-byte aligned, x2 32-byte aligned;
+ * workspace >= 256 bytes.
  * Errors: as qgmm_debug_accum, and DTYPE for any other weight type.
  */
 qgmm_status qgmm_debug_accum_mx(const qgmm_problem *p, const uint8_t *x1, const uint8_t *sfa, const void *x2,

@@ -1155,14 +1155,19 @@ __global__ void __launch_bounds__(PairCfg<W4>::THREADS, 1)
 // per byte (lower k in the low nibble), with an E8M0 scale per 32 k-elements (sfb
 // [e, n, k/32]).  Single CTA, M = 128 rows x N = 128 columns per tile, K = 128 per
 // stage.  The producer TMA-loads the x1 tile (128-byte swizzle) and the packed
-// weight tile (128 n-rows x 64 bytes), and its 32 lanes load the stage's scale
-// words (4 blocks of each row and column) into shared memory in the 32 x 16-byte
-// layout that tcgen05.cp .32x128b.warpx4 takes: byte (r % 32) * 16 + (r / 32) * 4 + b.
-// Four unpack warps turn each E2M1 nibble into the E4M3 byte of the same value
-// (exact: every E2M1 value is an E4M3 value) in a K-major 128-byte-swizzled tile.
-// The MMA thread copies the scale words into tensor memory and issues
-// tcgen05.mma.kind::mxf8f6f4.block_scale (E4M3 x E4M3, one scale byte per 32 K per
-// row of A and column of B, selected per instruction), accumulating f32 in TMEM.
+// weight tile through the padded 4-bit tensor-map type: every 16 E2M1 values (8
+// bytes in global memory) land in a 16-byte shared-memory chunk, data first, then 8
+// unused bytes, so the tile has the K-major 128-byte-swizzled layout of an 8-bit
+// operand, which is what tcgen05.mma reads for an E2M1 operand of kind::mxf8f6f4
+// (measured: the tensor core takes a group's 16 values from the chunk's first 8
+// bytes, lower nibble first, and ignores the rest).  The copy's transaction count
+// is the packed bytes (8 KB per stage), not the 16 KB it writes.  The producer's
+// 32 lanes also load the stage's scale words (4 blocks of each row and column) into
+// shared memory in the 32 x 16-byte layout that tcgen05.cp .32x128b.warpx4 takes:
+// byte (r % 32) * 16 + (r / 32) * 4 + b.  The MMA thread copies the scale words
+// into tensor memory and issues tcgen05.mma.kind::mxf8f6f4.block_scale (E4M3 x
+// E2M1, one scale byte per 32 K per row of A and column of B, selected per
+// instruction), accumulating f32 in TMEM.
 // The epilogue is the staged one with unit scale and pertokenScale: the block
 // scales already sit inside the accumulator, so y = (acc + bias) * logit.
 constexpr int MX_BN = 128;                     // output columns per MX tile
@@ -1170,21 +1175,19 @@ constexpr int MX_SF_BYTES = 512;               // one stage's scale words of 128
 constexpr uint32_t MX_TMEM_SF = 2 * MX_BN;     // TMEM column of the scale-factor buffers
 
 struct MxCfg {
-    static constexpr int STAGES = 4;
+    static constexpr int STAGES = 5;
     static constexpr int EPI_WARPS = 4;
-    static constexpr int UNPACK_WARPS = 4;
-    static constexpr int THREADS = (2 + EPI_WARPS + UNPACK_WARPS) * 32;
+    static constexpr int THREADS = (2 + EPI_WARPS) * 32;
     static constexpr int A_BYTES = BM * BK;            // x1 tile
-    static constexpr int B_BYTES = MX_BN * BK;         // unpacked weight tile (E4M3, K-major)
-    static constexpr int P_BYTES = MX_BN * BK / 2;     // packed E2M1 weight tile
-    static constexpr int NUM_BARS = 3 * STAGES + 2 + 2 + 1;
+    static constexpr int B_BYTES = MX_BN * BK;         // padded E2M1 weight tile (16 values per 16 bytes)
+    static constexpr int B_TX_BYTES = MX_BN * BK / 2;  // the bytes its copy reads, which the barrier counts
+    static constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 1;
     static constexpr int CTRL_BYTES = (NUM_BARS * 8 + 16 + 15) / 16 * 16;
     static constexpr int TABLE_BYTES = (2 * (MAX_E + 1) * 4 + 15) / 16 * 16;
     static constexpr int EPI_STAGE_BYTES = EPI_WARPS * 32 * EPI_LD * 4;
     static constexpr int ROWINFO_BYTES = EPI_WARPS * 32 * 16;
     static constexpr size_t OFF_B = size_t(STAGES) * A_BYTES;
-    static constexpr size_t OFF_P = OFF_B + size_t(STAGES) * B_BYTES;
-    static constexpr size_t OFF_SFA = OFF_P + size_t(STAGES) * P_BYTES;
+    static constexpr size_t OFF_SFA = OFF_B + size_t(STAGES) * B_BYTES;
     static constexpr size_t OFF_SFB = OFF_SFA + size_t(STAGES) * MX_SF_BYTES;
     static constexpr size_t OFF_CTRL = OFF_SFB + size_t(STAGES) * MX_SF_BYTES;
     static constexpr size_t OFF_TABLE = OFF_CTRL + CTRL_BYTES;
@@ -1193,18 +1196,6 @@ struct MxCfg {
     static constexpr size_t SMEM_BYTES = 1024 + OFF_ROWS + ROWINFO_BYTES;
     static_assert(SMEM_BYTES <= 232448, "shared memory above the sm_100 per-block limit");
 };
-
-// Eight E2M1 nibbles (lowest first) -> eight E4M3 bytes: the magnitude through an
-// 8-entry byte table (prmt), the sign from the nibble's top bit (prmt sign mode on
-// bytes whose top bit is that sign).
-__device__ __forceinline__ void e2m1x8_to_e4m3(uint32_t w, uint32_t &lo, uint32_t &hi)
-{
-    constexpr uint32_t LUT_LO = 0x3C383000u;   // 0, 0.5, 1, 1.5
-    constexpr uint32_t LUT_HI = 0x4C484440u;   // 2, 3, 4, 6
-    const uint32_t w4 = w << 4;
-    lo = __byte_perm(LUT_LO, LUT_HI, w & 0x7777u) | (__byte_perm(w4, w, 0xD9C8u) & 0x80808080u);
-    hi = __byte_perm(LUT_LO, LUT_HI, (w >> 16) & 0x7777u) | (__byte_perm(w4, w, 0xFBEAu) & 0x80808080u);
-}
 
 template <int EPI>
 __global__ void __launch_bounds__(MxCfg::THREADS, 1)
@@ -1217,14 +1208,12 @@ __global__ void __launch_bounds__(MxCfg::THREADS, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *smem_a = smem;
     uint8_t *smem_b = smem + Cfg::OFF_B;
-    uint8_t *smem_p = smem + Cfg::OFF_P;
     uint8_t *smem_sfa = smem + Cfg::OFF_SFA;
     uint8_t *smem_sfb = smem + Cfg::OFF_SFB;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_CTRL);
-    uint64_t *pfull = bars;           // x1 tile and packed weight tile landed
-    uint64_t *full = bars + S;        // weights unpacked and scale words written
-    uint64_t *empty = bars + 2 * S;   // MMAs finished reading the stage
-    uint64_t *tfull = bars + 3 * S;   // accumulator buffer ready for the epilogue
+    uint64_t *full = bars;            // x1 and weight tiles landed, scale words written
+    uint64_t *empty = bars + S;       // MMAs finished reading the stage
+    uint64_t *tfull = bars + 2 * S;   // accumulator buffer ready for the epilogue
     uint64_t *tempty = tfull + 2;     // epilogue drained the accumulator buffer
     uint64_t *drain = tempty + 2;     // all issued MMAs completed
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + Cfg::NUM_BARS);
@@ -1241,8 +1230,7 @@ __global__ void __launch_bounds__(MxCfg::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            ptx::mbar_init(&pfull[s], 1);
-            ptx::mbar_init(&full[s], Cfg::UNPACK_WARPS + 1);   // the unpack warps and the scale writer
+            ptx::mbar_init(&full[s], 2);   // the copies' expect_tx arrival and the scale writer's
             ptx::mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -1308,9 +1296,9 @@ __global__ void __launch_bounds__(MxCfg::THREADS, 1)
                     break;
                 }
                 if (lane == 0) {
-                    ptx::mbar_arrive_expect_tx(&pfull[stage], Cfg::A_BYTES + Cfg::P_BYTES);
-                    ptx::tma_load_2d(smem_a + stage * Cfg::A_BYTES, &map_a, &pfull[stage], kb * BK, c.row0);
-                    ptx::tma_load_3d(smem_p + stage * Cfg::P_BYTES, &map_b, &pfull[stage], kb * (BK / 2), n0, c.g);
+                    ptx::mbar_arrive_expect_tx(&full[stage], Cfg::A_BYTES + Cfg::B_TX_BYTES);
+                    ptx::tma_load_2d(smem_a + stage * Cfg::A_BYTES, &map_a, &full[stage], kb * BK, c.row0);
+                    ptx::tma_load_3d(smem_b + stage * Cfg::B_BYTES, &map_b, &full[stage], kb * BK, n0, c.g);
                 }
                 // scale words of the stage's 4 blocks: rows / columns lane, lane + 32, lane + 64, lane + 96
                 uint32_t wa[4], wb[4];
@@ -1338,7 +1326,7 @@ __global__ void __launch_bounds__(MxCfg::THREADS, 1)
             for (int s = 0; s < S; ++s) {
                 if (issued[s] == 0) continue;
                 volatile int never = 0;
-                ptx::mbar_wait(&pfull[s], (issued[s] - 1u) & 1u, &never);
+                ptx::mbar_wait(&full[s], (issued[s] - 1u) & 1u, &never);
             }
         }
         __syncwarp();
@@ -1347,6 +1335,7 @@ __global__ void __launch_bounds__(MxCfg::THREADS, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
+            uint32_t sf_buf = 0;
             int lt = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < T && ok; t += gridDim.x, ++lt) {
@@ -1365,8 +1354,9 @@ __global__ void __launch_bounds__(MxCfg::THREADS, 1)
                         break;
                     }
                     ptx::tc_fence_after();
-                    // this stage's scale words into TMEM (two buffers, by stage parity)
-                    const uint32_t sfa_t = tmem_base + MX_TMEM_SF + 8u * static_cast<uint32_t>(stage & 1);
+                    // this stage's scale words into TMEM (two buffers, alternating per k-block)
+                    const uint32_t sfa_t = tmem_base + MX_TMEM_SF + 8u * sf_buf;
+                    sf_buf ^= 1u;
                     const uint32_t sfb_t = sfa_t + 4u;
                     ptx::tmem_cp_32x128b_warpx4(sfa_t, ptx::smem_desc_noswizzle(
                                                            ptx::smem_addr(smem_sfa + stage * MX_SF_BYTES), 16, 128));
@@ -1378,8 +1368,8 @@ __global__ void __launch_bounds__(MxCfg::THREADS, 1)
                     for (int kk = 0; kk < BK / UMMA_K; ++kk) {
                         const uint64_t adesc = ptx::smem_desc_sw128(a0 + kk * UMMA_K, 16, 1024);
                         const uint64_t bdesc = ptx::smem_desc_sw128(b0 + kk * UMMA_K, 16, 1024);
-                        ptx::mma_mx_e4m3(d_tmem, adesc, bdesc, ptx::idesc_mx_e4m3(BM, MX_BN, kk, kk), sfa_t, sfb_t,
-                                         (kb | kk) != 0 ? 1u : 0u);
+                        ptx::mma_mx_e4m3(d_tmem, adesc, bdesc, ptx::idesc_mx_e4m3(BM, MX_BN, kk, kk, true), sfa_t,
+                                         sfb_t, (kb | kk) != 0 ? 1u : 0u);
                     }
                     ptx::mma_commit(&empty[stage]);
                     if (++stage == S) {
@@ -1412,48 +1402,6 @@ __global__ void __launch_bounds__(MxCfg::THREADS, 1)
                 break;
             }
             if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
-        }
-    } else {
-        // ------------------------------------------------ E2M1 -> E4M3 unpack into the K-major B tile
-        // Per pass a warp takes 8 weight rows x 4 packed 16-byte chunks (lanes 4r..4r+3:
-        // row r, chunks 0-3), reading 512 contiguous bytes; each chunk (32 k) becomes two
-        // 16-byte E4M3 chunks at the row's swizzled positions.
-        const int ut = threadIdx.x - (2 + Cfg::EPI_WARPS) * 32;   // 0..127
-        const int qc = ut & 3;
-        int stage = 0;
-        uint32_t phase = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < T && ok; t += gridDim.x) {
-            for (int kb = 0; kb < KB; ++kb) {
-                if (!ptx::mbar_wait(&pfull[stage], phase, abort_flag)) {
-                    fail();
-                    ok = false;
-                    break;
-                }
-                const uint8_t *pk = smem_p + stage * Cfg::P_BYTES;
-                uint8_t *bb = smem_b + stage * Cfg::B_BYTES;
-#pragma unroll
-                for (int it = 0; it < 4; ++it) {
-                    const int r = (ut >> 2) + 32 * it;    // weight row (output column) in the tile
-                    const uint4 w = *reinterpret_cast<const uint4 *>(pk + r * (BK / 2) + qc * 16);
-                    uint4 o0, o1;
-                    e2m1x8_to_e4m3(w.x, o0.x, o0.y);
-                    e2m1x8_to_e4m3(w.y, o0.z, o0.w);
-                    e2m1x8_to_e4m3(w.z, o1.x, o1.y);
-                    e2m1x8_to_e4m3(w.w, o1.z, o1.w);
-                    uint8_t *rowp = bb + r * 128;
-                    const int c0 = 2 * qc;                // 16-byte chunk (16 k) inside the 128-byte row
-                    *reinterpret_cast<uint4 *>(rowp + ((c0 ^ (r & 7)) << 4)) = o0;
-                    *reinterpret_cast<uint4 *>(rowp + (((c0 + 1) ^ (r & 7)) << 4)) = o1;
-                }
-                ptx::fence_async_shared();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&full[stage]);
-                if (++stage == S) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
         }
     }
 

@@ -351,7 +351,9 @@ __device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint6
 // Instruction descriptor for kind::mxf8f6f4 with E4M3 A and an E4M3 or E2M1 B
 // (b_e2m1), K-major A and B, shape M x N, E8M0 scale factors; a_sf / b_sf pick the
 // byte (the 32-element K block) of each 32-bit scale-factor word that this
-// instruction applies.
+// instruction applies.  An E2M1 operand sits in shared memory like an 8-bit one
+// (one 16-byte chunk per 16 K-values), each chunk holding its 16 values packed in
+// its first 8 bytes, lower K in the low nibble.
 __host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N, int a_sf, int b_sf, bool b_e2m1 = false)
 {
     return (static_cast<uint32_t>(b_sf & 3) << 4)   // B scale-factor byte
@@ -364,7 +366,7 @@ __host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N, int a_sf, int
            | (static_cast<uint32_t>(a_sf & 3) << 29);   // A scale-factor byte
 }
 
-// D[tmem] (+)= (A * scale_A) * (B * scale_B), E4M3 x E4M3 -> f32, one CTA, one E8M0
+// D[tmem] (+)= (A * scale_A) * (B * scale_B), E4M3 x (E4M3 or E2M1, by idesc) -> f32, one CTA, one E8M0
 // scale per 32 K-elements of each A row and each B column, read from tensor memory.
 __device__ __forceinline__ void mma_mx_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate)

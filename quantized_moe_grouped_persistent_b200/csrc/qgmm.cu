@@ -28,6 +28,7 @@ constexpr int kMaxDevices = 64;
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 struct DeviceInfo {
     int sms = 0;
@@ -244,14 +245,18 @@ qgmm_status make_maps(const qgmm_problem *p, const int8_t *x1, const void *x2, i
     const cuuint64_t ld = cuuint64_t(ld_x2(p));
     const bool bytes = p->weight_type != QGMM_W_INT4_PACKED_INT32;   // int8 or E4M3: one byte per element
     if (p->weight_type == QGMM_W_MXFP4) {
-        // E2M1 pairs (e, n, k/2): a box of 64 bytes (128 k) x 128 n-rows, unswizzled
+        // E2M1 pairs (e, n, k/2) through the padded 4-bit type: dimensions count 4-bit
+        // values, strides bytes; a box of 128 k-values (64 bytes read, 128 bytes
+        // written: each 16 values' 8 bytes, then 8 unused) x 128 n-rows, 128-byte
+        // swizzle -- the layout of a K-major 8-bit tile.  The type needs a 32-byte
+        // aligned base and strides that are multiples of 32 bytes (k % 128 == 0 gives them).
         const cuuint64_t kb = cuuint64_t(p->k / 2);
-        const cuuint64_t gdim[3] = {kb, cuuint64_t(p->n), cuuint64_t(p->e)};
+        const cuuint64_t gdim[3] = {cuuint64_t(p->k), cuuint64_t(p->n), cuuint64_t(p->e)};
         const cuuint64_t gstride[2] = {kb, kb * ld};
-        const cuuint32_t box[3] = {cuuint32_t(BK / 2), cuuint32_t(MX_BN), 1};
+        const cuuint32_t box[3] = {cuuint32_t(BK), cuuint32_t(MX_BN), 1};
         const cuuint32_t es[3] = {1, 1, 1};
-        if (enc(mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(x2), gdim, gstride, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+        if (enc(mb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void *>(x2), gdim, gstride, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return QGMM_ERR_CUDA;
     } else if (bytes && p->transpose_x2) {
@@ -552,7 +557,7 @@ qgmm_status finalize_impl(const qgmm_problem *p, const int8_t *x1, const void *x
     if (mx && (!scale || !pertoken_scale)) return QGMM_ERR_NULL_PTR;   // the block scales are required
     if (!aligned16(x1) || !aligned16(x2) || !aligned16(out) || (p->shared_bs > 0 && !aligned16(shared_input)) ||
         (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || !aligned16(scale) || !aligned16(bias) ||
-        (mx && !aligned16(pertoken_scale)))
+        (mx && (!aligned16(pertoken_scale) || !aligned32(x2))))   // the padded 4-bit copy's base: 32 bytes
         return QGMM_ERR_ALIGNMENT;
     if (ws_bytes < workspace_bytes(p)) return QGMM_ERR_WORKSPACE_TOO_SMALL;
     DeviceInfo *dev = nullptr;
@@ -719,7 +724,7 @@ QGMM_API qgmm_status qgmm_debug_accum_mx(const qgmm_problem *p, const uint8_t *x
     if (s != QGMM_OK) return s;
     if (p->weight_type != QGMM_W_MXFP4) return QGMM_ERR_DTYPE;
     if (!x1 || !sfa || !x2 || !sfb || !group_list || !acc_out || !workspace) return QGMM_ERR_NULL_PTR;
-    if (!aligned16(x1) || !aligned16(x2) || !aligned16(acc_out) || !aligned16(sfa) || !aligned16(sfb) ||
+    if (!aligned16(x1) || !aligned32(x2) || !aligned16(acc_out) || !aligned16(sfa) || !aligned16(sfb) ||
         (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
         return QGMM_ERR_ALIGNMENT;
     if (ws_bytes < kAlign) return QGMM_ERR_WORKSPACE_TOO_SMALL;
