@@ -215,7 +215,10 @@ qgmm_status qgmm_plan(const qgmm_problem *p, int32_t sms, qgmm_plan_info *info);
  *   pertoken_scale  f32 [m]; NULL = all ones
  *   group_list      int64 [e], required
  *   logit           f32 [m]; NULL = all ones
- *   row_index       int64 or int32 [m]; NULL = identity (needs output_bs >= total)
+ *   row_index       int64 or int32 [m]; NULL = identity (needs output_bs >= total).
+ *                   With NULL and no shared_input, the atomic mode stores each row
+ *                   directly (one contribution per output row: the same 0 + y) and
+ *                   zeroes only the rows past the groups' total
  *   bias            f32 [e, n]; NULL = zeros
  *   shared_input    bf16 bits [shared_bs, n]; required iff shared_bs > 0
  *   out             f32 [output_bs, n], fully overwritten (no need to clear it)

@@ -22,9 +22,10 @@
  *   - The grouped matmul then sees group_counts[j] = sum_s recv_counts[s*e + j]
  *     rows for expert j (a type-1 group list).
  *
- * The library computes offsets only; the exchange itself runs over NCCL (each
- * chunk received straight into its permuted place, so the permute costs no pass
- * of its own), and the matmuls through qgmm_finalize.
+ * The library computes the offsets and moves the chunks a card keeps for itself
+ * (qgmm_ep_permute_rows); the exchange with other cards runs over NCCL (each chunk
+ * received straight into its permuted place, so the permute costs no pass of its
+ * own), and the matmuls through qgmm_finalize.
  */
 #ifndef QGMM_EP_H
 #define QGMM_EP_H
@@ -57,6 +58,25 @@ extern "C" {
  */
 qgmm_status qgmm_ep_plan(int32_t world, int32_t e, const int64_t *send_counts, const int64_t *recv_counts,
                          int64_t *send_offsets, int64_t *recv_offsets, int64_t *group_counts, int64_t *totals);
+
+#define QGMM_EP_MAX_CHUNKS 32   /* chunks per qgmm_ep_permute_rows call: one per local expert */
+
+/*
+ * The chunks a card addresses to itself, moved to their permuted places by one
+ * kernel on `cuda_stream` (asynchronous).  For each chunk c with count[c] > 0, rows
+ * [src_row[c], src_row[c] + count[c]) of src are copied to rows [dst_row[c], ...)
+ * of dst.  src and dst are DEVICE pointers (4-byte aligned; 16-byte copies are used
+ * when both and row_bytes allow), rows row_bytes apart (row_bytes >= 4,
+ * row_bytes % 4 == 0); the chunk table (src_row, dst_row, count: int64 [nchunks],
+ * 0 <= nchunks <= QGMM_EP_MAX_CHUNKS) is in HOST memory and is passed to the kernel
+ * by value, so the caller may reuse it as soon as the call returns.  Source and
+ * destination ranges must not overlap.  Nothing is launched when every count is 0.
+ * Errors: NULL_PTR, SHAPE (a limit above broken, or a negative entry), ALIGNMENT,
+ * CUDA.
+ */
+qgmm_status qgmm_ep_permute_rows(const void *src, void *dst, int64_t row_bytes, int32_t nchunks,
+                                 const int64_t *src_row, const int64_t *dst_row, const int64_t *count,
+                                 void *cuda_stream);
 
 #ifdef __cplusplus
 }

@@ -13,6 +13,7 @@ Entry points mirror the C ABI:
     debug_accum(problem, x1, x2, group_list, acc_out, workspace)
     device_status(workspace) -> QGMM_DEV_* flags
     ep_plan(world, e, send_counts, recv_counts) -> offsets of the expert-parallel dispatch
+    ep_permute_rows(src, dst, src_rows, dst_rows, counts) -> a card's own chunks, one kernel
 """
 from __future__ import annotations
 
@@ -55,7 +56,7 @@ QGMM_DEV_TIMEOUT = 1 << 4
 EXPORTS = ("qgmm_finalize_workspace", "qgmm_finalize_launches", "qgmm_plan", "qgmm_finalize", "qgmm_finalize_profiled",
            "qgmm_per_token_quant", "qgmm_per_token_quant_mxfp8", "qgmm_debug_accum", "qgmm_debug_accum_mx",
            "qgmm_device_status",
-           "qgmm_finalize_static_scratch", "qgmm_ep_plan", "qgmm_status_string")
+           "qgmm_finalize_static_scratch", "qgmm_ep_plan", "qgmm_ep_permute_rows", "qgmm_status_string")
 
 
 class QgmmProblem(C.Structure):
@@ -108,6 +109,7 @@ def lib():
         L.qgmm_device_status.argtypes = [P, C.POINTER(C.c_uint32), P]
         L.qgmm_finalize_static_scratch.argtypes = [C.POINTER(QgmmProblem), P, P, P, P, P, P, P, P, P, P, P]
         L.qgmm_ep_plan.argtypes = [C.c_int32, C.c_int32, P, P, P, P, P, P]
+        L.qgmm_ep_permute_rows.argtypes = [P, P, I64, C.c_int32, P, P, P, P]
         L.qgmm_status_string.argtypes = [C.c_int]
         L.qgmm_status_string.restype = C.c_char_p
         for name in EXPORTS[:-1]:
@@ -279,3 +281,26 @@ def ep_plan(world: int, e: int, send_counts, recv_counts) -> dict:
     _check(lib().qgmm_ep_plan(int(world), int(e), ptr(sc), ptr(rc_), ptr(so), ptr(ro), ptr(gc), ptr(tot)),
            "qgmm_ep_plan")
     return {"send_offsets": so, "recv_offsets": ro, "group_counts": gc[:e], "bsk": int(tot[0]), "a": int(tot[1])}
+
+
+QGMM_EP_MAX_CHUNKS = 32
+
+
+def ep_permute_rows(src, dst, src_rows, dst_rows, counts, stream=None) -> None:
+    """Copy row chunks of device tensor ``src`` into ``dst`` (same row width), chunk c
+    taking ``counts[c]`` rows from ``src_rows[c]`` to ``dst_rows[c]``, in one kernel
+    (``qgmm_ep_permute_rows``).  The tables are host sequences of at most
+    QGMM_EP_MAX_CHUNKS entries."""
+    import numpy as np
+    if not (src.is_cuda and dst.is_cuda):
+        raise QgmmError(QGMM_ERR_UNSUPPORTED, "qgmm_ep_permute_rows: device tensors only")
+    row_bytes = src.stride(0) * src.element_size()
+    if dst.stride(0) * dst.element_size() != row_bytes or not src.is_contiguous() or not dst.is_contiguous():
+        raise QgmmError(QGMM_ERR_SHAPE, "qgmm_ep_permute_rows")
+    tabs = [np.ascontiguousarray(np.asarray(a, np.int64).reshape(-1)) for a in (src_rows, dst_rows, counts)]
+    n = tabs[2].size
+    if tabs[0].size != n or tabs[1].size != n:
+        raise QgmmError(QGMM_ERR_SHAPE, "qgmm_ep_permute_rows")
+    ptr = lambda a: a.ctypes.data_as(C.c_void_p)
+    _check(lib().qgmm_ep_permute_rows(_ptr(src), _ptr(dst), row_bytes, n, ptr(tabs[0]), ptr(tabs[1]), ptr(tabs[2]),
+                                      _stream(stream)), "qgmm_ep_permute_rows")

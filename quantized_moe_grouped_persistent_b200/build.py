@@ -10,7 +10,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libqgmm.so")
-MAIN = [os.path.join(HERE, "csrc", "qgmm.cu"), os.path.join(HERE, "csrc", "ep_plan.cu")]
+MAIN = [os.path.join(HERE, "csrc", "qgmm.cu"), os.path.join(HERE, "csrc", "ep_plan.cu"),
+        os.path.join(HERE, "csrc", "ep_permute.cu")]
 PROBE_LIB = os.path.join(HERE, "libqgmm_probe.so")
 PROBE = [os.path.join(HERE, "csrc", "probe_mma.cu")]
 NVCC_FLAGS = [

@@ -97,7 +97,8 @@ struct GemmArgs {
     const void *row_index;
     int32_t row_index_type;
     int64_t output_bs;
-    float *out;            // EPI_ATOMIC: out [output_bs, ldd]; EPI_STORE_Y: y [m, ldd]
+    float *out;            // EPI_ATOMIC: out [output_bs, ldd]; EPI_STORE_Y: y [store_rows, ldd]
+    int64_t store_rows;    // EPI_STORE_Y: rows of its destination (m for y; output_bs when it is out)
     int32_t *acc_out;      // EPI_RAW_ACC: [m, ldd]
     int64_t ldd;           // row stride of the destination (out, y or acc_out)
     const uint8_t *sfa;    // MX kernel: E8M0 scales of x1 [m, k/32]
@@ -311,8 +312,9 @@ __device__ __forceinline__ void epi_write_chunk(const GemmArgs &args, const floa
                 const float y3 = __fmul_rn(__fadd_rn(__fmul_rn(__fmul_rn(v.w, s4.w), p), b4.w), l);
                 if constexpr (EPI == EPI_ATOMIC) {
                     ptx::red_add_v4(args.out + d * ldd + col, y0, y1, y2, y3);
-                } else {
-                    *reinterpret_cast<float4 *>(args.out + d * ldd + col) = make_float4(y0, y1, y2, y3);
+                } else {   // stored as 0 + y, the value a sum starting from zero gives (-0 becomes +0)
+                    *reinterpret_cast<float4 *>(args.out + d * ldd + col) = make_float4(
+                        __fadd_rn(y0, 0.f), __fadd_rn(y1, 0.f), __fadd_rn(y2, 0.f), __fadd_rn(y3, 0.f));
                 }
             }
         }
@@ -369,6 +371,8 @@ __device__ __forceinline__ bool epilogue_tile(const GemmArgs &args, const TileCo
             const int64_t d = load_row_index(args.row_index, args.row_index_type, i);
             if (d < 0 || d >= args.output_bs) atomicOr(args.status, QGMM_DEV_ROW_INDEX_RANGE);
             else dst = d;
+        } else if (EPI == EPI_STORE_Y && i >= args.store_rows) {
+            atomicOr(args.status, QGMM_DEV_ROW_INDEX_RANGE);   // identity routing past output_bs
         } else {
             dst = i;
         }
@@ -460,8 +464,9 @@ __device__ __forceinline__ void epi_direct_rows(const GemmArgs &args, const uint
                 const float y1 = __fmul_rn(__fadd_rn(__fmul_rn(__fmul_rn(a1, sc[j].y), p), bs[j].y), l);
                 if constexpr (EPI == EPI_ATOMIC) {
                     ptx::red_add_v2(args.out + d * ldd + col, y0, y1);
-                } else {
-                    *reinterpret_cast<float2 *>(args.out + d * ldd + col) = make_float2(y0, y1);
+                } else {   // stored as 0 + y, as in the staged epilogue
+                    *reinterpret_cast<float2 *>(args.out + d * ldd + col) =
+                        make_float2(__fadd_rn(y0, 0.f), __fadd_rn(y1, 0.f));
                 }
             }
         }
@@ -492,6 +497,8 @@ __device__ __forceinline__ bool epilogue_tile_direct(const GemmArgs &args, const
                 const int64_t d = load_row_index(args.row_index, args.row_index_type, i);
                 if (d < 0 || d >= args.output_bs) atomicOr(args.status, QGMM_DEV_ROW_INDEX_RANGE);
                 else dst[k] = d;
+            } else if (EPI == EPI_STORE_Y && i >= args.store_rows) {
+                atomicOr(args.status, QGMM_DEV_ROW_INDEX_RANGE);   // identity routing past output_bs
             } else {
                 dst[k] = i;
             }
@@ -1480,6 +1487,24 @@ __device__ __forceinline__ int64_t groups_total_block(const int64_t *gl, int e, 
     }
     __syncthreads();
     return off[e];
+}
+
+// K1 for identity routing without sharedInput: every output row then receives at
+// most one source row, which the grouped GEMM stores directly (EPI_STORE_Y into out);
+// this kernel zeroes the rows at or past the groups' total, which receive none, and
+// clears the call's status word.
+__global__ void output_tail_zero_kernel(float *__restrict__ out, int64_t output_bs, int32_t n, int64_t ld,
+                                        const int64_t *gl, int e, int type, int64_t m, uint32_t *status)
+{
+    ptx::pdl_launch_dependents();   // the grouped GEMM may start its prologue and mainloop now
+    if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
+    __shared__ int32_t off[MAX_E + 1], cum[MAX_E + 1];
+    const int64_t total = groups_total_block(gl, e, type, m, off, cum, status, false);   // the GEMM reports
+    const int n4 = n / 4;
+    for (int64_t r = total + blockIdx.x; r < output_bs; r += gridDim.x) {
+        float4 *dst = reinterpret_cast<float4 *>(out + r * ld);
+        for (int c = threadIdx.x; c < n4; c += blockDim.x) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 }
 
 __global__ void det_hist_kernel(const int64_t *gl, int e, int type, int64_t m, const void *row_index, int ri_type,

@@ -513,6 +513,7 @@ GemmArgs base_args(const qgmm_problem *p, const int64_t *group_list, const Plan 
     a.b_kmajor = p->transpose_x2;
     a.row_index_type = p->row_index_type;
     a.output_bs = p->output_bs;
+    a.store_rows = p->m;
     a.status = status;
     a.ld_sb = ld_sb(p);
     a.ldd = p->n;   // y and acc_out rows; the atomic combine's launch sets ld_out
@@ -590,6 +591,22 @@ qgmm_status finalize_impl(const qgmm_problem *p, const int8_t *x1, const void *x
     a.row_index = row_index;
     const uint16_t *shared = p->shared_bs > 0 ? shared_input : nullptr;
 
+    if (!p->deterministic && !row_index && !shared) {
+        // Identity routing without sharedInput: an output row receives at most one
+        // source row, so the GEMM stores it (as 0 + y, the combine's value) instead of
+        // reducing into a zeroed output; only the rows past the groups' total are zeroed.
+        output_tail_zero_kernel<<<grid_for(p->output_bs, 1, dev->sms, 2), 256, 0, st>>>(
+            out, p->output_bs, static_cast<int32_t>(p->n), ld_out(p), group_list, static_cast<int>(p->e),
+            p->group_list_type, p->m, status);
+        if (cudaGetLastError() != cudaSuccess) return QGMM_ERR_CUDA;
+        a.out = out;
+        a.ldd = ld_out(p);
+        a.store_rows = p->output_bs;
+        if (ev_begin && cudaEventRecord(ev_begin, st) != cudaSuccess) return QGMM_ERR_CUDA;
+        if ((s = launch_gemm(EPI_STORE_Y, dev, p, pl, ma, mb, mb_tail, a, st)) != QGMM_OK) return s;
+        if (ev_end && cudaEventRecord(ev_end, st) != cudaSuccess) return QGMM_ERR_CUDA;
+        return QGMM_OK;
+    }
     if (!p->deterministic) {
         output_init_kernel<<<grid_for(p->output_bs, 1, dev->sms, 2), 256, 0, st>>>(
             out, p->output_bs, static_cast<int32_t>(p->n), ld_out(p), shared, ld_shared(p), p->shared_bs,

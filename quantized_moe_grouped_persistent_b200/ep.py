@@ -16,8 +16,9 @@ How it maps onto this library (marshalling only; no arithmetic in Python):
   - The exchange posts one send and one receive per non-empty (peer, expert) chunk
     in a single batched group of torch.distributed point-to-point operations (NCCL
     over NVLink on GPUs, gloo on the CPU), each receive landing straight at its
-    permuted offset: the permute costs no pass of its own.  Chunks a card addresses
-    to itself are device-to-device copies.  The activation scales travel the same
+    permuted offset: the permute costs no pass of its own.  The chunks a card
+    addresses to itself move in one library kernel (``qgmm_ep_permute_rows``) per
+    buffer.  The activation scales travel the same
     way (mx: the E8M0 rows; pertensor: the source card's scale, one f32 per row).
   - The grouped matmul is ``qgmm_finalize`` over the permuted rows with the
     per-expert counts as a type-1 group list, identity routing and unit logits, so
@@ -30,8 +31,8 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (QGMM_GROUP_COUNTS, QGMM_W_FP8_E4M3, QGMM_W_MXFP4, QgmmError, QGMM_ERR_SHAPE, ep_plan, finalize,
-               finalize_profiled, finalize_workspace, make_problem)
+from . import (QGMM_GROUP_COUNTS, QGMM_W_FP8_E4M3, QGMM_W_MXFP4, QgmmError, QGMM_ERR_SHAPE, ep_permute_rows, ep_plan,
+               finalize, finalize_profiled, finalize_workspace, make_problem)
 
 MODES = ("pertensor", "mx")
 
@@ -60,10 +61,14 @@ def _scalar(v) -> float:
 
 
 class Exchange:
-    """The AlltoAllv with the permute folded into where each chunk lands."""
+    """The AlltoAllv with the permute folded into where each chunk lands.
 
-    def __init__(self, world: int, rank: int, e: int, group=None):
+    ``local(src, dst, src_rows, dst_rows, counts)`` moves the card's own chunks; the
+    default is the library's one-kernel device copy (device tensors only)."""
+
+    def __init__(self, world: int, rank: int, e: int, group=None, local=None):
         self.world, self.rank, self.e, self.group = world, rank, e, group
+        self.local = ep_permute_rows if local is None else local
 
     def check_counts(self, send_counts, recv_counts, device) -> None:
         """Every card's receive counts must be its peers' send counts (page 2: the
@@ -85,19 +90,19 @@ class Exchange:
         with the same chunking.  Posts every transfer, then waits for all of them."""
         import torch.distributed as dist
         e, so, ro = self.e, plan["send_offsets"], plan["recv_offsets"]
+        own = slice(self.rank * e, (self.rank + 1) * e)   # the chunks this card keeps
+        if not np.array_equal(np.asarray(send_counts)[own], np.asarray(recv_counts)[own]):
+            raise QgmmError(QGMM_ERR_SHAPE, "ep exchange: own send and receive counts differ")
+        if int(np.asarray(send_counts)[own].sum()) > 0:
+            for src, dst in pairs:
+                self.local(src, dst, so[own], ro[own], np.asarray(send_counts)[own])
         ops = []
         for peer in range(self.world):
+            if peer == self.rank:
+                continue
             for j in range(e):
                 c = peer * e + j
                 sc, rc = int(send_counts[c]), int(recv_counts[c])
-                if peer == self.rank:      # chunk (self, j): a device copy to its permuted place
-                    if sc != rc:
-                        raise QgmmError(QGMM_ERR_SHAPE, "ep exchange: own send and receive counts differ")
-                    for b, (src, dst) in enumerate(pairs):
-                        if sc:
-                            dst[int(ro[self.rank * e + j]):int(ro[self.rank * e + j]) + rc].copy_(
-                                src[int(so[c]):int(so[c]) + sc])
-                    continue
                 for b, (src, dst) in enumerate(pairs):
                     tag = b * e + j
                     if sc:

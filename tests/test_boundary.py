@@ -27,8 +27,8 @@ def test_header_declares_the_abi():
         "qgmm_per_token_quant_mxfp8", "qgmm_debug_accum", "qgmm_debug_accum_mx", "qgmm_device_status",
         "qgmm_finalize_static_scratch",
         "qgmm_status_string",
-        "qgmm_finalize_launches", "qgmm_plan", "qgmm_ep_plan"])
-    assert _declared_functions((EP_HEADER,)) == ["qgmm_ep_plan"]
+        "qgmm_finalize_launches", "qgmm_plan", "qgmm_ep_plan", "qgmm_ep_permute_rows"])
+    assert _declared_functions((EP_HEADER,)) == ["qgmm_ep_permute_rows", "qgmm_ep_plan"]
 
 
 def test_library_exports_every_declared_symbol(qgmm):

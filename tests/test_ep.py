@@ -155,7 +155,27 @@ def test_ep_plan_null_pointers(qgmm):
     assert qgmm.lib().qgmm_ep_plan(2, 2, a, a, o, o, o, None) == qgmm.QGMM_ERR_NULL_PTR
 
 
+def test_ep_permute_rows_host_checks(qgmm):
+    import ctypes as C
+    L = qgmm.lib()
+    t = (C.c_int64 * 2)(0, 4)
+    z = (C.c_int64 * 2)(0, 0)
+    neg = (C.c_int64 * 2)(-1, 0)
+    assert L.qgmm_ep_permute_rows(None, None, 16, 2, t, t, z, None) == qgmm.QGMM_OK     # nothing to move
+    assert L.qgmm_ep_permute_rows(None, None, 16, 2, None, t, z, None) == qgmm.QGMM_ERR_NULL_PTR
+    assert L.qgmm_ep_permute_rows(None, None, 16, 33, t, t, z, None) == qgmm.QGMM_ERR_SHAPE
+    assert L.qgmm_ep_permute_rows(None, None, 6, 2, t, t, z, None) == qgmm.QGMM_ERR_SHAPE     # row_bytes % 4
+    assert L.qgmm_ep_permute_rows(None, None, 16, 2, t, t, neg, None) == qgmm.QGMM_ERR_SHAPE
+    assert L.qgmm_ep_permute_rows(None, None, 16, 2, t, t, t, None) == qgmm.QGMM_ERR_NULL_PTR  # rows, no buffers
+
+
 # ---------------------------------------------------------------- gloo exchange
+def _cpu_local(src, dst, src_rows, dst_rows, counts):
+    """The card's own chunks on CPU tensors (the library's copy kernel takes device tensors)."""
+    for a, b, n in zip(src_rows, dst_rows, counts):
+        dst[int(b):int(b) + int(n)] = src[int(a):int(a) + int(n)]
+
+
 def _free_port():
     s = socket.socket()
     s.bind(("127.0.0.1", 0))
@@ -197,7 +217,7 @@ def _exchange_main(rank, world, e, seed, port, out, mode):
         rng = np.random.default_rng(seed + 1 + rank)
         x = torch.from_numpy(rng.integers(0, 256, (bsk, 64), dtype=np.uint8))
         sf = torch.from_numpy(rng.integers(100, 140, (bsk, 2), dtype=np.uint8))
-        ex = Exchange(world, rank, e)
+        ex = Exchange(world, rank, e, local=_cpu_local)
         try:
             ex.check_counts(send, recv, "cpu")
         except Exception as err:                      # every rank sees the same gathered counts

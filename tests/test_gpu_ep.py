@@ -89,3 +89,24 @@ def test_grouped_matmul_with_no_rows_launches_nothing(ep_mod):
     out, sc, plan = m.dispatch(c.x, c.x_scale, c.send_counts, c.recv_counts)
     assert out.shape[0] == plan["a"] == int(c.recv_counts.sum())
     assert m.grouped(out[:0], sc[:0], np.zeros(p.e, np.int64)) is None
+
+
+@pytest.mark.parametrize("row_bytes", [7168, 224, 12, 4])
+def test_permute_rows_kernel(ep_mod, row_bytes):
+    from quantized_moe_grouped_persistent_b200 import ep_permute_rows
+    rng = np.random.default_rng(row_bytes)
+    counts = rng.integers(0, 40, 32)
+    counts[3] = 0
+    total = int(counts.sum())
+    src_rows = np.concatenate([[0], np.cumsum(counts)[:-1]])
+    order = rng.permutation(32)                         # destination order of the chunks
+    dst_rows = np.zeros(32, np.int64)
+    dst_rows[order] = np.concatenate([[0], np.cumsum(counts[order])[:-1]])
+    src = rng.integers(0, 256, (total, row_bytes), dtype=np.uint8)
+    want = np.zeros_like(src)
+    for a, b, n in zip(src_rows, dst_rows, counts):
+        want[b:b + n] = src[a:a + n]
+    dsrc = torch.from_numpy(src).cuda()
+    ddst = torch.zeros_like(dsrc)
+    ep_permute_rows(dsrc, ddst, src_rows, dst_rows, counts)
+    np.testing.assert_array_equal(ddst.cpu().numpy(), want)
