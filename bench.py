@@ -320,8 +320,10 @@ def time_e2e(d, p, steps, warmup, deterministic):
     return t0.elapsed_time(t1) / steps, h2d, d2h
 
 
-def gemm_kernel_label(plan):
+def gemm_kernel_label(plan, weight="int8"):
     """Which grouped-GEMM kernel(s) a call runs, from the library's own plan (qgmm_plan)."""
+    if weight == "mxfp4":
+        return "grouped_gemm_mx_kernel"
     if not plan["pair"]:
         return "grouped_gemm_kernel"
     if plan["gemm_launches"] == 2:
@@ -604,7 +606,7 @@ def main():
     op_launches = finalize_launches(d.problem(args.deterministic))
     launches_per_step = op_launches + (1 if d.prologue else 0)
     sms = torch.cuda.get_device_properties(dev_index).multi_processor_count
-    gemm_kernel = gemm_kernel_label(plan(d.problem(args.deterministic), sms))
+    gemm_kernel = gemm_kernel_label(plan(d.problem(args.deterministic), sms), p.weight)
 
     extras = {}
     if not args.no_extras:
