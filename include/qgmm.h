@@ -166,6 +166,11 @@ typedef struct {
  *                                      max(1, floor(max(2^24, m*n/16) / output_bs)))
  *   + (output_bs + 1)*4        bucket boundaries
  *   + m*4                      source rows grouped by destination
+ * QGMM_W_MXFP4 adds, after the above, each part rounded up to 256 bytes:
+ *   + (ceil(m/128) + e) * (k/128) * 512        x1's scale atoms
+ *   + e * (n/128) * (k/128) * 512              the weights' scale atoms
+ * (the scale words rearranged per call into the per-stage layout the MX kernel
+ * bulk-copies; as many bytes as the scale arrays themselves, plus padding).
  * Errors: NULL_PTR, SHAPE, DTYPE, UNSUPPORTED (transpose_x2 with int4 weights, or
  * QGMM_W_MXFP4 without transpose_x2).
  */
@@ -178,6 +183,7 @@ qgmm_status qgmm_finalize_workspace(const qgmm_problem *p, size_t *ws_bytes);
  * Atomic mode: the output init plus the grouped GEMM launches (1, or 2 when
  * full-height tiles run on CTA pairs and odd tails on a single-CTA launch).
  * Deterministic mode adds the five bucketing kernels and the final reduce.
+ * QGMM_W_MXFP4 adds the two kernels that write its scale atoms.
  * The per-token quant prologue is a separate call and is not counted.
  * Errors: NULL_PTR, SHAPE, DTYPE, UNSUPPORTED, CUDA (no usable device).
  */
@@ -347,7 +353,7 @@ qgmm_status qgmm_debug_accum(const qgmm_problem *p, const int8_t *x1, const void
  * same kernel qgmm_finalize runs for this type, with no epilogue arithmetic and no
  * combine.  x1 E4M3 [m, k], sfa E8M0 [m, k/32], x2 E2M1 pairs (e, n, k/2), sfb E8M0
  * [e, n, k/32], acc_out f32 [m, n]; all 16-byte aligned, x2 32-byte aligned;
- * workspace >= 256 bytes.
+ * workspace of qgmm_finalize_workspace(p) bytes (its scale atoms).
  * Errors: as qgmm_debug_accum, and DTYPE for any other weight type.
  */
 qgmm_status qgmm_debug_accum_mx(const qgmm_problem *p, const uint8_t *x1, const uint8_t *sfa, const void *x2,

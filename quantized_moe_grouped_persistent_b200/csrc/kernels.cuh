@@ -179,6 +179,7 @@ __device__ __forceinline__ uint32_t decode_groups_warp(const int64_t *gl, int e,
 
 struct TileCoord {
     int g, row0, row_end, nt;
+    int mt;      // m-tile index in the walk (the expert-major order of the groups' tiles)
     bool tail;   // SCHED_PAIRS_TAIL128: an M = 128 pair tile
 };
 
@@ -194,6 +195,7 @@ __device__ __forceinline__ TileCoord tile_coord(int t, int MT, int SW, const int
     const int r = t - s * per_slab;
     const int mt = r / SW;
     TileCoord c;
+    c.mt = mt;
     c.nt = s * SW + (r - mt * SW);
     int lo = 0, hi = e;  // cum[lo] <= mt < cum[hi]
     while (hi - lo > 1) {
@@ -1168,10 +1170,13 @@ __global__ void __launch_bounds__(PairCfg<W4>::THREADS, 1)
 // operand, which is what tcgen05.mma reads for an E2M1 operand of kind::mxf8f6f4
 // (measured: the tensor core takes a group's 16 values from the chunk's first 8
 // bytes, lower nibble first, and ignores the rest).  The copy's transaction count
-// is the packed bytes (8 KB per stage), not the 16 KB it writes.  The producer's
-// 32 lanes also load the stage's scale words (4 blocks of each row and column) into
-// shared memory in the 32 x 16-byte layout that tcgen05.cp .32x128b.warpx4 takes:
-// byte (r % 32) * 16 + (r / 32) * 4 + b.  The MMA thread copies the scale words
+// is the packed bytes (8 KB per stage), not the 16 KB it writes.  The stage's scale
+// words (4 blocks of each of the tile's rows and columns) arrive as two 512-byte
+// atoms, bulk-copied on the same barrier, already in the 32 x 16-byte layout that
+// tcgen05.cp .32x128b.warpx4 takes: byte (r % 32) * 16 + (r / 32) * 4 + b.  A pre-pass
+// (mx_sf_atoms_rows_kernel, mx_sf_atoms_cols_kernel) writes the atoms; loading the
+// words row by row in the producer cost a third of the kernel's time.  The MMA
+// thread copies the scale words
 // into tensor memory and issues tcgen05.mma.kind::mxf8f6f4.block_scale (E4M3 x
 // E2M1, one scale byte per 32 K per row of A and column of B, selected per
 // instruction), accumulating f32 in TMEM.
@@ -1237,7 +1242,7 @@ __global__ void __launch_bounds__(MxCfg::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            ptx::mbar_init(&full[s], 2);   // the copies' expect_tx arrival and the scale writer's
+            ptx::mbar_init(&full[s], 1);   // the producer's expect_tx arrival; the copies complete the bytes
             ptx::mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -1272,7 +1277,6 @@ __global__ void __launch_bounds__(MxCfg::THREADS, 1)
     const int SW = args.slab_ntiles;
     const int T = MT * NT;
     const int KB = args.k / BK;
-    const int64_t nb = args.k / 32;   // scale bytes per row / column
 
     // The status word is cleared by the kernel this one may overlap under programmatic
     // dependent launch: wait for that kernel before setting a bit in it.
@@ -1303,24 +1307,18 @@ __global__ void __launch_bounds__(MxCfg::THREADS, 1)
                     break;
                 }
                 if (lane == 0) {
-                    ptx::mbar_arrive_expect_tx(&full[stage], Cfg::A_BYTES + Cfg::B_TX_BYTES);
+                    // the x1 tile, the padded weight tile, and the stage's two 512-byte scale
+                    // atoms (arranged by mx_sf_atoms_*_kernel in the layout tcgen05.cp takes)
+                    ptx::mbar_arrive_expect_tx(&full[stage], Cfg::A_BYTES + Cfg::B_TX_BYTES + 2 * MX_SF_BYTES);
                     ptx::tma_load_2d(smem_a + stage * Cfg::A_BYTES, &map_a, &full[stage], kb * BK, c.row0);
                     ptx::tma_load_3d(smem_b + stage * Cfg::B_BYTES, &map_b, &full[stage], kb * BK, n0, c.g);
+                    ptx::bulk_load(smem_sfa + stage * MX_SF_BYTES,
+                                   args.sfa + (static_cast<int64_t>(c.mt) * KB + kb) * MX_SF_BYTES, MX_SF_BYTES,
+                                   &full[stage]);
+                    ptx::bulk_load(smem_sfb + stage * MX_SF_BYTES,
+                                   args.sfb + ((static_cast<int64_t>(c.g) * NT + c.nt) * KB + kb) * MX_SF_BYTES,
+                                   MX_SF_BYTES, &full[stage]);
                 }
-                // scale words of the stage's 4 blocks: rows / columns lane, lane + 32, lane + 64, lane + 96
-                uint32_t wa[4], wb[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int64_t r = static_cast<int64_t>(c.row0) + lane + 32 * j;
-                    wa[j] = r < args.m ? __ldg(reinterpret_cast<const unsigned int *>(args.sfa + r * nb + 4 * kb)) : 0u;
-                    const int64_t col = static_cast<int64_t>(c.g) * args.ld_sb + n0 + lane + 32 * j;
-                    wb[j] = __ldg(reinterpret_cast<const unsigned int *>(args.sfb + col * nb + 4 * kb));
-                }
-                *reinterpret_cast<uint4 *>(smem_sfa + stage * MX_SF_BYTES + lane * 16) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
-                *reinterpret_cast<uint4 *>(smem_sfb + stage * MX_SF_BYTES + lane * 16) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
-                ptx::fence_async_shared();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&full[stage]);
                 ++issued[stage];
                 if (++stage == S) {
                     stage = 0;
@@ -1417,6 +1415,48 @@ __global__ void __launch_bounds__(MxCfg::THREADS, 1)
     if (warp == 1) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem_base, 512);
+    }
+}
+
+// ---------------------------------------------------------------- MxA8W4 scale atoms
+// Atom layout (512 bytes, the 32 x 16-byte source of tcgen05.cp .32x128b.warpx4):
+// word i * 4 + j holds the scale bytes of k-blocks 4 kb .. 4 kb + 3 of the tile's
+// row (or column) i + 32 j.  x1's atoms are indexed (m-tile of the MX kernel's walk,
+// kb), the weights' (expert * n/128 + 128-column tile, kb).  One block of 128
+// threads per tile; thread i * 4 + j walks its row's words over k.
+__global__ void mx_sf_atoms_rows_kernel(const uint8_t *__restrict__ sfa, int64_t m, int32_t k, const int64_t *gl,
+                                        int e, int type, uint32_t *__restrict__ atoms)
+{
+    __shared__ int32_t off[MAX_E + 1], cum[MAX_E + 1];
+    if (threadIdx.x < 32) decode_groups_warp(gl, e, type, m, BM, SCHED_TILES, off, cum);   // the MX kernel's tiles
+    __syncthreads();
+    const int MT = cum[e];
+    const int KB = k / BK;
+    const int i = threadIdx.x >> 2, j = threadIdx.x & 3;
+    for (int mt = blockIdx.x; mt < MT; mt += gridDim.x) {
+        int lo = 0, hi = e;   // cum[lo] <= mt < cum[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (cum[mid] <= mt) lo = mid;
+            else hi = mid;
+        }
+        const int64_t r = int64_t(off[lo]) + int64_t(mt - cum[lo]) * BM + i + 32 * j;
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(sfa + (r < m ? r : 0) * (k / 32));
+        uint32_t *dst = atoms + int64_t(mt) * KB * 128 + threadIdx.x;
+        for (int kb = 0; kb < KB; ++kb) dst[int64_t(kb) * 128] = r < m ? __ldg(src + kb) : 0u;   // rows past m: 0
+    }
+}
+
+__global__ void mx_sf_atoms_cols_kernel(const uint8_t *__restrict__ sfb, int e, int32_t n, int64_t ld_sb, int32_t k,
+                                        uint32_t *__restrict__ atoms)
+{
+    const int NT = n / MX_BN, KB = k / BK;
+    const int i = threadIdx.x >> 2, j = threadIdx.x & 3;
+    for (int64_t a = blockIdx.x; a < int64_t(e) * NT; a += gridDim.x) {
+        const int64_t g = a / NT, nt = a - g * NT;
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(sfb + (g * ld_sb + nt * MX_BN + i + 32 * j) * (k / 32));
+        uint32_t *dst = atoms + a * KB * 128 + threadIdx.x;
+        for (int kb = 0; kb < KB; ++kb) dst[int64_t(kb) * 128] = __ldg(src + kb);
     }
 }
 

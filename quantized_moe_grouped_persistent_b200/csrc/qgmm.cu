@@ -144,9 +144,46 @@ DetLayout det_layout(const qgmm_problem *p)
     return L;
 }
 
+// MxA8W4: the scale atoms the MX kernel's producer bulk-copies (mx_sf_atoms_*_kernel),
+// after the mode's own workspace: x1's for every m-tile of the walk (at most
+// ceil(m/128) + e) and k-block, the weights' for every expert, 128-column tile and
+// k-block; 512 bytes each.
+struct MxAtoms {
+    size_t rows, cols, total;
+};
+
+MxAtoms mx_atoms(const qgmm_problem *p)
+{
+    MxAtoms A;
+    const size_t kb = size_t(p->k / BK);
+    A.rows = p->deterministic ? det_layout(p).total : kAlign;
+    A.cols = A.rows + align_up((size_t((p->m + BM - 1) / BM) + size_t(p->e)) * kb * MX_SF_BYTES);
+    A.total = A.cols + align_up(size_t(p->e) * size_t(p->n / MX_BN) * kb * MX_SF_BYTES);
+    return A;
+}
+
 size_t workspace_bytes(const qgmm_problem *p)
 {
+    if (p->weight_type == QGMM_W_MXFP4) return mx_atoms(p).total;
     return p->deterministic ? det_layout(p).total : kAlign;
+}
+
+// Write the MX kernel's scale atoms into the workspace (two kernels on `st`).
+qgmm_status mx_write_atoms(const qgmm_problem *p, const DeviceInfo *dev, const uint8_t *sfa, const uint8_t *sfb,
+                           const int64_t *group_list, uint8_t *ws, cudaStream_t st)
+{
+    const MxAtoms A = mx_atoms(p);
+    const int64_t mt_max = (p->m + BM - 1) / BM + p->e;
+    const int grid_rows = static_cast<int>(mt_max < 4 * int64_t(dev->sms) ? mt_max : 4 * int64_t(dev->sms));
+    mx_sf_atoms_rows_kernel<<<grid_rows, 128, 0, st>>>(sfa, p->m, static_cast<int32_t>(p->k), group_list,
+                                                       static_cast<int>(p->e), p->group_list_type,
+                                                       reinterpret_cast<uint32_t *>(ws + A.rows));
+    const int64_t col_tiles = p->e * (p->n / MX_BN);
+    const int grid_cols = static_cast<int>(col_tiles < 8 * int64_t(dev->sms) ? col_tiles : 8 * int64_t(dev->sms));
+    mx_sf_atoms_cols_kernel<<<grid_cols, 128, 0, st>>>(sfb, static_cast<int>(p->e), static_cast<int32_t>(p->n),
+                                                       ld_sb(p), static_cast<int32_t>(p->k),
+                                                       reinterpret_cast<uint32_t *>(ws + A.cols));
+    return cudaGetLastError() == cudaSuccess ? QGMM_OK : QGMM_ERR_CUDA;
 }
 
 int env_int(const char *name, int dflt)
@@ -578,9 +615,15 @@ qgmm_status finalize_impl(const qgmm_problem *p, const int8_t *x1, const void *x
     GemmArgs a = base_args(p, group_list, pl, status);
     if (mx) {
         // MxA8W4: scale and pertoken_scale hold the E8M0 block scales of the weights
-        // and of x1; the epilogue's own scale and pertokenScale are then 1
-        a.sfb = static_cast<const uint8_t *>(scale);
-        a.sfa = reinterpret_cast<const uint8_t *>(pertoken_scale);
+        // and of x1; the epilogue's own scale and pertokenScale are then 1.  The MX
+        // kernel reads them as per-stage atoms written into the workspace first.
+        if ((s = mx_write_atoms(p, dev, reinterpret_cast<const uint8_t *>(pertoken_scale),
+                                static_cast<const uint8_t *>(scale), group_list, static_cast<uint8_t *>(workspace),
+                                st)) != QGMM_OK)
+            return s;
+        const MxAtoms A = mx_atoms(p);
+        a.sfa = static_cast<const uint8_t *>(workspace) + A.rows;
+        a.sfb = static_cast<const uint8_t *>(workspace) + A.cols;
     } else {
         a.scale = scale;
         a.scale_bf16 = p->scale_type == QGMM_SCALE_BF16;
@@ -682,8 +725,9 @@ QGMM_API qgmm_status qgmm_finalize_launches(const qgmm_problem *p, int32_t *laun
     DeviceInfo *dev = nullptr;
     if ((s = device_info(&dev)) != QGMM_OK) return s;
     const Plan pl = make_plan(p, dev->sms, p->deterministic ? EPI_STORE_Y : EPI_ATOMIC);
-    // atomic: output init; deterministic: clear, histogram, column scan, scan, fill, then the reduce
-    *launches = (p->deterministic ? 6 : 1) + gemm_launches(pl);
+    // atomic: output init; deterministic: clear, histogram, column scan, scan, fill, then the reduce;
+    // MxA8W4 also writes its two kinds of scale atoms first
+    *launches = (p->deterministic ? 6 : 1) + gemm_launches(pl) + (p->weight_type == QGMM_W_MXFP4 ? 2 : 0);
     return QGMM_OK;
 }
 
@@ -744,7 +788,7 @@ QGMM_API qgmm_status qgmm_debug_accum_mx(const qgmm_problem *p, const uint8_t *x
     if (!aligned16(x1) || !aligned32(x2) || !aligned16(acc_out) || !aligned16(sfa) || !aligned16(sfb) ||
         (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
         return QGMM_ERR_ALIGNMENT;
-    if (ws_bytes < kAlign) return QGMM_ERR_WORKSPACE_TOO_SMALL;
+    if (ws_bytes < workspace_bytes(p)) return QGMM_ERR_WORKSPACE_TOO_SMALL;
     DeviceInfo *dev = nullptr;
     if ((s = device_info(&dev)) != QGMM_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
@@ -753,12 +797,14 @@ QGMM_API qgmm_status qgmm_debug_accum_mx(const qgmm_problem *p, const uint8_t *x
     CUtensorMap ma, mb;
     if ((s = make_maps(p, reinterpret_cast<const int8_t *>(x1), x2, pl.tile_rows, 32, &ma, &mb)) != QGMM_OK)
         return s;
+    if ((s = mx_write_atoms(p, dev, sfa, sfb, group_list, static_cast<uint8_t *>(workspace), st)) != QGMM_OK) return s;
     clear_status_kernel<<<1, 1, 0, st>>>(status);
     if (cudaGetLastError() != cudaSuccess) return QGMM_ERR_CUDA;
     GemmArgs a = base_args(p, group_list, pl, status);
     a.acc_out = reinterpret_cast<int32_t *>(acc_out);
-    a.sfa = sfa;
-    a.sfb = sfb;
+    const MxAtoms A = mx_atoms(p);
+    a.sfa = static_cast<const uint8_t *>(workspace) + A.rows;
+    a.sfb = static_cast<const uint8_t *>(workspace) + A.cols;
     return launch_gemm(EPI_RAW_ACC, dev, p, pl, ma, mb, mb, a, st);
 }
 
