@@ -8,7 +8,8 @@
 - The oracle's two dequant modes on hand-worked rows: pertensor (acc * weight
   scale) * the row's source-card scale, and mx with one 32-block.
 - ``qgmm_ep_plan`` (C ABI, a host call) against the same example, against a
-  brute force over random counts, and on its limits (page 2: e <= 32,
+  placement of every chunk compared with the oracle's dispatch over random counts
+  (also property-based over drawn domains), and on its limits (page 2: e <= 32,
   e * epWorldSize <= 256, 0 < BSK < 52428800, no negative count).
 - The exchange over gloo with 2 and 3 ranks (random counts, empty chunks, a card
   that receives nothing): every rank's permuted rows and scales equal the
@@ -267,3 +268,39 @@ def test_gloo_exchange_rejects_mismatched_counts():
     res = _run_ranks(2, 2, 23, mode="mismatch")
     assert all(r[1] == "raised" for r in res)
     assert all("expects other counts" in r[2] for r in res)
+
+
+def test_ep_plan_against_the_oracle_over_drawn_domains(qgmm):
+    """Hypothesis: drawn domains (1-8 cards, 1-32 experts per card, at most 256 in all,
+    chunk counts 0-6 with empty cards allowed on the receive side): every card's plan
+    places each chunk where the oracle's dispatch puts its rows."""
+    hyp = pytest.importorskip("hypothesis")
+    st = pytest.importorskip("hypothesis.strategies")
+    from oracle import ep
+
+    @hyp.settings(max_examples=60, deadline=None, derandomize=True)
+    @hyp.given(st.integers(1, 8), st.integers(1, 32), st.integers(0, 2 ** 31 - 1))
+    def check(world, e, seed):
+        hyp.assume(world * e <= 256)
+        rng = np.random.default_rng(seed)
+        counts = [rng.integers(0, 7, world * e) for _ in range(world)]
+        for c in counts:
+            c[rng.integers(0, world * e)] += 1                 # BSK >= 1 on every card
+        bufs = [_col(np.arange(int(c.sum())) + 100000 * s) for s, c in enumerate(counts)]
+        want = ep.dispatch(bufs, counts, e)
+        plans = [qgmm.ep_plan(world, e, counts[r],
+                              np.array([counts[s][r * e + j] for s in range(world) for j in range(e)]))
+                 for r in range(world)]
+        for r in range(world):
+            rows = np.full(plans[r]["a"], -1, np.int64)
+            for s in range(world):
+                for j in range(e):
+                    cnt = int(counts[s][r * e + j])
+                    so = int(plans[s]["send_offsets"][r * e + j])
+                    ro = int(plans[r]["recv_offsets"][s * e + j])
+                    rows[ro:ro + cnt] = bufs[s][so:so + cnt, 0]
+            np.testing.assert_array_equal(rows, want[r][0][:, 0])
+            np.testing.assert_array_equal(plans[r]["group_counts"], want[r][1])
+            assert plans[r]["bsk"] == int(counts[r].sum())
+
+    check()
