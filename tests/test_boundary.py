@@ -111,6 +111,21 @@ def test_workspace_sizes(qgmm):
         assert got == 256 + al(m * nn * 4) + al(segs * obs * 4) + al((obs + 1) * 4) + al(m * 4), (m, obs)
 
 
+def test_workspace_sizes_mx(qgmm):
+    """QGMM_W_MXFP4 adds its scale atoms after the mode's own part: (ceil(m/128) + e) * (k/128)
+    atoms for x1 and e * (n/128) * (k/128) for the weights, 512 bytes each, each part rounded
+    up to 256 bytes (the formula qgmm.h gives)."""
+    al = lambda v: (v + 255) // 256 * 256
+    for m, k, n, e, obs in ((32768, 2048, 7168, 128, 4096), (100, 256, 256, 3, 100), (1, 128, 256, 1, 1)):
+        atoms = al(((m + 127) // 128 + e) * (k // 128) * 512) + al(e * (n // 128) * (k // 128) * 512)
+        p = _prob(qgmm, m=m, k=k, n=n, e=e, output_bs=obs, weight_type=qgmm.QGMM_W_MXFP4, transpose_x2=True)
+        assert qgmm.finalize_workspace(p) == 256 + atoms, (m, k, n, e)
+        pd = _prob(qgmm, m=m, k=k, n=n, e=e, output_bs=obs, weight_type=qgmm.QGMM_W_MXFP4, transpose_x2=True,
+                   deterministic=True)
+        base = qgmm.finalize_workspace(_prob(qgmm, m=m, k=k, n=n, e=e, output_bs=obs, deterministic=True))
+        assert qgmm.finalize_workspace(pd) == base + atoms, (m, k, n, e)
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(m=0), "SHAPE"), (dict(m=(1 << 24) + 1), "SHAPE"),
     (dict(k=100), "SHAPE"), (dict(k=64), "SHAPE"), (dict(k=65536 + 128), "SHAPE"),
